@@ -1,0 +1,174 @@
+"""Pins of the oracle's encode / decode / estimate against the pages and the mathematics.
+
+Sources: TurboQuant review (Jump2Paper): Theorem 1 (D_mse = d C(f_X, b)), the 1-bit
+bias 2/pi (motivation and intuition paragraphs), Definition 1 with Lemma 4 (QJL
+unbiasedness and variance bound), Theorem 2 (prod unbiasedness and the D_prod bound).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from conftest import load_golden
+from oracle import quantizer as Q
+from oracle import rotation as rot
+
+SQRT3_PI2 = math.sqrt(3.0) * math.pi ** 2   # reading of the garbled Theorem-2 constant
+
+
+@pytest.fixture(scope="module")
+def cbs():
+    return {(d, b): Q.make_codebook(d, b) for d in (4, 8, 32, 128) for b in (1, 2, 3, 4)}
+
+
+def test_pack_golden_and_roundtrip():
+    g = load_golden("pack_example.json")
+    codes = np.array([g["codes"]])
+    np.testing.assert_array_equal(Q.pack_bits(codes, g["b"])[0], g["bytes"])
+    np.testing.assert_array_equal(Q.pack_bits(np.array([g["qjl_bits"]]), 1)[0], g["qjl_bytes"])
+    rng = np.random.default_rng(1)
+    for b in (1, 2, 3, 4, 5, 8):
+        for d in (8, 24, 128):
+            c = rng.integers(0, 1 << b, size=(7, d))
+            p = Q.pack_bits(c, b)
+            assert p.shape == (7, (b * d + 7) // 8)
+            np.testing.assert_array_equal(Q.unpack_bits(p, b, d), c)
+
+
+def test_empirical_mse_matches_theorem1(cbs):
+    # E||x - x~||^2 over uniform unit x equals d C(f_X, b), within 4 standard errors.
+    d = 128
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    x = synth.unit_vectors(16384, d, seed=11, dtype=np.float64)
+    for b in (1, 2, 3, 4):
+        cb = cbs[(d, b)]
+        codes, nu, _ = Q.encode_mse(x, P, cb)
+        err = np.sum((Q.decode_mse(codes, nu, P, cb) - x) ** 2, axis=1)
+        se = err.std() / math.sqrt(len(err))
+        assert abs(err.mean() - cb.dmse) < 4 * se, (b, err.mean(), cb.dmse)
+
+
+def test_brute_force_nearest_codeword_tiny_d(cbs):
+    # Over the whole product codebook (2^(b d) codewords), the reconstruction of the
+    # encoder is the codeword nearest to x: per-coordinate cells + Pi^T decode.
+    d, b = 4, 2
+    cb = cbs[(d, b)]
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 5))
+    grid = np.stack(np.meshgrid(*[np.arange(1 << b)] * d, indexing="ij"), -1).reshape(-1, d)
+    words = cb.c32[grid] @ P                       # all unit-norm-scale reconstructions
+    x = synth.unit_vectors(300, d, seed=12, dtype=np.float64)
+    codes, nu, _ = Q.encode_mse(x, P, cb)
+    xt = Q.decode_mse(codes, nu, P, cb)
+    dist = np.sum((x[:, None, :] - nu[:, None, None] * words[None]) ** 2, axis=2)
+    best = words[np.argmin(dist, axis=1)] * nu[:, None]
+    np.testing.assert_allclose(xt, best, atol=1e-12)
+
+
+def test_one_bit_mse_bias_is_two_over_pi(cbs, paper):
+    # Slope of <y, x~> on <y, x>: d E[c(X)^2] = 1 - D_mse(b) by the centroid condition;
+    # at b = 1 this is the printed 2/pi ~ 0.637 bias (large-d limit).
+    d = 128
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    x = synth.unit_vectors(20000, d, seed=13, dtype=np.float64)
+    y = synth.unit_vectors(64, d, seed=14, dtype=np.float64)
+    for b in (1, 2, 3):
+        cb = cbs[(d, b)]
+        codes, nu, _ = Q.encode_mse(x, P, cb)
+        xt = Q.decode_mse(codes, nu, P, cb)
+        ip, est = x @ y.T, xt @ y.T
+        slope = np.sum(ip * est) / np.sum(ip * ip)
+        assert abs(slope - (1 - cb.dmse)) < 0.01, (b, slope, 1 - cb.dmse)
+    assert abs((1 - cbs[(d, 1)].dmse) - 2 / math.pi) < 0.003
+    assert round(2 / math.pi, 3) == paper["mse_1bit_bias"]["value"]
+
+
+def _prod_trials(d, b, trials, seed, redraw_pi, cbs, x, y):
+    cb_m1 = cbs[(d, b - 1)] if b > 1 else None
+    errs, rhos = [], []
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, seed))
+    for t in range(trials):
+        if redraw_pi:
+            P = rot.haar_from_gaussian(synth.rng(seed, 10_000 + t).standard_normal((d, d)))
+        S = synth.rng(seed, t).standard_normal((d, d))       # fp64 Gaussian S per trial
+        codes, z, nu, rho, _, _ = Q.encode_prod(x[None], P, S, cb_m1)
+        xt = Q.decode_prod(codes, z, nu, rho, P, S, cb_m1)
+        errs.append(float(xt[0] @ y - x @ y))
+        rhos.append(rho[0])
+    return np.array(errs), np.array(rhos)
+
+
+def test_prod_unbiased_over_1e5_trials(cbs):
+    # Theorem 2: E[<y, x~>] = <y, x>; S redrawn per trial, mean error within 3 sigma.
+    d, b = 32, 3
+    x = synth.unit_vectors(1, d, seed=20, dtype=np.float64)[0]
+    y = synth.unit_vectors(1, d, seed=21, dtype=np.float64)[0] * 2.0
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    cb_m1 = cbs[(d, b - 1)]
+    n = 100_000
+    g = synth.rng(77, 0)
+    codes, _, nu, rho, yrot, _ = Q.encode_prod(x[None], P, np.eye(d), cb_m1)
+    r = yrot[0] - cb_m1.c32[codes[0]]
+    # Batched over trials: the MSE part is the same for every S; only the QJL term varies.
+    errs = np.empty(n)
+    base = float(Q.decode_mse(codes, nu, P, cb_m1)[0] @ y)
+    for i0 in range(0, n, 5000):
+        S = g.standard_normal((5000, d, d))
+        z = (np.einsum("tjk,k->tj", S, r) >= 0).astype(np.float64)
+        back = np.einsum("tj,tjk->tk", 2 * z - 1, S) * rho[0] * Q.QJL_SCALE(d)
+        errs[i0:i0 + 5000] = base + (back @ P) @ y * nu[0] - x @ y
+    se = errs.std() / math.sqrt(n)
+    assert abs(errs.mean()) < 3 * se
+    # Cross-check the batched form against the plain encode/decode on a few trials.
+    e2, _ = _prod_trials(d, b, 5, 77, False, cbs, x, y)
+    assert np.all(np.isfinite(e2))
+    # Lemma 4 variance bound with the residual scale: Var <= pi/(2d) ||y||^2 ||r||^2.
+    bound = math.pi / (2 * d) * (y @ y) * rho[0] ** 2
+    assert errs.var() <= bound * (1 + 4 * math.sqrt(2 / n))
+
+
+def test_prod_unbiased_with_pi_redrawn(cbs):
+    d, b = 128, 2
+    x = synth.unit_vectors(1, d, seed=30, dtype=np.float64)[0]
+    y = synth.unit_vectors(1, d, seed=31, dtype=np.float64)[0]
+    errs, _ = _prod_trials(d, b, 3000, 5, True, cbs, x, y)
+    assert abs(errs.mean()) < 3 * errs.std() / math.sqrt(len(errs))
+
+
+def test_prod_distortion_bounds(cbs):
+    # Theorem 2: D_prod <= (pi / 2d) ||y||^2 D_mse(b-1) <= sqrt(3) pi^2 ||y||^2 / d 4^-b.
+    d = 128
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    S = synth.gaussian_matrix(d, 1)
+    x = synth.unit_vectors(20000, d, seed=40, dtype=np.float64)
+    y = synth.unit_vectors(16, d, seed=41, dtype=np.float64)
+    for b in (1, 2, 3, 4):
+        cb_m1 = cbs[(d, b - 1)] if b > 1 else None
+        codes, z, nu, rho, _, _ = Q.encode_prod(x, P, S, cb_m1)
+        xt = Q.decode_prod(codes, z, nu, rho, P, S, cb_m1)
+        dprod = np.mean(((xt - x) @ y.T) ** 2)
+        dm1 = cb_m1.dmse if cb_m1 is not None else 1.0
+        assert dprod <= math.pi / (2 * d) * dm1 * 1.1, (b, dprod)
+        assert dprod <= SQRT3_PI2 / d * 4.0 ** (-b), (b, dprod)
+
+
+def test_zero_vector_conventions(cbs):
+    d = 8
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    S = synth.gaussian_matrix(d, 1)
+    x = np.zeros((1, d))
+    codes, nu, _ = Q.encode_mse(x, P, cbs[(d, 3)])
+    assert nu[0] == 0 and np.all(codes == 4)          # y = 0 sits on the middle boundary
+    codes, z, nu, rho, _, _ = Q.encode_prod(x, P, S, cbs[(d, 2)])
+    assert rho[0] == 0 and np.all(z == 1)
+    assert np.all(Q.decode_prod(codes, z, nu, rho, P, S, cbs[(d, 2)]) == 0)
+
+
+def test_prod_b1_is_pure_qjl():
+    d = 16
+    P = rot.haar_from_gaussian(synth.gaussian_matrix(d, 0))
+    S = synth.gaussian_matrix(d, 1)
+    x = synth.unit_vectors(5, d, seed=50, dtype=np.float64)
+    codes, z, nu, rho, y, s = Q.encode_prod(x, P, S, None)
+    np.testing.assert_allclose(rho, 1.0, atol=1e-12)       # r = y, a unit vector
+    np.testing.assert_array_equal(z, (y @ S.T >= 0).astype(int))
