@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Benchmark: TurboQuant_prod prefill encode of a KV-cache key batch plus decode scoring.
+
+One step = the hot path over one batch:
+  1. tq_quantize_prod of keys [1 batch, 32 heads, 32768 tokens, d=128] bf16
+     (b = 3: 2-bit Lloyd-Max codes + 1-bit QJL, randomized Hadamard rotation, S bf16);
+  2. tq_score of one bf16 decode query per head against that head's 32768 compressed keys.
+Metric: quantize Mvec/s & score Gkeys/s (d=128, b=3); value = vectors that went through
+the whole step per second over all ranks, in Mvec/s. Per-kernel rates and the HBM
+roofline of the dominant kernel (the encoder) are reported beside it.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+For N > 1 launch with torchrun (one rank per GPU); each rank quantizes its own batch
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "quantize Mvec/s & score Gkeys/s (d=128, b=3); % of HBM roofline"
+HEADS, TOKENS, D, BITS = 32, 32768, 128, 3
+N_VEC = HEADS * TOKENS
+# Algorithmic bytes per vector of the encoder: 256 B bf16 in; 32 B codes + 16 B QJL +
+# 4 B norm + 4 B residual norm out.
+ENC_BYTES_PER_VEC = 2 * D + (BITS - 1) * D // 8 + D // 8 + 8
+# Per key of the scorer: 32 B codes + 16 B QJL + 8 B norms in, 4 B score out.
+SCORE_BYTES_PER_KEY = (BITS - 1) * D // 8 + D // 8 + 8 + 4
+WORKLOAD = "turboquant_prod b=3 RHT prefill encode of KV keys [1,32,32768,128] bf16 + one decode query per head scored"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def stored_traffic(kernel_key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        ent = t.get(kernel_key)
+        if not ent:
+            return None
+        import hashlib
+        src = os.path.join(ROOT, ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != ent["source_sha"]:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [s.strip() for s in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(heads: int, seed: int):
+    """The oracle (fp64 numpy) on `heads` heads of the workload; returns (vectors, seconds, threads)."""
+    from oracle import quantizer as OQ
+    from oracle import rotation as OR
+    eps = synth.rht_signs(D)
+    S = OR.round_bf16(synth.gaussian_matrix(D, synth.SEED_S))
+    Pi = OR.rht_matrix(eps)
+    cb = OQ.make_codebook(D, BITS - 1)
+    qv = synth.bf16_from_bits(synth.decode_queries(HEADS, D))
+    data = [synth.bf16_from_bits(synth.kv_prefill_batch(HEADS, TOKENS, D, seed=seed, head_range=(h, h + 1))[0])
+            for h in range(heads)]
+    t0 = time.perf_counter()
+    for h in range(heads):
+        codes, z, nu, rho, _, _ = OQ.encode_prod(data[h], Pi, S, cb)
+        OQ.pack_bits(codes, BITS - 1)
+        OQ.pack_bits(z, 1)
+        xt = OQ.decode_prod(codes, z, nu, rho, Pi, S, cb)
+        OQ.estimate(qv[h:h + 1], xt)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    return heads * TOKENS, dt, threads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    heads = 4
+    for _ in range(args.warmup):
+        oracle_sample(heads, synth.SEED_DATA)
+    times, threads = [], 1
+    for _ in range(args.steps):
+        n, dt, threads = oracle_sample(heads, synth.SEED_DATA)
+        times.append(dt)
+    tot = sum(times)
+    value = heads * TOKENS * args.steps / tot / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mvec/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": f"{heads} of {HEADS} heads per step ({heads * TOKENS} vectors)"},
+        "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{heads} heads x {TOKENS} tokens per step, fp64 numpy oracle"},
+        "e2e": {"value": value, "unit": "Mvec/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=HEADS, help="smaller batch for profiling runs")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import vector_quantization_tq_b200 as tq
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    heads = args.heads
+    nvec = heads * TOKENS
+
+    # state: prod b=3, RHT signs (seed 0), S ~ N(0,1) stored bf16 (seed 1)
+    st = tq.State(D, BITS, tq.PROD, tq.ROT_RHT, tq.BF16, device=local, signs=synth.rht_signs(D),
+                  s=synth.gaussian_matrix(D, synth.SEED_S))
+    # each rank its own batch (weak scaling)
+    seed = synth.SEED_DATA + 100 * rank
+    kbits = synth.kv_prefill_batch(HEADS, TOKENS, D, seed=seed, head_range=(0, heads)).reshape(nvec, D)
+    qbits = synth.decode_queries(HEADS, D)[:heads]
+    x = torch.from_numpy(kbits.view(np.int16)).to(dev).view(torch.bfloat16)
+    q = torch.from_numpy(qbits.view(np.int16)).to(dev).view(torch.bfloat16)
+    codes, qjl, norms, rnorms = st.empty_planes(nvec, dev)
+    scores = torch.empty((heads, 1, TOKENS), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
+        tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
+            ev[i][1].record(stream)
+            tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+            ev[i][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    enc_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    sc_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    step_ms = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([step_ms, enc_ms, sc_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, enc_ms, sc_ms = [float(v) for v in t.tolist()]
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hx = x.cpu().pin_memory()
+        hq = q.cpu().pin_memory()
+        hc = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+        hz = torch.empty(qjl.shape, dtype=qjl.dtype).pin_memory()
+        hn = torch.empty(norms.shape, dtype=norms.dtype).pin_memory()
+        hr = torch.empty(rnorms.shape, dtype=rnorms.dtype).pin_memory()
+        hs = torch.empty(scores.shape, dtype=scores.dtype).pin_memory()
+        dx = torch.empty_like(x)
+        dq = torch.empty_like(q)
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            tq.quantize_prod(st, dx, codes, qjl, norms, rnorms, stream=stream)
+            tq.score(st, dq, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+            hc.copy_(codes, non_blocking=True)
+            hz.copy_(qjl, non_blocking=True)
+            hn.copy_(norms, non_blocking=True)
+            hr.copy_(rnorms, non_blocking=True)
+            hs.copy_(scores, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        ne2e = max(3, args.steps // 2)
+        for _ in range(ne2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = s0.elapsed_time(s1) / ne2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = hx.numel() * hx.element_size() + hq.numel() * hq.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in (hc, hz, hn, hr, hs))
+        e2e = {"value": nvec * world / (e2e_ms / 1e3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_s, dt, threads = oracle_sample(8, seed)
+        cpu = {"value": n_s / dt / 1e6, "unit": "Mvec/s", "cores": threads, "kind": "oracle",
+               "sample": f"8 of 32 heads ({n_s} vectors) of the same batch: fp64 numpy encode + pack + decode + "
+                         f"estimate, {dt:.2f} s wall"}
+
+    peak, peak_kind = measured_peaks()
+    enc_gbs = ENC_BYTES_PER_VEC * nvec / (enc_ms / 1e3) / 1e9
+    sc_gbs = SCORE_BYTES_PER_KEY * nvec / (sc_ms / 1e3) / 1e9
+    traffic = stored_traffic("encode_prod_d128")
+    line = {
+        "metric": METRIC,
+        "value": nvec * world / (step_ms / 1e3) / 1e6,
+        "unit": "Mvec/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "vectors_per_rank": nvec, "heads": heads, "tokens": TOKENS, "d": D,
+                   "b": BITS, "mode": "prod", "rotation": "rht", "matrix_dtype": "bf16",
+                   "l2": "inputs larger than L2 (256 MiB of bf16 keys per step per rank)",
+                   "parallelism": f"dp{world} (independent batches)"},
+        "quantize_mvec_s": nvec * world / (enc_ms / 1e3) / 1e6,
+        "score_gkeys_s": nvec * world / (sc_ms / 1e3) / 1e9,
+        "kernels_ms": {"encode": enc_ms, "score": sc_ms},
+        "roofline": {"bound": "hbm", "achieved": enc_gbs, "peak": peak, "unit": "GB/s", "frac": enc_gbs / peak,
+                     "traffic": traffic, "kernel": "encode (tq_quantize_prod)",
+                     "algorithmic_bytes_per_launch": ENC_BYTES_PER_VEC * nvec, "peak_kind": peak_kind},
+        "score_roofline": {"bound": "hbm", "achieved": sc_gbs, "peak": peak, "unit": "GB/s", "frac": sc_gbs / peak},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    st.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

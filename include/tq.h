@@ -1,0 +1,230 @@
+/*
+ * tq.h - C ABI of libtq: TurboQuant-style online vector quantization on B200 (sm_100a).
+ *
+ * The operations follow the TurboQuant review (Jump2Paper, arXiv 2504.19874):
+ *   - Lemma 1 / Theorem 1 (MSE): a random rotation Pi makes every coordinate of a unit
+ *     vector follow f_X(x) ~ (1 - x^2)^((d-3)/2); each coordinate then gets a b-bit
+ *     Lloyd-Max code for f_X, and x~ = ||x|| Pi^T c[idx].
+ *   - Definition 1 (QJL) and Theorem 2 (prod): the prod quantizer keeps (b-1)-bit MSE
+ *     codes plus sign(S r) of the residual r and ||r||, S i.i.d. N(0,1) d x d; its
+ *     inner-product estimate is unbiased.
+ *   - Problem statement: Q maps R^d to B = b*d bits; Q^{-1} reconstructs.
+ * and the AI Trends summary of the TurboQuant video (chapter "L2 normalize + RHT
+ * matrix": store the norm, normalise, rotate by a randomized Hadamard transform whose
+ * inverse is its transpose).
+ *
+ * Conventions for every call:
+ *   - Every function returns an int status (TQ_OK = 0). Nothing is thrown across the ABI.
+ *     Arguments are validated before any launch; on an error nothing is launched and
+ *     no output is touched. tq_status_string() gives the text.
+ *   - Pointers named h_* are host pointers; every other buffer pointer is a device
+ *     pointer on the state's device. The caller owns all data buffers; the library owns
+ *     tq_state objects (free with tq_state_destroy).
+ *   - Device work is asynchronous on the given cudaStream_t (passed as void*; NULL is
+ *     the legacy default stream). Buffers must stay valid until the stream reaches it.
+ *   - A CUDA error seen at launch is returned as TQ_ECUDA; tq_last_cuda_error() gives
+ *     the cudaError_t value of the calling thread's last such error.
+ *   - Distinct states may be used from distinct threads. A state is read-only after
+ *     creation, so concurrent calls on one state are safe as long as their output
+ *     buffers and workspaces differ.
+ *
+ * Data layout (structure of arrays, n vectors):
+ *   codes   uint8 [n][code_bytes], code_bytes = ceil(b_mse * d / 8): each vector's
+ *           codes form one LSB-first bit stream, code j in bits [j*b_mse, j*b_mse+b_mse)
+ *           (bit i of byte k is stream bit 8k+i). b_mse = b (MSE) or b-1 (prod).
+ *   qjl     uint8 [n][d/8] (prod only): bit j = 1 iff (S r)_j >= 0.
+ *   norms   float [n]: ||x||.     rnorms  float [n] (prod only): ||r|| of the unit vector.
+ *   vectors fp32 or bf16 rows of d elements, row stride ld elements (ld >= d); rows must
+ *           start on 16-byte boundaries (ld*elem_size and the base pointer multiples of 16).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------- */
+#define TQ_OK            0
+#define TQ_EINVAL        1  /* a null pointer, size, stride, alignment or value is invalid */
+#define TQ_EUNSUPPORTED  2  /* valid but not supported here (e.g. RHT with d not a power of 2) */
+#define TQ_ENOMEM        3  /* host or device allocation failed, or a workspace is too small */
+#define TQ_ECUDA         4  /* the CUDA runtime returned an error */
+#define TQ_EDEVICE       5  /* a kernel reported an error through its status word */
+
+/* ---- enums --------------------------------------------------------------------------- */
+#define TQ_MSE        0     /* TurboQuant_mse: b-bit codes + ||x||                          */
+#define TQ_PROD       1     /* TurboQuant_prod: (b-1)-bit codes + QJL signs + ||x|| + ||r|| */
+#define TQ_ROT_DENSE  0     /* Pi = Haar-random orthogonal matrix (QR of a Gaussian matrix)  */
+#define TQ_ROT_RHT    1     /* Pi = H_d diag(eps) / sqrt(d), Sylvester Hadamard H_d          */
+#define TQ_F32        0
+#define TQ_BF16       1
+
+/*
+ * Host utilities (no device work): the draws and the rotation that tq_state_create uses
+ * when it is given no draws, so that a caller can reproduce or inspect them.
+ *   tq_draw_gaussian  count N(0,1) draws of Philox4x32-10 keyed by seed (Box-Muller).
+ *   tq_draw_signs     count signs (+1/-1) of Philox4x32-10 keyed by seed.
+ *   tq_haar_rotation  Pi = Q diag(sign(diag R)) from the Householder QR of the row-major
+ *                     d x d matrix h_g, in fp64 (before any rounding to mat_dtype).
+ * Errors: TQ_EINVAL for NULL pointers, d < 2, or a singular h_g.
+ */
+int tq_draw_gaussian(uint64_t seed, size_t count, double* h_out);
+int tq_draw_signs(uint64_t seed, size_t count, int8_t* h_out);
+int tq_haar_rotation(int d, const double* h_g, double* h_pi);
+
+/* Which host copy tq_state_copy() returns. */
+#define TQ_FIELD_CENTROIDS 0  /* 2^b_mse fp64 centroids (ascending)                */
+#define TQ_FIELD_BOUNDS    1  /* 2^b_mse - 1 fp64 boundaries                       */
+#define TQ_FIELD_PI        2  /* d*d row-major Pi, the values stored on the device */
+#define TQ_FIELD_SIGNS     3  /* d RHT signs (+1/-1)                               */
+#define TQ_FIELD_S         4  /* d*d row-major S, the values stored on the device  */
+
+typedef struct tq_params {
+    int32_t d;          /* dimension, 2 <= d; kernels: d in {32,64,128,256,512,1024,1536,2048} */
+    int32_t b;          /* bits per coordinate: MSE 1..8, prod 1..9 (prod b=1 is pure QJL)    */
+    int32_t mode;       /* TQ_MSE or TQ_PROD                                                  */
+    int32_t rot;        /* TQ_ROT_DENSE or TQ_ROT_RHT (d a power of two)                       */
+    int32_t mat_dtype;  /* device storage of dense Pi and of S: TQ_F32 or TQ_BF16              */
+    int32_t device;     /* CUDA device ordinal that holds the state                           */
+    uint64_t seed_pi;   /* Philox key used when no rotation draws are supplied                 */
+    uint64_t seed_s;    /* Philox key used when S is not supplied                              */
+} tq_params;
+
+typedef struct tq_state tq_state;
+
+/* Text of a status code (static string, never NULL). */
+const char* tq_status_string(int status);
+
+/* cudaError_t value of the calling thread's last TQ_ECUDA (0 if none). */
+int tq_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int tq_version(void);
+
+/*
+ * Lloyd-Max codebook of the Lemma-1 law f_X for dimension d and b bits (host only, fp64).
+ * Jump2Paper review, Theorem 1 (MSE): continuous 1-D k-means on f_X; the optimal MSE is
+ * D_mse = d * C(f_X, b). Writes 2^b centroids (ascending; antisymmetric about 0), 2^b-1
+ * boundaries (midpoints) and D_mse. Any output pointer may be NULL.
+ * Errors: TQ_EINVAL if d < 2 or b outside 1..8.
+ */
+int tq_build_codebook(int d, int b, double* h_centroids, double* h_bounds, double* h_dmse);
+
+/*
+ * Create a state: codebook, rotation, and (prod) the QJL matrix S, copied to the device.
+ *   h_gauss_pi  TQ_ROT_DENSE: d*d row-major N(0,1) draws G; Pi = Q diag(sign(diag R)) from
+ *               the Householder QR of G (Jump2Paper: the paper's rotation is a QR rotation).
+ *               NULL: G is drawn from Philox4x32-10 keyed by seed_pi (Box-Muller).
+ *   h_signs     TQ_ROT_RHT: d signs (+1/-1). NULL: drawn from Philox keyed by seed_pi.
+ *   h_s         TQ_PROD: d*d row-major S (Definition 1). NULL: drawn from Philox keyed by seed_s.
+ * Pi and S are rounded once to mat_dtype; those stored values define the transform.
+ * Pointers that the mode does not use are ignored. The state is owned by the caller and
+ * freed with tq_state_destroy().
+ * Errors: TQ_EINVAL (bad params / NULL out), TQ_EUNSUPPORTED (RHT with d not a power of 2,
+ * or d not supported by the kernels), TQ_ENOMEM, TQ_ECUDA.
+ */
+int tq_state_create(const tq_params* p, const double* h_gauss_pi, const int8_t* h_signs,
+                    const double* h_s, tq_state** out);
+
+/* Free a state and its device memory (NULL is allowed). */
+int tq_state_destroy(tq_state* st);
+
+/* Copy of the parameters the state was created with. */
+int tq_state_params(const tq_state* st, tq_params* out);
+
+/* Bits of MSE code per coordinate (b or b-1), and D_mse of that codebook. */
+int tq_state_codebook_info(const tq_state* st, int* b_mse, double* dmse);
+
+/* Host copy of one field as fp64 (see TQ_FIELD_*). `count` is the capacity of h_out in
+ * elements; TQ_EINVAL if it is smaller than the field or the field is absent. */
+int tq_state_copy(const tq_state* st, int field, double* h_out, size_t count);
+
+/* Serialise a state into h_buf (checkpoint). With h_buf NULL, *bytes receives the size.
+ * Errors: TQ_ENOMEM if *bytes is smaller than needed (then *bytes is set to the size). */
+int tq_state_export(const tq_state* st, void* h_buf, size_t* bytes);
+
+/* Rebuild a state from tq_state_export() output on `device` (-1: the exported device). */
+int tq_state_import(const void* h_buf, size_t bytes, int device, tq_state** out);
+
+/* Per-vector plane widths in bytes: codes (ceil(b_mse*d/8)) and qjl (d/8 or 0). */
+int tq_code_layout(const tq_state* st, size_t* code_bytes, size_t* qjl_bytes);
+
+/*
+ * TurboQuant_mse encode of n vectors x (dtype TQ_F32 / TQ_BF16, row stride ld elements):
+ * norms[i] = ||x_i||, y = Pi x_i / ||x_i||, codes = b-bit Lloyd-Max cell of each y_j
+ * (the upper cell on a tie), packed as in the layout above. The state must be TQ_MSE.
+ * n = 0 is a no-op. Errors: TQ_EINVAL, TQ_ECUDA.
+ */
+int tq_quantize_mse(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
+                    uint8_t* codes, float* norms, void* stream);
+
+/*
+ * TurboQuant_prod encode (Jump2Paper, Theorem 2): (b-1)-bit MSE codes of y = Pi x/||x||,
+ * residual r = y - c[idx] (rotated domain), rnorms[i] = ||r||, qjl bits of sign(S r).
+ * The state must be TQ_PROD. A zero vector stores norm 0, the codes of y = 0, r = 0.
+ */
+int tq_quantize_prod(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
+                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+
+/*
+ * Reconstruction Q^{-1}: out[i] = ||x|| Pi^T (c[idx] + ||r|| sqrt(pi/2)/d S^T (2z - 1))
+ * (the QJL term only for prod; qjl and rnorms are ignored for MSE and may be NULL).
+ * out is fp32 [n][d], row stride d.
+ */
+int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl,
+               const float* norms, const float* rnorms, int64_t n, float* out, void* stream);
+
+/*
+ * Inner-product estimates <q, x~> straight from the packed codes, grouped:
+ *   queries q [groups][nq][d] (dtype TQ_F32/TQ_BF16, contiguous rows),
+ *   keys (codes/qjl/norms/rnorms) [groups][n],
+ *   scores fp32 [groups][nq][n]: scores[g][i][k] = <q[g][i], x~[g][k]>.
+ * Computed through the rotated query q' = Pi q and u = S q':
+ *   <q, x~> = ||x|| ( sum_j q'_j c[idx_j] + ||r|| sqrt(pi/2)/d sum_j u_j (2 z_j - 1) ).
+ * groups = 1 is plain all-pairs scoring; groups = heads with nq = 1 is one decode query
+ * per head against that head's keys.
+ */
+int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int64_t nq,
+             const uint8_t* codes, const uint8_t* qjl, const float* norms, const float* rnorms,
+             int64_t n, float* scores, void* stream);
+
+/* Workspace bytes that tq_attend_decode needs for H heads and T tokens. */
+int tq_attend_workspace(const tq_state* ks, const tq_state* vs, int H, int64_t T, size_t* bytes);
+
+/*
+ * One decode step of attention over a compressed cache (per head h, T tokens):
+ *   s_t = scale * <q_h, k~_t>,  p = softmax(s),  out_h = sum_t p_t v~_t.
+ * K is compressed by `ks` (MSE or prod), V by `vs` (MSE). Both states must have the same d.
+ * Planes are [H][T] (token-major within a head); q is [H][d] (TQ_F32/TQ_BF16); out fp32 [H][d].
+ * The value sum is accumulated in the rotated domain and Pi_V^T is applied once per head.
+ * workspace: device memory of at least tq_attend_workspace() bytes, 256-byte aligned.
+ * Errors: TQ_ENOMEM if ws_bytes is too small.
+ */
+int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H,
+                     int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                     const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                     float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes that tq_search_topk needs. */
+int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes);
+
+/*
+ * Top-k database vectors by estimated inner product for each of nq queries
+ * (Jump2Paper: nearest-neighbour search over compressed vectors). Planes as tq_score with
+ * groups = 1. idx int64 [nq][k] and vals fp32 [nq][k], best first; ties to the lower index.
+ * 1 <= k <= 64 and k <= n.
+ */
+int tq_search_topk(const tq_state* st, const void* q, int qdtype, int64_t nq,
+                   const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                   const float* rnorms, int64_t n, int k, int64_t* idx, float* vals,
+                   void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -1,0 +1,140 @@
+"""C-ABI tests that need no GPU: exports, host-side computations, validation paths.
+
+The host codebook builder and QR rotation of libtq are compared with the oracle (which
+is pinned to the pages separately); the Philox generator is pinned to the published
+known-answer vectors of Philox4x32-10.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+
+import synth
+import vector_quantization_tq_b200 as tq
+from oracle import codebook as ocb
+from oracle import rotation as orot
+
+
+def test_every_declared_symbol_is_exported():
+    names = tq.declared_symbols()
+    assert len(names) >= 23
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    lib = tq.lib()
+    for code in range(6):
+        assert lib.tq_status_string(code)
+    assert lib.tq_status_string(99) == b"unknown status"
+    assert lib.tq_version() >= 100
+
+
+@pytest.mark.parametrize("d", [3, 64, 128, 256, 1536])
+def test_codebook_matches_oracle(d):
+    for b in (1, 2, 3, 4):
+        c, t, D = tq.build_codebook(d, b)
+        oc, ot, oD, _ = ocb.lloyd_max(d, b)
+        np.testing.assert_allclose(c, oc, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(t, ot, atol=1e-12, rtol=0)
+        assert abs(D - oD) < 1e-11
+        assert t[len(t) // 2] == 0.0          # exactly antisymmetric
+
+
+def test_codebook_high_bits_fixed_point():
+    # b = 6 and 8: Lloyd-Max conditions hold (centroid = cell mean, boundary = midpoint).
+    for d, b in ((128, 6), (128, 8)):
+        c, t, D = tq.build_codebook(d, b)
+        edges = np.concatenate(([-1.0], t, [1.0]))
+        m0 = ocb.cdf(edges[1:], d) - ocb.cdf(edges[:-1], d)
+        m1 = ocb.first_moment(edges[:-1], edges[1:], d)
+        np.testing.assert_allclose(c, m1 / m0, atol=1e-12)
+        np.testing.assert_allclose(t, 0.5 * (c[1:] + c[:-1]), atol=0)
+        assert 4.0 ** -b <= D <= math.sqrt(3) * math.pi / 2 * 4.0 ** -b
+
+
+def test_codebook_rejects_bad_args():
+    lib = tq.lib()
+    assert lib.tq_build_codebook(1, 3, None, None, None) == 1
+    assert lib.tq_build_codebook(128, 0, None, None, None) == 1
+    assert lib.tq_build_codebook(128, 9, None, None, None) == 1
+
+
+def _uniform53(hi, lo):
+    v = ((hi >> 5) << 26) | (lo >> 6)
+    return (v + 1.0) / 9007199254740992.0
+
+
+def test_philox_known_answers_through_gaussian_draws():
+    # Philox4x32-10 known-answer vectors (Salmon et al., SC 2011, Random123 distribution):
+    #   key (0,0), counter (0,0,0,0) -> 6627e8d5 e169c58d bc57ac4c 9b00dbd8
+    #   key (ffffffff,ffffffff), counter all ffffffff -> 408f276d 41c83b0e a20bc7c6 6d5451fd
+    # Draws 0 and 1 of seed 0 are the Box-Muller pair of the first vector.
+    w = [0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8]
+    u1, u2 = _uniform53(w[0], w[1]), _uniform53(w[2], w[3])
+    r = math.sqrt(-2 * math.log(u1))
+    want = [r * math.cos(2 * math.pi * u2), r * math.sin(2 * math.pi * u2)]
+    got = tq.draw_gaussian(0, 2)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+
+
+def test_philox_streams_are_deterministic_and_keyed():
+    a = tq.draw_gaussian(2 ** 64 - 1, 8)
+    np.testing.assert_array_equal(a, tq.draw_gaussian(2 ** 64 - 1, 8))
+    assert not np.allclose(a, tq.draw_gaussian(0, 8))
+    # draw i of a longer stream equals draw i of a shorter one (counter-based)
+    np.testing.assert_array_equal(tq.draw_gaussian(5, 1001)[:999], tq.draw_gaussian(5, 999))
+
+
+def test_gaussian_draw_statistics():
+    z = tq.draw_gaussian(12345, 200_000)
+    assert abs(z.mean()) < 4 / math.sqrt(len(z))
+    assert abs(z.var() - 1) < 4 * math.sqrt(2 / len(z))
+    s = tq.draw_signs(7, 100_000)
+    assert set(np.unique(s)) == {-1, 1}
+    assert abs(s.mean()) < 4 / math.sqrt(len(s))
+
+
+@pytest.mark.parametrize("d", [8, 128, 256])
+def test_haar_rotation_matches_oracle(d):
+    g = synth.gaussian_matrix(d, seed=0)
+    P = tq.haar_rotation(g)
+    np.testing.assert_allclose(P, orot.haar_from_gaussian(g), atol=1e-12)
+
+
+def test_state_create_validation_without_gpu():
+    lib = tq.lib()
+    h = ctypes.c_void_p()
+    bad = [
+        tq.Params(128, 3, 7, 0, 0, 0, 0, 1),      # mode
+        tq.Params(128, 3, 0, 5, 0, 0, 0, 1),      # rotation
+        tq.Params(128, 0, 0, 0, 0, 0, 0, 1),      # bits
+        tq.Params(128, 3, 0, 0, 9, 0, 0, 1),      # matrix dtype
+        tq.Params(1, 3, 0, 0, 0, 0, 0, 1),        # d
+        tq.Params(128, 3, 0, 0, 0, -1, 0, 1),     # device
+    ]
+    for p in bad:
+        assert lib.tq_state_create(ctypes.byref(p), None, None, None, ctypes.byref(h)) == 1
+    unsup = [tq.Params(96, 3, 0, 1, 0, 0, 0, 1),  # RHT needs a power of two
+             tq.Params(100, 3, 0, 0, 0, 0, 0, 1)]  # no kernel for d = 100
+    for p in unsup:
+        assert lib.tq_state_create(ctypes.byref(p), None, None, None, ctypes.byref(h)) == 2
+    assert lib.tq_state_create(None, None, None, None, ctypes.byref(h)) == 1
+    assert lib.tq_state_destroy(None) == 0
+
+
+def test_null_state_calls_are_rejected():
+    lib = tq.lib()
+    assert lib.tq_quantize_mse(None, None, 0, 1, 128, None, None, None) == 1
+    assert lib.tq_quantize_prod(None, None, 0, 1, 128, None, None, None, None, None) == 1
+    assert lib.tq_dequant(None, None, None, None, None, 1, None, None) == 1
+    assert lib.tq_score(None, None, 0, 1, 1, None, None, None, None, 1, None, None) == 1
+    n = ctypes.c_size_t()
+    assert lib.tq_attend_workspace(None, None, 1, 1, ctypes.byref(n)) == 1
+    assert lib.tq_search_workspace(None, 1, 1, 1, ctypes.byref(n)) == 1
+    assert lib.tq_state_import(None, 0, 0, None) == 1
+    buf = ctypes.create_string_buffer(b"XXXX" + bytes(200))
+    h = ctypes.c_void_p()
+    assert lib.tq_state_import(buf, 204, 0, ctypes.byref(h)) == 1

@@ -1,0 +1,329 @@
+"""Python binding of libtq (TurboQuant-style online vector quantization on B200).
+
+Argument marshalling only: every call goes straight to the C ABI declared in
+include/tq.h, and every step of the computation runs in the library's CUDA kernels
+(host-only steps: codebook and state creation). PyTorch tensors are accepted for
+device buffers and streams; plain integers (device addresses) work too.
+
+The library must be built first (``python vector_quantization_tq_b200/build.py`` or
+``__graft_entry__.build()``); importing this package without it raises ImportError.
+There is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+__all__ = [
+    "TQError", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
+    "MSE", "PROD", "ROT_DENSE", "ROT_RHT", "F32", "BF16",
+    "build_codebook", "draw_gaussian", "draw_signs", "haar_rotation",
+    "State", "quantize_mse", "quantize_prod", "dequant", "score",
+    "attend_workspace", "attend_decode", "search_workspace", "search_topk",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "tq.h")
+
+MSE, PROD = 0, 1
+ROT_DENSE, ROT_RHT = 0, 1
+F32, BF16 = 0, 1
+FIELD_CENTROIDS, FIELD_BOUNDS, FIELD_PI, FIELD_SIGNS, FIELD_S = 0, 1, 2, 3, 4
+STATUS = {0: "TQ_OK", 1: "TQ_EINVAL", 2: "TQ_EUNSUPPORTED", 3: "TQ_ENOMEM", 4: "TQ_ECUDA", 5: "TQ_EDEVICE"}
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_lib.tq_status_string(status).decode()})"
+                         + (f", cudaError {_lib.tq_last_cuda_error()}" if status == 4 else ""))
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("b", ctypes.c_int32), ("mode", ctypes.c_int32),
+                ("rot", ctypes.c_int32), ("mat_dtype", ctypes.c_int32), ("device", ctypes.c_int32),
+                ("seed_pi", ctypes.c_uint64), ("seed_s", ctypes.c_uint64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libtq.so is not built at {LIB_PATH}; run `python vector_quantization_tq_b200/build.py`")
+    return ctypes.CDLL(LIB_PATH, mode=ctypes.RTLD_GLOBAL)
+
+
+_lib = _load()
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_DP = ctypes.POINTER(ctypes.c_double)
+
+_SIGS = {
+    "tq_status_string": (ctypes.c_char_p, [_I]),
+    "tq_last_cuda_error": (_I, []),
+    "tq_version": (_I, []),
+    "tq_build_codebook": (_I, [_I, _I, _DP, _DP, _DP]),
+    "tq_draw_gaussian": (_I, [ctypes.c_uint64, _SZ, _DP]),
+    "tq_draw_signs": (_I, [ctypes.c_uint64, _SZ, _P]),
+    "tq_haar_rotation": (_I, [_I, _DP, _DP]),
+    "tq_state_create": (_I, [ctypes.POINTER(Params), _DP, _P, _DP, ctypes.POINTER(_P)]),
+    "tq_state_destroy": (_I, [_P]),
+    "tq_state_params": (_I, [_P, ctypes.POINTER(Params)]),
+    "tq_state_codebook_info": (_I, [_P, ctypes.POINTER(_I), _DP]),
+    "tq_state_copy": (_I, [_P, _I, _DP, _SZ]),
+    "tq_state_export": (_I, [_P, _P, ctypes.POINTER(_SZ)]),
+    "tq_state_import": (_I, [_P, _SZ, _I, ctypes.POINTER(_P)]),
+    "tq_code_layout": (_I, [_P, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
+    "tq_quantize_mse": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P]),
+    "tq_quantize_prod": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _P]),
+    "tq_dequant": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P]),
+    "tq_score": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
+    "tq_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
+    "tq_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _SZ, _P]),
+    "tq_search_workspace": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_SZ)]),
+    "tq_search_topk": (_I, [_P, _P, _I, _I64, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def lib():
+    return _lib
+
+
+def declared_symbols(header: str = HEADER_PATH):
+    """Names of the functions declared in include/tq.h."""
+    with open(header) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise TQError(rc, what)
+
+
+def _ptr(t):
+    """Device (or host) address of a tensor / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available() and torch.cuda.is_initialized():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _dp(a):
+    return a.ctypes.data_as(_DP) if a is not None else None
+
+
+# ---- host-only calls -------------------------------------------------------------------
+
+def build_codebook(d: int, b: int):
+    """(centroids[2^b], boundaries[2^b-1], D_mse) from the library's host codebook builder."""
+    c = np.zeros(1 << b)
+    t = np.zeros(max(1, (1 << b) - 1))
+    D = ctypes.c_double()
+    _check(_lib.tq_build_codebook(d, b, _dp(c), _dp(t), ctypes.byref(D)), "tq_build_codebook")
+    return c, t[: (1 << b) - 1], D.value
+
+
+def draw_gaussian(seed: int, count: int) -> np.ndarray:
+    out = np.zeros(count)
+    _check(_lib.tq_draw_gaussian(seed, count, _dp(out)), "tq_draw_gaussian")
+    return out
+
+
+def draw_signs(seed: int, count: int) -> np.ndarray:
+    out = np.zeros(count, dtype=np.int8)
+    _check(_lib.tq_draw_signs(seed, count, out.ctypes.data), "tq_draw_signs")
+    return out
+
+
+def haar_rotation(g: np.ndarray) -> np.ndarray:
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    d = g.shape[0]
+    out = np.zeros((d, d))
+    _check(_lib.tq_haar_rotation(d, _dp(g), _dp(out)), "tq_haar_rotation")
+    return out
+
+
+# ---- states ----------------------------------------------------------------------------
+
+class State:
+    """A quantizer state (codebook, rotation, QJL matrix) held by libtq on one device."""
+
+    def __init__(self, d: int, b: int, mode: int = MSE, rot: int = ROT_DENSE, mat_dtype: int = F32,
+                 device: int = 0, seed_pi: int = 0, seed_s: int = 1, gauss_pi=None, signs=None, s=None,
+                 _handle=None):
+        self._h = _P()
+        if _handle is not None:
+            self._h = _handle
+        else:
+            p = Params(d, b, mode, rot, mat_dtype, device, seed_pi, seed_s)
+            g = None if gauss_pi is None else np.ascontiguousarray(gauss_pi, dtype=np.float64)
+            sg = None if signs is None else np.ascontiguousarray(signs, dtype=np.int8)
+            sm = None if s is None else np.ascontiguousarray(s, dtype=np.float64)
+            _check(_lib.tq_state_create(ctypes.byref(p), _dp(g), None if sg is None else sg.ctypes.data,
+                                        _dp(sm), ctypes.byref(self._h)), "tq_state_create")
+        p = Params()
+        _check(_lib.tq_state_params(self._h, ctypes.byref(p)), "tq_state_params")
+        self.params = p
+        bm, dm = _I(), ctypes.c_double()
+        _check(_lib.tq_state_codebook_info(self._h, ctypes.byref(bm), ctypes.byref(dm)), "tq_state_codebook_info")
+        self.b_mse, self.dmse = bm.value, dm.value
+        cb, qb = _SZ(), _SZ()
+        _check(_lib.tq_code_layout(self._h, ctypes.byref(cb), ctypes.byref(qb)), "tq_code_layout")
+        self.code_bytes, self.qjl_bytes = cb.value, qb.value
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def d(self):
+        return self.params.d
+
+    @property
+    def mode(self):
+        return self.params.mode
+
+    def copy(self, field: int) -> np.ndarray:
+        d, L = self.params.d, 1 << self.b_mse
+        size = {FIELD_CENTROIDS: L, FIELD_BOUNDS: max(0, L - 1), FIELD_PI: d * d, FIELD_SIGNS: d, FIELD_S: d * d}[field]
+        out = np.zeros(max(1, size))
+        _check(_lib.tq_state_copy(self._h, field, _dp(out), out.size), "tq_state_copy")
+        out = out[:size]
+        return out.reshape(d, d) if field in (FIELD_PI, FIELD_S) else out
+
+    def export(self) -> bytes:
+        n = _SZ()
+        _check(_lib.tq_state_export(self._h, None, ctypes.byref(n)), "tq_state_export")
+        buf = ctypes.create_string_buffer(n.value)
+        _check(_lib.tq_state_export(self._h, buf, ctypes.byref(n)), "tq_state_export")
+        return buf.raw[: n.value]
+
+    @classmethod
+    def from_bytes(cls, blob: bytes, device: int = -1) -> "State":
+        h = _P()
+        buf = ctypes.create_string_buffer(blob, len(blob))
+        _check(_lib.tq_state_import(buf, len(blob), device, ctypes.byref(h)), "tq_state_import")
+        return cls(0, 0, _handle=h)
+
+    def close(self):
+        if self._h:
+            _lib.tq_state_destroy(self._h)
+            self._h = _P()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # allocation helpers (torch device tensors; plumbing only)
+    def empty_planes(self, n: int, device=None):
+        import torch
+        dev = device if device is not None else torch.device("cuda", self.params.device)
+        codes = torch.empty((n, self.code_bytes), dtype=torch.uint8, device=dev)
+        norms = torch.empty(n, dtype=torch.float32, device=dev)
+        if self.mode == PROD:
+            qjl = torch.empty((n, self.qjl_bytes), dtype=torch.uint8, device=dev)
+            rnorms = torch.empty(n, dtype=torch.float32, device=dev)
+            return codes, qjl, norms, rnorms
+        return codes, None, norms, None
+
+
+# ---- device calls ----------------------------------------------------------------------
+
+def quantize_mse(st: State, x, codes, norms, stream=None, n=None, ld=None, dtype=None):
+    n = x.shape[0] if n is None else n
+    ld = x.stride(0) if ld is None else ld
+    dt = _dtype_code(x) if dtype is None else dtype
+    _check(_lib.tq_quantize_mse(st.handle, _ptr(x), dt, n, ld, _ptr(codes), _ptr(norms), _stream(stream)),
+           "tq_quantize_mse")
+
+
+def quantize_prod(st: State, x, codes, qjl, norms, rnorms, stream=None, n=None, ld=None, dtype=None):
+    n = x.shape[0] if n is None else n
+    ld = x.stride(0) if ld is None else ld
+    dt = _dtype_code(x) if dtype is None else dtype
+    _check(_lib.tq_quantize_prod(st.handle, _ptr(x), dt, n, ld, _ptr(codes), _ptr(qjl), _ptr(norms),
+                                 _ptr(rnorms), _stream(stream)), "tq_quantize_prod")
+
+
+def dequant(st: State, codes, qjl, norms, rnorms, out, stream=None, n=None):
+    n = norms.shape[0] if n is None else n
+    _check(_lib.tq_dequant(st.handle, _ptr(codes), _ptr(qjl), _ptr(norms), _ptr(rnorms), n, _ptr(out),
+                           _stream(stream)), "tq_dequant")
+
+
+def score(st: State, q, codes, qjl, norms, rnorms, scores, groups: int = 1, nq=None, n=None, stream=None):
+    """scores[g][i][k] = estimate of <q[g][i], x[g][k]>; q is [groups*nq, d] or [groups, nq, d]."""
+    nq = (q.shape[-2] if q.dim() == 3 else q.shape[0] // groups) if nq is None else nq
+    n = norms.shape[-1] if n is None else n
+    if norms.dim() == 1 and n == norms.shape[0] and groups > 1:
+        n = norms.shape[0] // groups
+    _check(_lib.tq_score(st.handle, _ptr(q), _dtype_code(q), groups, nq, _ptr(codes), _ptr(qjl), _ptr(norms),
+                         _ptr(rnorms), n, _ptr(scores), _stream(stream)), "tq_score")
+
+
+def attend_workspace(ks: State, vs: State, H: int, T: int) -> int:
+    n = _SZ()
+    _check(_lib.tq_attend_workspace(ks.handle, vs.handle, H, T, ctypes.byref(n)), "tq_attend_workspace")
+    return n.value
+
+
+def attend_decode(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale: float, out,
+                  workspace, ws_bytes=None, H=None, T=None, stream=None):
+    H = q.shape[0] if H is None else H
+    T = knorms.numel() // H if T is None else T
+    ws_bytes = (workspace.numel() * workspace.element_size() if workspace is not None else 0) \
+        if ws_bytes is None else ws_bytes
+    _check(_lib.tq_attend_decode(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, _ptr(kcodes), _ptr(kqjl),
+                                 _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out),
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "tq_attend_decode")
+
+
+def search_workspace(st: State, nq: int, n: int, k: int) -> int:
+    out = _SZ()
+    _check(_lib.tq_search_workspace(st.handle, nq, n, k, ctypes.byref(out)), "tq_search_workspace")
+    return out.value
+
+
+def search_topk(st: State, q, codes, qjl, norms, rnorms, k: int, idx, vals, workspace, ws_bytes=None,
+                stream=None):
+    nq, n = q.shape[0], norms.shape[0]
+    ws_bytes = (workspace.numel() * workspace.element_size() if workspace is not None else 0) \
+        if ws_bytes is None else ws_bytes
+    _check(_lib.tq_search_topk(st.handle, _ptr(q), _dtype_code(q), nq, _ptr(codes), _ptr(qjl), _ptr(norms),
+                               _ptr(rnorms), n, k, _ptr(idx), _ptr(vals), _ptr(workspace), ws_bytes,
+                               _stream(stream)), "tq_search_topk")

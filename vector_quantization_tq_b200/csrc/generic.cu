@@ -1,0 +1,831 @@
+// General-purpose libtq kernels: encode (TurboQuant_mse / _prod), dequant, score,
+// decode attention and top-k search, for every supported d, fp32 or bf16 state.
+//
+// Thread layout: a group of NT threads owns one vector at a time, each thread E
+// consecutive coordinates (j = tid*E + e, d = NT*E). For d <= 256 a group is one warp
+// and a block holds 8 independent groups; for d >= 512 a group is the whole block.
+//
+// The rotation and QJL products are CUDA-core FMA loops over the stored matrices
+// (fp32 accumulate), the RHT is an in-register / shuffle / shared-memory butterfly.
+// The specialised tensor-core encoder for d = 128 lives in encode_tc.cu.
+#include "common.cuh"
+
+namespace tq {
+namespace {
+
+template <int NT>
+__device__ __forceinline__ void group_sync() {
+    if constexpr (NT == 32) __syncwarp(); else __syncthreads();
+}
+
+// Sum over the NT threads of a group; `red` holds NT/32 floats (used when NT > 32).
+template <int NT>
+__device__ __forceinline__ float group_sum(float v, float* red) {
+    v = warp_sum(v);
+    if constexpr (NT == 32) {
+        return v;
+    } else {
+        const int w = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) red[w] = v;
+        __syncthreads();
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < NT / 32; ++i) s += red[i];
+        __syncthreads();
+        return s;
+    }
+}
+
+// In-place unnormalised Sylvester Walsh-Hadamard transform of the group's vector:
+// stages with stride < E in registers, then across threads (shuffle or shared memory).
+// For element j with bit h clear: y_j = x_j + x_{j+h}; with it set: y_j = x_{j-h} - x_j.
+template <int E, int NT>
+__device__ __forceinline__ void fwht(float (&v)[E], int tid, float* xch) {
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if ((e & h) == 0) {
+                const float a = v[e], b = v[e + h];
+                v[e] = a + b;
+                v[e + h] = a - b;
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < NT; m <<= 1) {
+        if (m < 32) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+                v[e] = (tid & m) ? (o - v[e]) : (v[e] + o);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) xch[tid * E + e] = v[e];
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float o = xch[(tid ^ m) * E + e];
+                v[e] = (tid & m) ? (o - v[e]) : (v[e] + o);
+            }
+            __syncthreads();
+        }
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ int groups_per_block() { return NT == 32 ? 8 : 1; }
+
+// ------------------------------------------------------------------------------------
+// Encode: norm, rotate, normalise, quantize, (prod) residual + QJL signs, pack.
+// Per group shared memory: d floats (broadcast buffer) + d bytes codes + d bytes signs.
+// ------------------------------------------------------------------------------------
+template <int E, int NT>
+__global__ void __launch_bounds__(NT == 32 ? 256 : NT)
+encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t n, int64_t ld,
+              uint8_t* __restrict__ codes, uint8_t* __restrict__ qjl, float* __restrict__ norms,
+              float* __restrict__ rnorms) {
+    constexpr int D = NT * E;
+    constexpr int GPB = (NT == 32) ? 8 : 1;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float* ctab = reinterpret_cast<float*>(smem_raw);                 // kMaxLevels
+    float* ttab = ctab + kMaxLevels;                                   // kMaxLevels
+    float* red = ttab + kMaxLevels;                                    // 8
+    const int g = threadIdx.x / NT;
+    const int tid = threadIdx.x % NT;
+    float* vbuf = red + 8 + g * D;                                     // D floats per group
+    uint8_t* cbuf = reinterpret_cast<uint8_t*>(red + 8 + GPB * D) + g * 2 * D;
+    uint8_t* zbuf = cbuf + D;
+    for (int i = threadIdx.x; i < st.L; i += blockDim.x) {
+        ctab[i] = st.c[i];
+        ttab[i] = st.t[i];
+    }
+    __syncthreads();
+    const bool prod = (st.mode == TQ_PROD);
+    const int lane = threadIdx.x & 31;
+    const int warp_in_group = tid >> 5;
+    constexpr int WPG = NT / 32;
+
+    for (int64_t vec = (int64_t)blockIdx.x * GPB + g; vec < n; vec += (int64_t)gridDim.x * GPB) {
+        float xv[E];
+        load_elems<E>(x, dtype, vec * ld + (int64_t)tid * E, xv);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(xv[e], xv[e], ss);
+        const float nu = sqrtf(group_sum<NT>(ss, red));
+        float y[E];
+        if (st.rot == TQ_ROT_RHT) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) y[e] = rht_neg(st, tid * E + e) ? -xv[e] : xv[e];
+            fwht<E, NT>(y, tid, vbuf);
+            const float sc = (nu > 0.f) ? st.rsqrt_d / nu : 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) y[e] *= sc;
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) vbuf[tid * E + e] = xv[e];
+            group_sync<NT>();
+            matvec_cols<E>(st.piT, st.mat_dtype, D, tid * E, vbuf, y);
+            group_sync<NT>();
+            const float sc = (nu > 0.f) ? 1.f / nu : 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) y[e] *= sc;
+        }
+        // quantize (+ residual)
+        float r[E];
+        float rr = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            int c = 0;
+            if (st.b_mse > 0) c = quantize_coord(st, ttab, y[e]);
+            cbuf[tid * E + e] = (uint8_t)c;
+            r[e] = (nu > 0.f) ? (y[e] - (st.b_mse > 0 ? ctab[c] : 0.f)) : 0.f;
+            rr = fmaf(r[e], r[e], rr);
+        }
+        if (prod) {
+            const float rho = sqrtf(group_sum<NT>(rr, red));
+#pragma unroll
+            for (int e = 0; e < E; ++e) vbuf[tid * E + e] = r[e];
+            group_sync<NT>();
+            float s[E];
+            matvec_cols<E>(st.sT, st.mat_dtype, D, tid * E, vbuf, s);
+#pragma unroll
+            for (int e = 0; e < E; ++e) zbuf[tid * E + e] = (s[e] >= 0.f) ? 1 : 0;
+            if (tid == 0) {
+                norms[vec] = nu;
+                rnorms[vec] = rho;
+            }
+        } else if (tid == 0) {
+            norms[vec] = nu;
+        }
+        group_sync<NT>();
+        // pack codes: stream bit p = 32w + lane -> code p / b, bit p % b
+        if (st.b_mse > 0) {
+            const int b = st.b_mse;
+            const int W = b * D / 32;
+            uint32_t* out = reinterpret_cast<uint32_t*>(codes + vec * st.code_bytes);
+            for (int w = warp_in_group; w < W; w += WPG) {
+                const int p = 32 * w + lane;
+                const int j = p / b;
+                const uint32_t bit = (cbuf[j] >> (p - j * b)) & 1u;
+                const uint32_t word = __ballot_sync(0xffffffffu, bit);
+                if (lane == 0) out[w] = word;
+            }
+        }
+        if (prod) {
+            uint32_t* out = reinterpret_cast<uint32_t*>(qjl + vec * st.qjl_bytes);
+            for (int w = warp_in_group; w < D / 32; w += WPG) {
+                const uint32_t word = __ballot_sync(0xffffffffu, zbuf[32 * w + lane]);
+                if (lane == 0) out[w] = word;
+            }
+        }
+        group_sync<NT>();
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Dequant: x~ = ||x|| Pi^T (c[idx] + ||r|| sqrt(pi/2)/d S^T (2z-1)).
+// ------------------------------------------------------------------------------------
+template <int E, int NT>
+__global__ void __launch_bounds__(NT == 32 ? 256 : NT)
+dequant_kernel(const DevState st, const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
+               const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
+               float* __restrict__ out) {
+    constexpr int D = NT * E;
+    constexpr int GPB = (NT == 32) ? 8 : 1;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float* ctab = reinterpret_cast<float*>(smem_raw);
+    const int g = threadIdx.x / NT;
+    const int tid = threadIdx.x % NT;
+    float* vbuf = ctab + kMaxLevels + g * D;
+    for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
+    __syncthreads();
+    const bool prod = (qjl != nullptr);
+    const int nwords = st.code_bytes / 4;
+    for (int64_t vec = (int64_t)blockIdx.x * GPB + g; vec < n; vec += (int64_t)gridDim.x * GPB) {
+        float yt[E];
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(codes + vec * st.code_bytes);
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            yt[e] = (st.b_mse > 0) ? ctab[extract_code(row, nwords, tid * E + e, st.b_mse)] : 0.f;
+        if (prod) {
+            const uint8_t* zr = qjl + vec * st.qjl_bytes;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = tid * E + e;
+                vbuf[j] = ((__ldg(zr + (j >> 3)) >> (j & 7)) & 1u) ? 1.f : -1.f;
+            }
+            group_sync<NT>();
+            float t[E];
+            matvec_cols<E>(st.s, st.mat_dtype, D, tid * E, vbuf, t);   // (S^T z)_k = sum_j S[j][k] z_j
+            group_sync<NT>();
+            const float a = __ldg(rnorms + vec) * st.qjl_scale;
+#pragma unroll
+            for (int e = 0; e < E; ++e) yt[e] = fmaf(a, t[e], yt[e]);
+        }
+        float xo[E];
+        if (st.rot == TQ_ROT_RHT) {
+            fwht<E, NT>(yt, tid, vbuf);
+#pragma unroll
+            for (int e = 0; e < E; ++e) xo[e] = (rht_neg(st, tid * E + e) ? -yt[e] : yt[e]) * st.rsqrt_d;
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) vbuf[tid * E + e] = yt[e];
+            group_sync<NT>();
+            matvec_cols<E>(st.pi, st.mat_dtype, D, tid * E, vbuf, xo);   // x_k = sum_j Pi[j][k] y_j
+            group_sync<NT>();
+        }
+        const float nu = __ldg(norms + vec);
+        float* o = out + vec * D + tid * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = xo[e] * nu;
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Query preparation inside a block: qp = Pi q and u = S qp for `count` queries
+// (rows of q with stride d, fp32 or bf16) into shared memory [count][d].
+// ------------------------------------------------------------------------------------
+__device__ void prep_queries(const DevState& st, const void* q, int qdtype, int count,
+                             float* qs, float* qp, float* u) {
+    const int d = st.d;
+    for (int i = threadIdx.x; i < count * d; i += blockDim.x)
+        qs[i] = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + i)
+                                   : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + i));
+    __syncthreads();
+    if (st.rot == TQ_ROT_RHT) {
+        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
+            const int j = i % d;
+            qp[i] = rht_neg(st, j) ? -qs[i] : qs[i];
+        }
+        __syncthreads();
+        for (int h = 1; h < d; h <<= 1) {
+            for (int p = threadIdx.x; p < count * d / 2; p += blockDim.x) {
+                const int qi = p / (d / 2), pr = p % (d / 2);
+                const int j = (pr / h) * 2 * h + (pr % h);
+                float* v = qp + qi * d;
+                const float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+            __syncthreads();
+        }
+        for (int i = threadIdx.x; i < count * d; i += blockDim.x) qp[i] *= st.rsqrt_d;
+    } else {
+        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
+            const int qi = i / d, j = i % d;
+            float a = 0.f;
+            for (int k = 0; k < d; ++k) a = fmaf(mat_elem(st.piT, st.mat_dtype, (int64_t)k * d + j), qs[qi * d + k], a);
+            qp[i] = a;
+        }
+    }
+    __syncthreads();
+    if (st.mode == TQ_PROD) {
+        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
+            const int qi = i / d, j = i % d;
+            float a = 0.f;
+            for (int k = 0; k < d; ++k) a = fmaf(mat_elem(st.sT, st.mat_dtype, (int64_t)k * d + j), qp[qi * d + k], a);
+            u[i] = a;
+        }
+    }
+    __syncthreads();
+}
+
+
+// The two sums of an estimate for up to QT queries against one key:
+//   a1 = sum_j qp_j c[idx_j],  a2 = sum_j u_j (2 z_j - 1).
+template <int QT>
+__device__ __forceinline__ void score_sums(const DevState& st, const float* ctab, const float* qp,
+                                           const float* u, int nqt, const uint8_t* codes,
+                                           const uint8_t* qjl, int64_t key, float (&a1)[QT],
+                                           float (&a2)[QT]) {
+    const int d = st.d;
+#pragma unroll
+    for (int i = 0; i < QT; ++i) a1[i] = a2[i] = 0.f;
+    if (st.b_mse > 0) {
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(codes + key * st.code_bytes);
+        const int b = st.b_mse;
+        const uint32_t mask = (1u << b) - 1u;
+        uint64_t buf = 0;
+        int have = 0, wi = 0;
+        for (int j = 0; j < d; ++j) {
+            if (have < b) {
+                buf |= (uint64_t)__ldg(row + wi++) << have;
+                have += 32;
+            }
+            const float cv = ctab[buf & mask];
+            buf >>= b;
+            have -= b;
+#pragma unroll
+            for (int i = 0; i < QT; ++i)
+                if (i < nqt) a1[i] = fmaf(qp[i * d + j], cv, a1[i]);
+        }
+    }
+    if (qjl != nullptr) {
+        const uint32_t* zr = reinterpret_cast<const uint32_t*>(qjl + key * st.qjl_bytes);
+        for (int w = 0; w < d / 32; ++w) {
+            const uint32_t word = __ldg(zr + w);
+            for (int bt = 0; bt < 32; ++bt) {
+                const float sg = ((word >> bt) & 1u) ? 1.f : -1.f;
+                const int j = w * 32 + bt;
+#pragma unroll
+                for (int i = 0; i < QT; ++i)
+                    if (i < nqt) a2[i] = fmaf(u[i * d + j], sg, a2[i]);
+            }
+        }
+    }
+}
+
+constexpr int kScoreQT = 8;
+constexpr int kScoreThreads = 256;
+
+size_t score_smem_bytes(int d) { return (size_t)(kMaxLevels + 3 * kScoreQT * d) * sizeof(float); }
+
+__global__ void __launch_bounds__(kScoreThreads)
+score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t nq,
+             const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
+             const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
+             float* __restrict__ scores) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int d = st.d;
+    float* ctab = reinterpret_cast<float*>(smem_raw);
+    float* qs = ctab + kMaxLevels;
+    float* qp = qs + kScoreQT * d;
+    float* u = qp + kScoreQT * d;
+    const int64_t grp = blockIdx.z;
+    const int64_t q0 = (int64_t)blockIdx.y * kScoreQT;
+    const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
+    for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
+    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
+    prep_queries(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * d) * qelem,
+                 qdtype, nqt, qs, qp, u);
+    for (int64_t key = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; key < n;
+         key += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t gk = grp * n + key;
+        float a1[kScoreQT], a2[kScoreQT];
+        score_sums<kScoreQT>(st, ctab, qp, u, nqt, codes, qjl, gk, a1, a2);
+        const float nu = __ldg(norms + gk);
+        const float g2 = (qjl != nullptr) ? __ldg(rnorms + gk) * st.qjl_scale : 0.f;
+        for (int i = 0; i < nqt; ++i) scores[(grp * nq + q0 + i) * n + key] = nu * fmaf(g2, a2[i], a1[i]);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Decode attention, split over tokens (flash-decoding style), then a combine launch.
+// Partial record per (head, split): m, l, acc[d] (value sum in the rotated domain).
+// ------------------------------------------------------------------------------------
+constexpr int kAttThreads = 256;
+constexpr int kAttMaxJ = kMaxDim / kAttThreads;   // coordinates per thread when d > 256
+
+size_t attend_smem_bytes(int d) {
+    const int accs = (d > kAttThreads) ? d : kAttThreads;
+    return (size_t)(2 * kMaxLevels + 3 * d + kAttThreads + 32 + accs) * sizeof(float);
+}
+
+__global__ void __launch_bounds__(kAttThreads)
+attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict__ q, int qdtype,
+                    int64_t T, int64_t chunk, const uint8_t* __restrict__ kcodes,
+                    const uint8_t* __restrict__ kqjl, const float* __restrict__ knorms,
+                    const float* __restrict__ krnorms, const uint8_t* __restrict__ vcodes,
+                    const float* __restrict__ vnorms, float scale, float* __restrict__ part) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int d = ks.d;
+    const int h = blockIdx.y;
+    const int split = blockIdx.x;
+    const int nsplit = gridDim.x;
+    float* kc = reinterpret_cast<float*>(smem_raw);      // K centroids
+    float* vc = kc + kMaxLevels;                          // V centroids
+    float* qs = vc + kMaxLevels;                          // d
+    float* qp = qs + d;                                   // d
+    float* u = qp + d;                                    // d
+    float* wt = u + d;                                    // kAttThreads weights p_t * ||v_t||
+    float* red = wt + kAttThreads;                        // 32
+    float* accs = red + 32;                               // max(d, kAttThreads)
+    for (int i = threadIdx.x; i < ks.L; i += blockDim.x) kc[i] = ks.c[i];
+    for (int i = threadIdx.x; i < vs.L; i += blockDim.x) vc[i] = vs.c[i];
+    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
+    prep_queries(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u);
+
+    const int64_t t_begin = (int64_t)split * chunk;
+    const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
+    // Value accumulation layout: d <= 256: `per` threads per coordinate split the tokens;
+    // d > 256: each thread owns coordinates threadIdx.x + m*256 for all tokens.
+    const int per = (d <= kAttThreads) ? kAttThreads / d : 1;
+    const int jpt = (d <= kAttThreads) ? 1 : d / kAttThreads;
+    const int j0 = (d <= kAttThreads) ? (threadIdx.x % d) : threadIdx.x;
+    const int half = (d <= kAttThreads) ? (threadIdx.x / d) : 0;
+    float acc[kAttMaxJ];
+#pragma unroll
+    for (int m = 0; m < kAttMaxJ; ++m) acc[m] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const int vnw = vs.code_bytes / 4;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += kAttThreads) {
+        const int cnt = (int)(t_end - t0 < kAttThreads ? t_end - t0 : kAttThreads);
+        float s = -INFINITY;
+        if (threadIdx.x < cnt) {
+            const int64_t gk = (int64_t)h * T + t0 + threadIdx.x;
+            float a1[1], a2[1];
+            score_sums<1>(ks, kc, qp, u, 1, kcodes, kqjl, gk, a1, a2);
+            const float g2 = (kqjl != nullptr) ? __ldg(krnorms + gk) * ks.qjl_scale : 0.f;
+            s = scale * __ldg(knorms + gk) * fmaf(g2, a2[0], a1[0]);
+        }
+        float mx = warp_max(s);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        float tmax = red[0];
+        for (int i = 1; i < kAttThreads / 32; ++i) tmax = fmaxf(tmax, red[i]);
+        __syncthreads();
+        const float m_new = fmaxf(m_run, tmax);
+        const float alpha = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
+        const float p = (threadIdx.x < cnt) ? __expf(s - m_new) : 0.f;
+        const float psum = warp_sum(p);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = psum;
+        if (threadIdx.x < cnt) wt[threadIdx.x] = p * __ldg(vnorms + (int64_t)h * T + t0 + threadIdx.x);
+        __syncthreads();
+        float tsum = 0.f;
+        for (int i = 0; i < kAttThreads / 32; ++i) tsum += red[i];
+        l_run = l_run * alpha + tsum;
+        m_run = m_new;
+#pragma unroll
+        for (int m = 0; m < kAttMaxJ; ++m) acc[m] *= alpha;
+        for (int t = half; t < cnt; t += per) {
+            const uint32_t* row =
+                reinterpret_cast<const uint32_t*>(vcodes + ((int64_t)h * T + t0 + t) * vs.code_bytes);
+            const float w = wt[t];
+#pragma unroll
+            for (int m = 0; m < kAttMaxJ; ++m)
+                if (m < jpt) acc[m] = fmaf(w, vc[extract_code(row, vnw, j0 + m * kAttThreads, vs.b_mse)], acc[m]);
+        }
+        __syncthreads();
+    }
+    float* rec = part + ((int64_t)h * nsplit + split) * (d + 2);
+    if (d <= kAttThreads) {
+        accs[half * d + j0] = acc[0];
+        __syncthreads();
+        for (int jj = threadIdx.x; jj < d; jj += blockDim.x) {
+            float a = 0.f;
+            for (int hh = 0; hh < per; ++hh) a += accs[hh * d + jj];
+            rec[2 + jj] = a;
+        }
+    } else {
+        for (int m = 0; m < jpt; ++m) rec[2 + j0 + m * kAttThreads] = acc[m];
+    }
+    if (threadIdx.x == 0) {
+        rec[0] = m_run;
+        rec[1] = l_run;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ part, float* __restrict__ out) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int d = vs.d;
+    const int h = blockIdx.x;
+    float* o = reinterpret_cast<float*>(smem_raw);   // d
+    const float* base = part + (int64_t)h * nsplit * (d + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (d + 2)]);
+    float Lsum = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float m = base[s * (d + 2)];
+        if (m != -INFINITY) Lsum += base[s * (d + 2) + 1] * __expf(m - M);
+    }
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        float a = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const float m = base[s * (d + 2)];
+            if (m != -INFINITY) a = fmaf(base[s * (d + 2) + 2 + j], __expf(m - M), a);
+        }
+        o[j] = a / Lsum;
+    }
+    __syncthreads();
+    // out = Pi_V^T o
+    if (vs.rot == TQ_ROT_RHT) {
+        for (int hh = 1; hh < d; hh <<= 1) {
+            for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
+                const int j = (p / hh) * 2 * hh + (p % hh);
+                const float a = o[j], b = o[j + hh];
+                o[j] = a + b;
+                o[j + hh] = a - b;
+            }
+            __syncthreads();
+        }
+        for (int k = threadIdx.x; k < d; k += blockDim.x)
+            out[(int64_t)h * d + k] = (rht_neg(vs, k) ? -o[k] : o[k]) * vs.rsqrt_d;
+    } else {
+        for (int k = threadIdx.x; k < d; k += blockDim.x) {
+            float a = 0.f;
+            for (int j = 0; j < d; ++j) a = fmaf(mat_elem(vs.pi, vs.mat_dtype, (int64_t)j * d + k), o[j], a);
+            out[(int64_t)h * d + k] = a;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Top-k search: per (query tile, key block) candidates, then a per-query merge.
+// Order: larger value first; equal values -> lower index first.
+// ------------------------------------------------------------------------------------
+constexpr int kSearchThreads = 256;
+
+__device__ __forceinline__ bool better(float v1, int64_t i1, float v2, int64_t i2) {
+    return (v1 > v2) || (v1 == v2 && i1 < i2);
+}
+
+// Block-wide selection of the best (v, i) among the threads' current candidates.
+__device__ __forceinline__ void block_best(float v, int64_t i, float* rv, int64_t* ri, float& bv, int64_t& bi) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        const int64_t oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (better(ov, oi, v, i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        rv[w] = v;
+        ri[w] = i;
+    }
+    __syncthreads();
+    bv = rv[0];
+    bi = ri[0];
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k)
+        if (better(rv[k], ri[k], bv, bi)) {
+            bv = rv[k];
+            bi = ri[k];
+        }
+    __syncthreads();
+}
+
+// Scores of a block of keys for up to kScoreQT queries, then the block's k best per query.
+// Taken slots are overwritten with NaN, which never compares better.
+__global__ void __launch_bounds__(kSearchThreads)
+search_block_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t nq,
+                    const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
+                    const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n, int k,
+                    int block_keys, float* __restrict__ cand_v, int64_t* __restrict__ cand_i) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int d = st.d;
+    float* ctab = reinterpret_cast<float*>(smem_raw);
+    float* qs = ctab + kMaxLevels;
+    float* qp = qs + kScoreQT * d;
+    float* u = qp + kScoreQT * d;
+    float* rv = u + kScoreQT * d;                                   // 8
+    int64_t* ri = reinterpret_cast<int64_t*>(rv + 8);               // 8
+    float* sv = reinterpret_cast<float*>(ri + 8);                   // kScoreQT * block_keys
+    const int64_t q0 = (int64_t)blockIdx.y * kScoreQT;
+    const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
+    for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
+    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
+    prep_queries(st, reinterpret_cast<const unsigned char*>(q) + (size_t)(q0 * d) * qelem, qdtype, nqt, qs, qp, u);
+    const int64_t k0 = (int64_t)blockIdx.x * block_keys;
+    for (int local = threadIdx.x; local < block_keys; local += blockDim.x) {
+        const int64_t key = k0 + local;
+        if (key < n) {
+            float a1[kScoreQT], a2[kScoreQT];
+            score_sums<kScoreQT>(st, ctab, qp, u, nqt, codes, qjl, key, a1, a2);
+            const float nu = __ldg(norms + key);
+            const float g2 = (qjl != nullptr) ? __ldg(rnorms + key) * st.qjl_scale : 0.f;
+            for (int i = 0; i < nqt; ++i) sv[i * block_keys + local] = nu * fmaf(g2, a2[i], a1[i]);
+        } else {
+            for (int i = 0; i < nqt; ++i) sv[i * block_keys + local] = __int_as_float(0x7fc00000);
+        }
+    }
+    __syncthreads();
+    const int64_t nblk = gridDim.x;
+    for (int i = 0; i < nqt; ++i) {
+        float* row = sv + i * block_keys;
+        for (int sel = 0; sel < k; ++sel) {
+            float bv = -INFINITY;
+            int64_t bi = INT64_MAX;
+            for (int t = threadIdx.x; t < block_keys; t += blockDim.x)
+                if (better(row[t], k0 + t, bv, bi)) {
+                    bv = row[t];
+                    bi = k0 + t;
+                }
+            float wv;
+            int64_t wi;
+            block_best(bv, bi, rv, ri, wv, wi);
+            if (threadIdx.x == 0) {
+                const int64_t o = ((q0 + i) * nblk + blockIdx.x) * k + sel;
+                cand_v[o] = wv;
+                cand_i[o] = wi;
+                if (wi != INT64_MAX) row[wi - k0] = __int_as_float(0x7fc00000);
+            }
+            __syncthreads();
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kSearchThreads)
+search_merge_kernel(int64_t ncand, int k, const float* __restrict__ cand_v, const int64_t* __restrict__ cand_i,
+                    int64_t* __restrict__ idx, float* __restrict__ vals) {
+    __shared__ float rv[8];
+    __shared__ int64_t ri[8];
+    __shared__ int64_t taken[64];
+    const int64_t qi = blockIdx.x;
+    const float* cv = cand_v + qi * ncand;
+    const int64_t* ci = cand_i + qi * ncand;
+    for (int sel = 0; sel < k; ++sel) {
+        float bv = -INFINITY;
+        int64_t bi = INT64_MAX;
+        for (int64_t t = threadIdx.x; t < ncand; t += blockDim.x) {
+            const int64_t id = ci[t];
+            if (id == INT64_MAX) continue;
+            bool used = false;
+            for (int s = 0; s < sel; ++s) used |= (taken[s] == id);
+            if (!used && better(cv[t], id, bv, bi)) {
+                bv = cv[t];
+                bi = id;
+            }
+        }
+        float wv;
+        int64_t wi;
+        block_best(bv, bi, rv, ri, wv, wi);
+        if (threadIdx.x == 0) {
+            taken[sel] = wi;
+            idx[qi * k + sel] = wi;
+            vals[qi * k + sel] = wv;
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// launch helpers
+// ------------------------------------------------------------------------------------
+int num_sms() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+template <int E, int NT>
+int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
+                    uint8_t* qjl, float* norms, float* rnorms, cudaStream_t s) {
+    constexpr int GPB = (NT == 32) ? 8 : 1;
+    const int threads = NT * GPB;
+    const size_t smem = (2 * kMaxLevels + 8) * sizeof(float) + GPB * (NT * E) * (sizeof(float) + 2);
+    auto kern = encode_kernel<E, NT>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t blocks_needed = (n + GPB - 1) / GPB;
+    const int blocks = (int)std::min<int64_t>(blocks_needed, (int64_t)num_sms() * 16);
+    kern<<<blocks, threads, smem, s>>>(st, x, dtype, n, ld, codes, qjl, norms, rnorms);
+    return (int)cudaGetLastError();
+}
+
+template <int E, int NT>
+int launch_dequant_t(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                     const float* rnorms, int64_t n, float* out, cudaStream_t s) {
+    constexpr int GPB = (NT == 32) ? 8 : 1;
+    const int threads = NT * GPB;
+    const size_t smem = kMaxLevels * sizeof(float) + GPB * (NT * E) * sizeof(float);
+    auto kern = dequant_kernel<E, NT>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t blocks_needed = (n + GPB - 1) / GPB;
+    const int blocks = (int)std::min<int64_t>(blocks_needed, (int64_t)num_sms() * 16);
+    kern<<<blocks, threads, smem, s>>>(st, codes, qjl, norms, rnorms, n, out);
+    return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
+                          uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    switch (st.d) {
+        case 32: return launch_encode_t<1, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 64: return launch_encode_t<2, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 128: return launch_encode_t<4, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 256: return launch_encode_t<8, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 512: return launch_encode_t<8, 64>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 1024: return launch_encode_t<8, 128>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 1536: return launch_encode_t<8, 192>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        case 2048: return launch_encode_t<8, 256>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                   const float* rnorms, int64_t n, float* out, void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    switch (st.d) {
+        case 32: return launch_dequant_t<1, 32>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 64: return launch_dequant_t<2, 32>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 128: return launch_dequant_t<4, 32>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 256: return launch_dequant_t<8, 32>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 512: return launch_dequant_t<8, 64>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 1024: return launch_dequant_t<8, 128>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 1536: return launch_dequant_t<8, 192>(st, codes, qjl, norms, rnorms, n, out, s);
+        case 2048: return launch_dequant_t<8, 256>(st, codes, qjl, norms, rnorms, n, out, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
+                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                 void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t smem = score_smem_bytes(st.d);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t qtiles = (nq + kScoreQT - 1) / kScoreQT;
+    if (qtiles > 65535) return (int)cudaErrorInvalidConfiguration;
+    int64_t kb = (n + kScoreThreads - 1) / kScoreThreads;
+    const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / std::max<int64_t>(1, qtiles * groups));
+    kb = std::min<int64_t>(kb, std::max<int64_t>(want, 1));
+    kb = std::min<int64_t>(kb, 1 << 20);
+    dim3 grid((unsigned)kb, (unsigned)qtiles, (unsigned)groups);
+    score_kernel<<<grid, kScoreThreads, smem, s>>>(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, scores);
+    return (int)cudaGetLastError();
+}
+
+namespace {
+int attend_splits(int H, int64_t T) {
+    int64_t target = (int64_t)num_sms() * 4;
+    int64_t sp = std::max<int64_t>(1, target / std::max(1, H));
+    sp = std::min<int64_t>(sp, (T + kAttThreads - 1) / kAttThreads);
+    return (int)std::max<int64_t>(1, sp);
+}
+}  // namespace
+
+size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T) {
+    if (H <= 0 || T <= 0) return 0;
+    const int sp = attend_splits(H, T);
+    return (size_t)H * sp * (ks.d + 2) * sizeof(float);
+}
+
+int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
+                  const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+                  const uint8_t* vcodes, const float* vnorms, float scale, float* out, void* ws, size_t ws_bytes,
+                  void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    const int sp = attend_splits(H, T);
+    const int64_t chunk = (T + sp - 1) / sp;
+    const int nsplit = (int)((T + chunk - 1) / chunk);
+    float* part = reinterpret_cast<float*>(ws);
+    const size_t smem = attend_smem_bytes(ks.d);
+    if (smem > 48 * 1024)
+        cudaFuncSetAttribute(attend_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid((unsigned)nsplit, (unsigned)H);
+    attend_split_kernel<<<grid, kAttThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms, krnorms,
+                                                         vcodes, vnorms, scale, part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+    attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, out);
+    return (int)cudaGetLastError();
+}
+
+namespace {
+int search_block_keys(int d) {
+    const size_t base = score_smem_bytes(d) + 8 * 4 + 8 * 8;
+    const size_t budget = 200 * 1024;
+    int keys = (int)((budget - base) / (kScoreQT * sizeof(float)));
+    keys = std::min(keys, 4096);
+    return std::max(kSearchThreads, keys / kSearchThreads * kSearchThreads);
+}
+int64_t search_blocks(int64_t n, int d) {
+    const int bk = search_block_keys(d);
+    return (n + bk - 1) / bk;
+}
+}  // namespace
+
+size_t search_workspace_bytes(const DevState& st, int64_t nq, int64_t n, int k) {
+    if (nq <= 0 || n <= 0) return 0;
+    const size_t nc = (size_t)nq * search_blocks(n, st.d) * k;
+    size_t b = nc * sizeof(float);
+    b = (b + 255) & ~(size_t)255;
+    return b + nc * sizeof(int64_t);
+}
+
+int launch_search(const DevState& st, const void* q, int qdtype, int64_t nq, const uint8_t* codes,
+                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int k, int64_t* idx,
+                  float* vals, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws_bytes;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int bk = search_block_keys(st.d);
+    const int64_t nblk = search_blocks(n, st.d);
+    const size_t nc = (size_t)nq * nblk * k;
+    float* cand_v = reinterpret_cast<float*>(ws);
+    const size_t off = (nc * sizeof(float) + 255) & ~(size_t)255;
+    int64_t* cand_i = reinterpret_cast<int64_t*>(reinterpret_cast<unsigned char*>(ws) + off);
+    const size_t smem = score_smem_bytes(st.d) + 8 * 4 + 8 * 8 + (size_t)kScoreQT * bk * sizeof(float);
+    cudaFuncSetAttribute(search_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t qtiles = (nq + kScoreQT - 1) / kScoreQT;
+    if (qtiles > 65535 || nblk > (1ll << 31) - 1 || nq > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)nblk, (unsigned)qtiles);
+    search_block_kernel<<<grid, kSearchThreads, smem, s>>>(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, k, bk,
+                                                            cand_v, cand_i);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+    search_merge_kernel<<<(unsigned)nq, kSearchThreads, 0, s>>>((int64_t)nblk * k, k, cand_v, cand_i, idx, vals);
+    return (int)cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,551 @@
+// C ABI of libtq: argument validation, state management, dispatch to the kernels.
+// The operations are defined in include/tq.h (with the passages they follow).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+namespace tq {
+
+static thread_local int g_last_cuda_error = 0;
+
+void set_cuda_error(int err) { g_last_cuda_error = err; }
+
+namespace {
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) return;
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) return;
+        ok = true;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool kernel_dim_supported(int d) {
+    switch (d) {
+        case 32: case 64: case 128: case 256: case 512: case 1024: case 1536: case 2048:
+            return true;
+        default:
+            return false;
+    }
+}
+
+bool is_pow2(int d) { return d > 0 && (d & (d - 1)) == 0; }
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return TQ_OK;
+    set_cuda_error((int)e);
+    (void)cudaGetLastError();   // clear a non-sticky error
+    return (e == cudaErrorMemoryAllocation) ? TQ_ENOMEM : TQ_ECUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_vectors(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld) {
+    if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_EINVAL;
+    if (n < 0) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    if (!x || ld < st->p.d) return TQ_EINVAL;
+    const int64_t es = (dtype == TQ_F32) ? 4 : 2;
+    if (!aligned16(x) || ((ld * es) & 15)) return TQ_EINVAL;
+    return TQ_OK;
+}
+
+uint16_t to_bf16_bits(float v) {
+    float r = bf16_round_host(v);
+    uint32_t u;
+    std::memcpy(&u, &r, 4);
+    return (uint16_t)(u >> 16);
+}
+
+// Upload Pi, Pi^T, S, S^T at the stored dtype and fill the kernel view.
+int finish_state(tq_state* st) {
+    const tq_params& p = st->p;
+    const int d = p.d;
+    tq::DevState& ds = st->dev;
+    std::memset(&ds, 0, sizeof(ds));
+    ds.d = d;
+    ds.b_mse = st->b_mse;
+    ds.L = 1 << st->b_mse;
+    ds.mode = p.mode;
+    ds.rot = p.rot;
+    ds.mat_dtype = p.mat_dtype;
+    ds.code_bytes = (st->b_mse * d + 7) / 8;
+    ds.qjl_bytes = (p.mode == TQ_PROD) ? d / 8 : 0;
+    ds.qjl_scale = (float)(std::sqrt(M_PI / 2.0) / d);
+    ds.rsqrt_d = (float)(1.0 / std::sqrt((double)d));
+    for (int i = 0; i < ds.L; ++i) ds.c[i] = (float)st->centroids[i];
+    for (int i = 0; i + 1 < ds.L; ++i) ds.t[i] = (float)st->bounds[i];
+    if (p.rot == TQ_ROT_RHT)
+        for (int j = 0; j < d; ++j)
+            if (st->signs[j] < 0) ds.signs[j / 32] |= 1u << (j % 32);
+
+    const size_t es = (p.mat_dtype == TQ_F32) ? 4 : 2;
+    const size_t mat = (size_t)d * d * es;
+    const bool dense = (p.rot == TQ_ROT_DENSE);
+    const bool prod = (p.mode == TQ_PROD);
+    const size_t nmat = (dense ? 2 : 0) + (prod ? 2 : 0);
+    if (nmat == 0) return TQ_OK;
+
+    std::vector<unsigned char> host(nmat * mat);
+    auto put = [&](size_t slot, const std::vector<double>& m, bool transpose) {
+        unsigned char* dst = host.data() + slot * mat;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) {
+                double v = transpose ? m[(size_t)j * d + i] : m[(size_t)i * d + j];
+                size_t o = (size_t)i * d + j;
+                if (p.mat_dtype == TQ_F32) {
+                    float f = (float)v;
+                    std::memcpy(dst + o * 4, &f, 4);
+                } else {
+                    uint16_t h = to_bf16_bits((float)v);
+                    std::memcpy(dst + o * 2, &h, 2);
+                }
+            }
+    };
+    size_t slot = 0;
+    size_t pi_slot = 0, s_slot = 0;
+    if (dense) {
+        pi_slot = slot;
+        put(slot++, st->pi, false);
+        put(slot++, st->pi, true);
+    }
+    if (prod) {
+        s_slot = slot;
+        put(slot++, st->s, false);
+        put(slot++, st->s, true);
+    }
+    DeviceGuard g(p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    cudaError_t e = cudaMalloc(&st->d_mem, host.size());
+    if (e != cudaSuccess) {
+        st->d_mem = nullptr;
+        return cuda_status(e);
+    }
+    e = cudaMemcpy(st->d_mem, host.data(), host.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_status(e);
+    unsigned char* base = (unsigned char*)st->d_mem;
+    if (dense) {
+        ds.pi = base + pi_slot * mat;
+        ds.piT = base + (pi_slot + 1) * mat;
+    }
+    if (prod) {
+        ds.s = base + s_slot * mat;
+        ds.sT = base + (s_slot + 1) * mat;
+    }
+    return TQ_OK;
+}
+
+double stored_value(double v, int dtype) {
+    return (dtype == TQ_F32) ? (double)(float)v : (double)bf16_round_host((float)v);
+}
+
+int validate_params(const tq_params* p) {
+    if (!p) return TQ_EINVAL;
+    if (p->mode != TQ_MSE && p->mode != TQ_PROD) return TQ_EINVAL;
+    if (p->rot != TQ_ROT_DENSE && p->rot != TQ_ROT_RHT) return TQ_EINVAL;
+    if (p->mat_dtype != TQ_F32 && p->mat_dtype != TQ_BF16) return TQ_EINVAL;
+    if (p->d < 2 || p->d > kMaxDim) return p->d < 2 ? TQ_EINVAL : TQ_EUNSUPPORTED;
+    if (p->mode == TQ_MSE && (p->b < 1 || p->b > 8)) return TQ_EINVAL;
+    if (p->mode == TQ_PROD && (p->b < 1 || p->b > 9)) return TQ_EINVAL;
+    if (p->device < 0) return TQ_EINVAL;
+    if (p->rot == TQ_ROT_RHT && !is_pow2(p->d)) return TQ_EUNSUPPORTED;
+    if (!kernel_dim_supported(p->d)) return TQ_EUNSUPPORTED;
+    return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_status_string(int status) {
+    switch (status) {
+        case TQ_OK: return "ok";
+        case TQ_EINVAL: return "invalid argument";
+        case TQ_EUNSUPPORTED: return "unsupported configuration";
+        case TQ_ENOMEM: return "out of memory or workspace too small";
+        case TQ_ECUDA: return "CUDA runtime error";
+        case TQ_EDEVICE: return "device-side error";
+        default: return "unknown status";
+    }
+}
+
+int tq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int tq_version(void) { return 100; }
+
+int tq_build_codebook(int d, int b, double* h_c, double* h_t, double* h_dmse) {
+    if (d < 2 || b < 1 || b > 8) return TQ_EINVAL;
+    return build_codebook(d, b, h_c, h_t, h_dmse);
+}
+
+int tq_draw_gaussian(uint64_t seed, size_t count, double* h_out) {
+    if (!h_out && count) return TQ_EINVAL;
+    philox_gaussian(seed, count, h_out);
+    return TQ_OK;
+}
+
+int tq_draw_signs(uint64_t seed, size_t count, int8_t* h_out) {
+    if (!h_out && count) return TQ_EINVAL;
+    philox_signs(seed, count, h_out);
+    return TQ_OK;
+}
+
+int tq_haar_rotation(int d, const double* h_g, double* h_pi) {
+    if (d < 2 || !h_g || !h_pi) return TQ_EINVAL;
+    return haar_from_gaussian(d, h_g, h_pi);
+}
+
+int tq_state_create(const tq_params* p, const double* h_gauss_pi, const int8_t* h_signs,
+                    const double* h_s, tq_state** out) {
+    if (!out) return TQ_EINVAL;
+    *out = nullptr;
+    int rc = validate_params(p);
+    if (rc != TQ_OK) return rc;
+    tq_state* st = new (std::nothrow) tq_state();
+    if (!st) return TQ_ENOMEM;
+    st->p = *p;
+    const int d = p->d;
+    st->b_mse = (p->mode == TQ_MSE) ? p->b : p->b - 1;
+    const int L = 1 << st->b_mse;
+    st->centroids.assign(L, 0.0);
+    st->bounds.assign(L > 1 ? L - 1 : 0, 0.0);
+    if (st->b_mse > 0) {
+        rc = build_codebook(d, st->b_mse, st->centroids.data(), st->bounds.data(), &st->dmse);
+    } else {
+        st->dmse = 1.0;   // 0-bit MSE: x~_mse = 0, D = E||y||^2 = 1
+    }
+    if (rc != TQ_OK) {
+        delete st;
+        return rc;
+    }
+    if (p->rot == TQ_ROT_DENSE) {
+        std::vector<double> g;
+        const double* gp = h_gauss_pi;
+        if (!gp) {
+            g.resize((size_t)d * d);
+            philox_gaussian(p->seed_pi, g.size(), g.data());
+            gp = g.data();
+        }
+        st->pi.resize((size_t)d * d);
+        rc = haar_from_gaussian(d, gp, st->pi.data());
+        if (rc != TQ_OK) {
+            delete st;
+            return rc;
+        }
+        for (double& v : st->pi) v = stored_value(v, p->mat_dtype);
+    } else {
+        st->signs.resize(d);
+        if (h_signs) {
+            for (int j = 0; j < d; ++j) {
+                if (h_signs[j] != 1 && h_signs[j] != -1) {
+                    delete st;
+                    return TQ_EINVAL;
+                }
+                st->signs[j] = h_signs[j];
+            }
+        } else {
+            philox_signs(p->seed_pi, d, st->signs.data());
+        }
+    }
+    if (p->mode == TQ_PROD) {
+        st->s.resize((size_t)d * d);
+        if (h_s) {
+            for (size_t i = 0; i < st->s.size(); ++i) {
+                if (!std::isfinite(h_s[i])) {
+                    delete st;
+                    return TQ_EINVAL;
+                }
+                st->s[i] = h_s[i];
+            }
+        } else {
+            philox_gaussian(p->seed_s, st->s.size(), st->s.data());
+        }
+        for (double& v : st->s) v = stored_value(v, p->mat_dtype);
+    }
+    rc = finish_state(st);
+    if (rc != TQ_OK) {
+        tq_state_destroy(st);
+        return rc;
+    }
+    *out = st;
+    return TQ_OK;
+}
+
+int tq_state_destroy(tq_state* st) {
+    if (!st) return TQ_OK;
+    int rc = TQ_OK;
+    if (st->d_mem) {
+        DeviceGuard g(st->p.device);
+        cudaError_t e = cudaFree(st->d_mem);
+        if (e != cudaSuccess) rc = cuda_status(e);
+    }
+    delete st;
+    return rc;
+}
+
+int tq_state_params(const tq_state* st, tq_params* out) {
+    if (!st || !out) return TQ_EINVAL;
+    *out = st->p;
+    return TQ_OK;
+}
+
+int tq_state_codebook_info(const tq_state* st, int* b_mse, double* dmse) {
+    if (!st) return TQ_EINVAL;
+    if (b_mse) *b_mse = st->b_mse;
+    if (dmse) *dmse = st->dmse;
+    return TQ_OK;
+}
+
+int tq_state_copy(const tq_state* st, int field, double* h_out, size_t count) {
+    if (!st || !h_out) return TQ_EINVAL;
+    switch (field) {
+        case TQ_FIELD_CENTROIDS:
+            if (count < st->centroids.size()) return TQ_EINVAL;
+            std::copy(st->centroids.begin(), st->centroids.end(), h_out);
+            return TQ_OK;
+        case TQ_FIELD_BOUNDS:
+            if (count < st->bounds.size()) return TQ_EINVAL;
+            std::copy(st->bounds.begin(), st->bounds.end(), h_out);
+            return TQ_OK;
+        case TQ_FIELD_PI:
+            if (st->pi.empty() || count < st->pi.size()) return TQ_EINVAL;
+            std::copy(st->pi.begin(), st->pi.end(), h_out);
+            return TQ_OK;
+        case TQ_FIELD_SIGNS:
+            if (st->signs.empty() || count < st->signs.size()) return TQ_EINVAL;
+            for (size_t i = 0; i < st->signs.size(); ++i) h_out[i] = st->signs[i];
+            return TQ_OK;
+        case TQ_FIELD_S:
+            if (st->s.empty() || count < st->s.size()) return TQ_EINVAL;
+            std::copy(st->s.begin(), st->s.end(), h_out);
+            return TQ_OK;
+        default:
+            return TQ_EINVAL;
+    }
+}
+
+// Export format (little-endian host layout): magic "TQS1", tq_params, b_mse, dmse,
+// then the sizes and contents of centroids, bounds, pi, signs, s.
+int tq_state_export(const tq_state* st, void* h_buf, size_t* bytes) {
+    if (!st || !bytes) return TQ_EINVAL;
+    const size_t need = 4 + sizeof(tq_params) + sizeof(int32_t) + sizeof(double) + 5 * sizeof(uint64_t) +
+                        8 * (st->centroids.size() + st->bounds.size() + st->pi.size() + st->s.size()) +
+                        st->signs.size();
+    if (!h_buf) {
+        *bytes = need;
+        return TQ_OK;
+    }
+    if (*bytes < need) {
+        *bytes = need;
+        return TQ_ENOMEM;
+    }
+    unsigned char* o = (unsigned char*)h_buf;
+    auto put = [&](const void* src, size_t n) {
+        std::memcpy(o, src, n);
+        o += n;
+    };
+    put("TQS1", 4);
+    put(&st->p, sizeof(tq_params));
+    int32_t bm = st->b_mse;
+    put(&bm, sizeof(bm));
+    put(&st->dmse, sizeof(double));
+    uint64_t sz[5] = {st->centroids.size(), st->bounds.size(), st->pi.size(), st->signs.size(), st->s.size()};
+    put(sz, sizeof(sz));
+    put(st->centroids.data(), 8 * sz[0]);
+    put(st->bounds.data(), 8 * sz[1]);
+    put(st->pi.data(), 8 * sz[2]);
+    put(st->signs.data(), sz[3]);
+    put(st->s.data(), 8 * sz[4]);
+    *bytes = need;
+    return TQ_OK;
+}
+
+int tq_state_import(const void* h_buf, size_t bytes, int device, tq_state** out) {
+    if (!h_buf || !out) return TQ_EINVAL;
+    *out = nullptr;
+    const unsigned char* in = (const unsigned char*)h_buf;
+    const unsigned char* end = in + bytes;
+    auto get = [&](void* dst, size_t n) -> bool {
+        if ((size_t)(end - in) < n) return false;
+        std::memcpy(dst, in, n);
+        in += n;
+        return true;
+    };
+    char magic[4];
+    tq_params p;
+    int32_t bm;
+    double dmse;
+    uint64_t sz[5];
+    if (!get(magic, 4) || std::memcmp(magic, "TQS1", 4) != 0) return TQ_EINVAL;
+    if (!get(&p, sizeof(p)) || !get(&bm, sizeof(bm)) || !get(&dmse, sizeof(dmse)) || !get(sz, sizeof(sz)))
+        return TQ_EINVAL;
+    if (device >= 0) p.device = device;
+    int rc = validate_params(&p);
+    if (rc != TQ_OK) return rc;
+    const size_t d2 = (size_t)p.d * p.d;
+    const int want_bm = (p.mode == TQ_MSE) ? p.b : p.b - 1;
+    if (bm != want_bm || sz[0] != (1ull << bm) || sz[1] != (sz[0] - 1) ||
+        sz[2] != (p.rot == TQ_ROT_DENSE ? d2 : 0) || sz[3] != (p.rot == TQ_ROT_RHT ? (size_t)p.d : 0) ||
+        sz[4] != (p.mode == TQ_PROD ? d2 : 0))
+        return TQ_EINVAL;
+    tq_state* st = new (std::nothrow) tq_state();
+    if (!st) return TQ_ENOMEM;
+    st->p = p;
+    st->b_mse = bm;
+    st->dmse = dmse;
+    st->centroids.resize(sz[0]);
+    st->bounds.resize(sz[1]);
+    st->pi.resize(sz[2]);
+    st->signs.resize(sz[3]);
+    st->s.resize(sz[4]);
+    bool ok = get(st->centroids.data(), 8 * sz[0]) && get(st->bounds.data(), 8 * sz[1]) &&
+              get(st->pi.data(), 8 * sz[2]) && get(st->signs.data(), sz[3]) && get(st->s.data(), 8 * sz[4]);
+    if (!ok) {
+        delete st;
+        return TQ_EINVAL;
+    }
+    rc = finish_state(st);
+    if (rc != TQ_OK) {
+        tq_state_destroy(st);
+        return rc;
+    }
+    *out = st;
+    return TQ_OK;
+}
+
+int tq_code_layout(const tq_state* st, size_t* code_bytes, size_t* qjl_bytes) {
+    if (!st) return TQ_EINVAL;
+    if (code_bytes) *code_bytes = (size_t)st->dev.code_bytes;
+    if (qjl_bytes) *qjl_bytes = (size_t)st->dev.qjl_bytes;
+    return TQ_OK;
+}
+
+int tq_quantize_mse(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
+                    uint8_t* codes, float* norms, void* stream) {
+    if (!st || st->p.mode != TQ_MSE) return TQ_EINVAL;
+    int rc = check_vectors(st, x, dtype, n, ld);
+    if (rc != TQ_OK || n == 0) return rc;
+    if (!codes || !norms || !aligned16(codes) || !aligned16(norms)) return TQ_EINVAL;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, nullptr, norms, nullptr, stream));
+}
+
+int tq_quantize_prod(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
+                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+    if (!st || st->p.mode != TQ_PROD) return TQ_EINVAL;
+    int rc = check_vectors(st, x, dtype, n, ld);
+    if (rc != TQ_OK || n == 0) return rc;
+    if ((st->b_mse > 0 && (!codes || !aligned16(codes))) || !qjl || !norms || !rnorms ||
+        !aligned16(qjl) || !aligned16(norms) || !aligned16(rnorms))
+        return TQ_EINVAL;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, qjl, norms, rnorms, stream));
+}
+
+int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
+               const float* rnorms, int64_t n, float* out, void* stream) {
+    if (!st || n < 0) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    const bool prod = st->p.mode == TQ_PROD;
+    if ((st->b_mse > 0 && !codes) || !norms || !out || (prod && (!qjl || !rnorms))) return TQ_EINVAL;
+    if (!aligned16(out)) return TQ_EINVAL;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_dequant(st->dev, codes, prod ? qjl : nullptr, norms,
+                                                   prod ? rnorms : nullptr, n, out, stream));
+}
+
+int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int64_t nq,
+             const uint8_t* codes, const uint8_t* qjl, const float* norms, const float* rnorms,
+             int64_t n, float* scores, void* stream) {
+    if (!st || groups < 0 || nq < 0 || n < 0) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (groups == 0 || nq == 0 || n == 0) return TQ_OK;
+    if (groups > 65535) return TQ_EUNSUPPORTED;
+    const bool prod = st->p.mode == TQ_PROD;
+    if (!q || !scores || !norms || (st->b_mse > 0 && !codes) || (prod && (!qjl || !rnorms)))
+        return TQ_EINVAL;
+    if (!aligned16(q)) return TQ_EINVAL;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_score(st->dev, q, qdtype, groups, nq, codes, prod ? qjl : nullptr,
+                                                 norms, prod ? rnorms : nullptr, n, scores, stream));
+}
+
+int tq_attend_workspace(const tq_state* ks, const tq_state* vs, int H, int64_t T, size_t* bytes) {
+    if (!ks || !vs || !bytes || H < 0 || T < 0) return TQ_EINVAL;
+    *bytes = attend_workspace_bytes(ks->dev, H, T);
+    return TQ_OK;
+}
+
+int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H,
+                     int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                     const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,
+                     float* out, void* workspace, size_t ws_bytes, void* stream) {
+    if (!ks || !vs || H < 0 || T < 0) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (vs->p.mode != TQ_MSE || ks->p.d != vs->p.d || ks->p.device != vs->p.device) return TQ_EINVAL;
+    if (!std::isfinite(scale)) return TQ_EINVAL;
+    if (H == 0) return TQ_OK;
+    if (T == 0) return TQ_EINVAL;   // softmax over no tokens is undefined
+    const bool prod = ks->p.mode == TQ_PROD;
+    if (!q || !out || !knorms || !vnorms || (ks->b_mse > 0 && !kcodes) || !vcodes ||
+        (prod && (!kqjl || !krnorms)))
+        return TQ_EINVAL;
+    if (!aligned16(q) || !aligned16(out)) return TQ_EINVAL;
+    const size_t need = attend_workspace_bytes(ks->dev, H, T);
+    if (need > 0 && (!workspace || ((uintptr_t)workspace & 255u))) return TQ_EINVAL;
+    if (ws_bytes < need) return TQ_ENOMEM;
+    DeviceGuard g(ks->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, kcodes, prod ? kqjl : nullptr,
+                                                  knorms, prod ? krnorms : nullptr, vcodes, vnorms, scale, out,
+                                                  workspace, ws_bytes, stream));
+}
+
+int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes) {
+    if (!st || !bytes || nq < 0 || n < 0 || k < 1 || k > 64) return TQ_EINVAL;
+    *bytes = search_workspace_bytes(st->dev, nq, n, k);
+    return TQ_OK;
+}
+
+int tq_search_topk(const tq_state* st, const void* q, int qdtype, int64_t nq, const uint8_t* codes,
+                   const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int k,
+                   int64_t* idx, float* vals, void* workspace, size_t ws_bytes, void* stream) {
+    if (!st || nq < 0 || n < 0 || k < 1 || k > 64) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (nq == 0) return TQ_OK;
+    if (k > n) return TQ_EINVAL;
+    const bool prod = st->p.mode == TQ_PROD;
+    if (!q || !idx || !vals || !norms || (st->b_mse > 0 && !codes) || (prod && (!qjl || !rnorms)))
+        return TQ_EINVAL;
+    if (!aligned16(q)) return TQ_EINVAL;
+    const size_t need = search_workspace_bytes(st->dev, nq, n, k);
+    if (need > 0 && (!workspace || ((uintptr_t)workspace & 255u))) return TQ_EINVAL;
+    if (ws_bytes < need) return TQ_ENOMEM;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_search(st->dev, q, qdtype, nq, codes, prod ? qjl : nullptr, norms,
+                                                  prod ? rnorms : nullptr, n, k, idx, vals, workspace, ws_bytes,
+                                                  stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,83 @@
+// Internal declarations shared by the host library and the kernels of libtq.
+// Not part of the public ABI (include/tq.h is).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kMaxLevels = 256;      // 2^b_mse with b_mse <= 8
+constexpr int kMaxDim = 2048;        // largest d the kernels accept
+
+// Everything a kernel needs about a state, passed by value as a kernel parameter
+// (lives in the constant bank: uniform reads of the codebook are broadcasts).
+struct DevState {
+    int d;
+    int b_mse;          // bits of MSE code per coordinate (0 for prod b=1)
+    int L;              // 2^b_mse
+    int mode;           // TQ_MSE / TQ_PROD
+    int rot;            // TQ_ROT_DENSE / TQ_ROT_RHT
+    int mat_dtype;      // TQ_F32 / TQ_BF16
+    int code_bytes;     // ceil(b_mse*d/8)
+    int qjl_bytes;      // d/8 (prod) or 0
+    float qjl_scale;    // sqrt(pi/2)/d
+    float rsqrt_d;      // 1/sqrt(d) (RHT normalisation)
+    const void* pi;     // Pi, row-major [d][d] (dense)
+    const void* piT;    // Pi^T, row-major [d][d] (dense)
+    const void* s;      // S, row-major [d][d] (prod)
+    const void* sT;     // S^T, row-major [d][d] (prod)
+    uint32_t signs[kMaxDim / 32];  // RHT: bit j set <=> eps_j = -1
+    float c[kMaxLevels];           // centroids (fp32 stored values)
+    float t[kMaxLevels];           // boundaries t[0..L-2]
+};
+
+}  // namespace tq
+
+struct tq_state {
+    tq_params p;
+    int b_mse;
+    double dmse;
+    std::vector<double> centroids;   // fp64 Lloyd-Max centroids
+    std::vector<double> bounds;      // fp64 boundaries
+    std::vector<double> pi;          // stored Pi values (after rounding), row-major
+    std::vector<int8_t> signs;       // RHT signs
+    std::vector<double> s;           // stored S values (after rounding), row-major
+    void* d_mem = nullptr;           // one device allocation holding pi, piT, s, sT
+    tq::DevState dev;                // kernel view
+};
+
+namespace tq {
+
+// ---- host helpers (host.cpp / codebook.cpp / linalg.cpp) ----
+int build_codebook(int d, int b, double* c, double* t, double* dmse);
+void philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+void philox_gaussian(uint64_t seed, size_t count, double* out);
+void philox_signs(uint64_t seed, size_t count, int8_t* out);
+int haar_from_gaussian(int d, const double* g, double* pi_out);
+float bf16_round_host(float x);
+void set_cuda_error(int err);
+
+// ---- kernel launchers (kernels .cu files); all return a cudaError_t value ----
+int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld,
+                  uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl,
+                   const float* norms, const float* rnorms, int64_t n, float* out, void* stream);
+int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq,
+                 const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                 const float* rnorms, int64_t n, float* scores, void* stream);
+size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
+int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
+                  int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                  const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,
+                  float* out, void* ws, size_t ws_bytes, void* stream);
+size_t search_workspace_bytes(const DevState& st, int64_t nq, int64_t n, int k);
+int launch_search(const DevState& st, const void* q, int qdtype, int64_t nq,
+                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                  const float* rnorms, int64_t n, int k, int64_t* idx, float* vals, void* ws,
+                  size_t ws_bytes, void* stream);
+
+}  // namespace tq
