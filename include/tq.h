@@ -102,6 +102,13 @@ const char* tq_status_string(int status);
 /* cudaError_t value of the calling thread's last TQ_ECUDA (0 if none). */
 int tq_last_cuda_error(void);
 
+/*
+ * Synchronise `device` and report kernel-side errors: TQ_EDEVICE if a kernel of this
+ * library gave up a bounded wait (it then recorded an error word and returned without
+ * finishing); the word is cleared by this call. TQ_OK otherwise; TQ_ECUDA on a CUDA error.
+ */
+int tq_device_status(int device);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int tq_version(void);
 

@@ -273,3 +273,24 @@ def test_search_topk_small():
                 assert est[i, gi[i, j]] >= kth - ABS_SCORE   # a swap at the cut is allowed
         np.testing.assert_allclose(gv[i], est[i, gi[i]], atol=ABS_SCORE)
         assert np.all(np.diff(gv[i]) <= 0)
+
+
+# --------------------------------------------------------------------------------------
+# The tensor-core encoder (d = 128, RHT, bf16 input): tails of every size, strided rows.
+# --------------------------------------------------------------------------------------
+@pytest.mark.parametrize("b,mode", [(2, 1), (3, 1), (4, 1), (1, 0), (2, 0), (3, 0), (4, 0)])
+@pytest.mark.parametrize("n,pad", [(1, 0), (127, 8), (129, 0), (5000, 8)])
+def test_tc_encoder(b, mode, n, pad):
+    d = 128
+    pair = Pair(tq, d, b, mode, tq.ROT_RHT, tq.BF16)
+    bits = synth.kv_prefill_batch(1, n, d, seed=31 + n)[0]
+    buf = np.zeros((n, d + pad), np.uint16)
+    buf[:, :d] = bits
+    xd = dev_bf16(buf)[:, :d]
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    gpu, gplanes = gpu_encode(pair, xd, n)
+    tq.device_status(0)
+    bad = check_codes(pair, gpu, enc)
+    xt_o = pair.decode(enc)
+    xt_g = gpu_dequant(pair, gplanes, n)
+    assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2

@@ -66,6 +66,7 @@ _SIGS = {
     "tq_status_string": (ctypes.c_char_p, [_I]),
     "tq_last_cuda_error": (_I, []),
     "tq_version": (_I, []),
+    "tq_device_status": (_I, [_I]),
     "tq_build_codebook": (_I, [_I, _I, _DP, _DP, _DP]),
     "tq_draw_gaussian": (_I, [ctypes.c_uint64, _SZ, _DP]),
     "tq_draw_signs": (_I, [ctypes.c_uint64, _SZ, _P]),
@@ -95,6 +96,11 @@ for _name, (_res, _args) in _SIGS.items():
 
 def lib():
     return _lib
+
+
+def device_status(device: int = 0):
+    """Synchronise `device`; raise TQError(TQ_EDEVICE) if a kernel recorded an error."""
+    _check(_lib.tq_device_status(device), "tq_device_status")
 
 
 def declared_symbols(header: str = HEADER_PATH):

@@ -1,0 +1,427 @@
+// Tensor-core encoder for d = 128 with the randomized Hadamard rotation and bf16 input
+// (TurboQuant_prod with S stored bf16, or TurboQuant_mse).
+//
+// TurboQuant review (Jump2Paper): Theorem 1 (rotate, per-coordinate Lloyd-Max code),
+// Definition 1 + Theorem 2 (QJL signs of S r on the residual, ||r|| kept); AI Trends
+// summary of the TurboQuant video (L2 normalise + RHT).
+//
+// Layout of the work: a CTA of 128 threads owns tiles of 128 vectors; thread t is vector t
+// of the tile, which is also TMEM lane t of the MMA accumulator.
+//   1. TMA (128-byte swizzle) brings the tile's bf16 rows into shared memory, two stages
+//      deep, so the next tile streams in while this one is computed.
+//   2. Each thread reads its row, flips the RHT signs on the packed bf16 bits, converts to
+//      fp32, takes ||x||, runs the 7-stage Walsh-Hadamard butterfly in registers (paired
+//      fp32 adds), scales by 1/(sqrt(d) ||x||), quantizes against the Lloyd-Max boundaries,
+//      and writes codes and norms.
+//   3. prod: the residual r = y - c[idx] is split as r = hi + lo (both bf16, lo = bf16(r - hi))
+//      and written to TMEM as the MMA A operand; one thread issues 16 tcgen05.mma
+//      (K = 128 for hi, then for lo) against S held in shared memory (K-major core
+//      matrices), accumulating S r in fp32 in TMEM. The split keeps the error of S r at
+//      about 2^-16 |S||r|, so a sign is decided as fp32 arithmetic on r would decide it.
+//   4. Each thread reads its 128 accumulator columns back (tcgen05.ld) and packs the signs
+//      [(S r)_j >= 0] into 16 bytes.
+// Every wait is bounded; on a timeout the kernel records an error word and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace tq {
+
+__device__ int g_tq_device_error = 0;
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kD = 128;
+constexpr uint32_t kTmemCols = 256;   // [0,128) accumulator, [128,192) A hi, [192,256) A lo
+
+struct TcParams {
+    uint8_t* codes;
+    uint8_t* qjl;
+    float* norms;
+    float* rnorms;
+    const uint16_t* s;        // S, bf16, row-major [128][128]
+    int64_t n;
+    float rsqrt_d;
+    float t[16];              // boundaries
+    float c[16];              // centroids
+    uint32_t sgn[64];         // XOR mask per bf16 pair: bit 15 / bit 31 flip elements 2i / 2i+1
+};
+
+struct __align__(1024) TcSmem {
+    uint8_t x[2][2][kTile * 128];   // [stage][half]: 128 rows x 128 bytes, 128B-swizzled
+    uint8_t s[kD * kD * 2];         // S as the B operand: K-major core matrices
+    uint64_t bar_x[2];
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int pad;
+};
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// Walsh-Hadamard butterfly over 128 values held as 64 float2 (v[i] = elements 2i, 2i+1).
+__device__ __forceinline__ void fwht128(float2 (&v)[64]) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float a = v[i].x, b = v[i].y;
+        v[i] = f2(a + b, a - b);
+    }
+    const float2 m1 = f2(-1.f, -1.f);
+#pragma unroll
+    for (int k = 1; k < 64; k <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if ((i & k) == 0) {
+                const float2 a = v[i], b = v[i + k];
+                v[i] = __fadd2_rn(a, b);
+                v[i + k] = __ffma2_rn(b, m1, a);
+            }
+        }
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void put_code(uint32_t (&cw)[4 * (B > 0 ? B : 1)], int j, uint32_t code) {
+    const int bit = j * B;
+    const int w = bit >> 5, sh = bit & 31;
+    cw[w] |= code << sh;
+    if (sh + B > 32) cw[w + 1] |= code >> (32 - sh);
+}
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(kTile, 2)
+encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem& sm = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int64_t ntiles = (p.n + kTile - 1) / kTile;
+
+    if (tid == 0) {
+        ptx::prefetch_tmap(&tmap);
+        ptx::mbar_init(&sm.bar_x[0], 1);
+        ptx::mbar_init(&sm.bar_x[1], 1);
+        ptx::mbar_init(&sm.bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    if constexpr (PROD) {
+        if (warp == 0) {
+            ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
+            ptx::tmem_relinquish();
+        }
+        // S into shared memory: chunk c (8 values along K) of row n at c*2048 + (n/8)*128 + (n%8)*16
+        for (int i = tid; i < kD * 16; i += kTile) {
+            const int row = i >> 4, c = i & 15;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.s + row * kD + c * 8));
+            *reinterpret_cast<uint4*>(sm.s + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
+        }
+        ptx::fence_proxy_async_smem();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = PROD ? sm.tmem_base : 0u;
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+
+    auto issue = [&](int stg, int64_t tile) {
+        ptx::mbar_arrive_expect_tx(&sm.bar_x[stg], 2 * kTile * 128);
+        ptx::tma_load_2d(sm.x[stg][0], &tmap, 0, (int)(tile * kTile), &sm.bar_x[stg]);
+        ptx::tma_load_2d(sm.x[stg][1], &tmap, 64, (int)(tile * kTile), &sm.bar_x[stg]);
+    };
+    uint32_t pending = 0u;   // bit s: a load into stage s is in flight
+    const int64_t t0 = blockIdx.x;
+    if (t0 < ntiles) {
+        if (tid == 0) issue(0, t0);
+        pending |= 1u;
+    }
+    if (t0 + gridDim.x < ntiles) {
+        if (tid == 0) issue(1, t0 + gridDim.x);
+        pending |= 2u;
+    }
+    uint32_t xphase = 0u;    // bit s: parity of the next phase of stage s
+    uint32_t mphase = 0u;
+    bool failed = false;
+    const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
+    const uint32_t s_addr = ptx::smem_addr(sm.s);
+
+    int it = 0;
+    for (int64_t tile = t0; tile < ntiles; tile += gridDim.x, ++it) {
+        const int stg = it & 1;
+        const bool ok = ptx::mbar_wait(&sm.bar_x[stg], (xphase >> stg) & 1u);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        xphase ^= 1u << stg;
+        pending &= ~(1u << stg);
+        // ---- read this thread's row (undo the 128-byte swizzle) ----
+        uint32_t w[64];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint8_t* base = sm.x[stg][h] + tid * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4*>(base + ((c ^ (tid & 7)) << 4));
+                w[h * 32 + c * 4 + 0] = q.x;
+                w[h * 32 + c * 4 + 1] = q.y;
+                w[h * 32 + c * 4 + 2] = q.z;
+                w[h * 32 + c * 4 + 3] = q.w;
+            }
+        }
+        __syncthreads();   // every thread has its row: the stage can be refilled
+        const int64_t nxt = tile + 2 * (int64_t)gridDim.x;
+        if (nxt < ntiles) {
+            if (tid == 0) issue(stg, nxt);
+            pending |= 1u << stg;
+        }
+        // ---- signs, fp32, norm ----
+        float2 v[64];
+        float2 ss = f2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const uint32_t u = w[i] ^ p.sgn[i];
+            v[i] = f2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+            ss = __ffma2_rn(v[i], v[i], ss);
+        }
+        const float nu = sqrtf(ss.x + ss.y);
+        fwht128(v);
+        const float sc = (nu > 0.f) ? p.rsqrt_d / nu : 0.f;
+        const float2 sc2 = f2(sc, sc);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = __fmul2_rn(v[i], sc2);
+
+        // ---- quantize, residual ----
+        constexpr int NW = 4 * (B > 0 ? B : 1);
+        uint32_t cw[NW];
+#pragma unroll
+        for (int i = 0; i < NW; ++i) cw[i] = 0u;
+        float2 rr2 = f2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            float r[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float y = e ? v[i].y : v[i].x;
+                const int j = 2 * i + e;
+                uint32_t code;
+                float cv;
+                if constexpr (B == 2) {
+                    // symmetric 4-level codebook: sign and |y| >= t_2
+                    // cells: y < t0 = -t2 | t0 <= y < 0 | 0 <= y < t2 | t2 <= y (upper cell on a tie)
+                    const uint32_t neg = __float_as_uint(y) >> 31;
+                    const bool big = (y >= p.t[2]) | (y < p.t[0]);
+                    const float mag = big ? p.c[3] : p.c[2];
+                    code = ((neg ^ 1u) << 1) | ((uint32_t)big ^ neg);
+                    cv = __uint_as_float(__float_as_uint(mag) | (neg << 31));
+                } else if constexpr (B == 1) {
+                    const uint32_t neg = __float_as_uint(y) >> 31;
+                    code = neg ^ 1u;
+                    cv = __uint_as_float(__float_as_uint(p.c[1]) | (neg << 31));
+                } else {
+                    code = 0;
+                    cv = p.c[0];
+#pragma unroll
+                    for (int k = 0; k < (1 << B) - 1; ++k) {
+                        if (y >= p.t[k]) {
+                            code = k + 1;
+                            cv = p.c[k + 1];
+                        }
+                    }
+                }
+                put_code<B>(cw, j, code);
+                r[e] = (nu > 0.f) ? (y - cv) : 0.f;
+            }
+            v[i] = f2(r[0], r[1]);
+            rr2 = __ffma2_rn(v[i], v[i], rr2);
+        }
+        const int64_t row = tile * kTile + tid;
+        if (row < p.n) {
+            uint4* co = reinterpret_cast<uint4*>(p.codes + row * (16 * B));
+#pragma unroll
+            for (int q = 0; q < B; ++q) co[q] = make_uint4(cw[4 * q], cw[4 * q + 1], cw[4 * q + 2], cw[4 * q + 3]);
+            p.norms[row] = nu;
+            if constexpr (PROD) p.rnorms[row] = sqrtf(rr2.x + rr2.y);
+        }
+        if constexpr (PROD) {
+            // ---- A = [hi | lo] into TMEM columns 128.. ----
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                uint32_t hi[32], lo[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float2 r = v[part * 32 + q];
+                    const __nv_bfloat162 h = __float22bfloat162_rn(r);
+                    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+                    const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
+                    const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), r);
+                    const __nv_bfloat162 lb = __float22bfloat162_rn(l);
+                    hi[q] = hb;
+                    lo[q] = *reinterpret_cast<const uint32_t*>(&lb);
+                }
+                ptx::tmem_st32(t_lane + 128 + part * 32, hi);
+                ptx::tmem_st32(t_lane + 192 + part * 32, lo);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 128 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 192 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, 1u);
+                ptx::mma_commit(&sm.bar_mma);
+            }
+            const bool mok = ptx::mbar_wait(&sm.bar_mma, mphase);
+            if (__syncthreads_or(!mok)) {
+                failed = true;
+                break;
+            }
+            mphase ^= 1u;
+            ptx::tc_fence_after();
+            // ---- signs of S r ----
+            uint32_t zw[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t acc[32];
+                ptx::tmem_ld32(t_lane + q * 32, acc);
+                ptx::tmem_wait_ld();
+                uint32_t word = 0u;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) word |= (__uint_as_float(acc[j]) >= 0.f ? 1u : 0u) << j;
+                zw[q] = word;
+            }
+            ptx::tc_fence_before();
+            if (row < p.n) *reinterpret_cast<uint4*>(p.qjl + row * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+        }
+    }
+    if (failed) {
+        if (tid == 0) atomicExch(&g_tq_device_error, 1);
+        // let copies in flight land before the shared memory goes away (bounded)
+        for (int s2 = 0; s2 < 2; ++s2)
+            if ((pending >> s2) & 1u) (void)ptx::mbar_wait(&sm.bar_x[s2], (xphase >> s2) & 1u);
+        if (PROD) (void)ptx::mbar_wait(&sm.bar_mma, mphase, 100000000ull);
+    }
+    __syncthreads();
+    if constexpr (PROD) {
+        if (warp == 0) {
+            ptx::tc_fence_after();
+            ptx::tmem_dealloc(tmem, kTmemCols);
+        }
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+int sm_count() {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+template <int B, bool PROD>
+int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl, float* norms,
+              float* rnorms, cudaStream_t stream) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return (int)cudaErrorNotSupported;
+    CUtensorMap tmap;
+    const cuuint64_t gdim[2] = {(cuuint64_t)kD, (cuuint64_t)n};
+    const cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {64, kTile};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
+    TcParams p;
+    p.codes = codes;
+    p.qjl = qjl;
+    p.norms = norms;
+    p.rnorms = rnorms;
+    p.s = reinterpret_cast<const uint16_t*>(st.s);
+    p.n = n;
+    p.rsqrt_d = st.rsqrt_d;
+    for (int i = 0; i < 16; ++i) {
+        p.t[i] = (i < st.L - 1) ? st.t[i] : 0.f;
+        p.c[i] = (i < st.L) ? st.c[i] : 0.f;
+    }
+    for (int i = 0; i < 64; ++i) {
+        const bool n0 = (st.signs[(2 * i) >> 5] >> ((2 * i) & 31)) & 1u;
+        const bool n1 = (st.signs[(2 * i + 1) >> 5] >> ((2 * i + 1) & 31)) & 1u;
+        p.sgn[i] = (n0 ? 0x8000u : 0u) | (n1 ? 0x80000000u : 0u);
+    }
+    const size_t smem = sizeof(TcSmem) + 1024;
+    auto kern = encode_tc_kernel<B, PROD>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    const int64_t ntiles = (n + kTile - 1) / kTile;
+    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * 2);
+    kern<<<grid, kTile, smem, stream>>>(tmap, p);
+    return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+// True when the tensor-core encoder handles this configuration.
+bool encode_tc_supported(const DevState& st, int dtype, int64_t n, int64_t ld) {
+    if (st.d != kD || st.rot != TQ_ROT_RHT || dtype != TQ_BF16) return false;
+    if (n <= 0 || n >= (int64_t)1 << 31 || ld < kD) return false;
+    if (st.mode == TQ_PROD) return st.mat_dtype == TQ_BF16 && st.b_mse >= 1 && st.b_mse <= 3;
+    return st.b_mse >= 1 && st.b_mse <= 4;
+}
+
+int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl,
+                     float* norms, float* rnorms, void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    if (st.mode == TQ_PROD) {
+        switch (st.b_mse) {
+            case 1: return launch_tc<1, true>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+            case 2: return launch_tc<2, true>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+            case 3: return launch_tc<3, true>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+            default: return (int)cudaErrorInvalidValue;
+        }
+    }
+    switch (st.b_mse) {
+        case 1: return launch_tc<1, false>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+        case 2: return launch_tc<2, false>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+        case 3: return launch_tc<3, false>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+        case 4: return launch_tc<4, false>(st, x, n, ld, codes, qjl, norms, rnorms, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+int read_device_error(int* flag) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tq_device_error, sizeof(int));
+    if (e != cudaSuccess) return (int)e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_tq_device_error, &zero, sizeof(int));
+        if (e != cudaSuccess) return (int)e;
+    }
+    *flag = v;
+    return 0;
+}
+
+}  // namespace tq

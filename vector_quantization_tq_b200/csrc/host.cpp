@@ -189,6 +189,18 @@ int tq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int tq_version(void) { return 100; }
 
+int tq_device_status(int device) {
+    if (device < 0) return TQ_EINVAL;
+    DeviceGuard g(device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    int flag = 0;
+    int rc = read_device_error(&flag);
+    if (rc != 0) return cuda_status((cudaError_t)rc);
+    return flag ? TQ_EDEVICE : TQ_OK;
+}
+
 int tq_build_codebook(int d, int b, double* h_c, double* h_t, double* h_dmse) {
     if (d < 2 || b < 1 || b > 8) return TQ_EINVAL;
     return build_codebook(d, b, h_c, h_t, h_dmse);

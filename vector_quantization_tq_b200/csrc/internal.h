@@ -69,6 +69,7 @@ int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl,
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq,
                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
                  const float* rnorms, int64_t n, float* scores, void* stream);
+int read_device_error(int* flag);
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
                   int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
