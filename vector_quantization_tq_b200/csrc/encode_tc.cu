@@ -187,10 +187,7 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
         const float nu = sqrtf(ss.x + ss.y);
         fwht128(v);
-        const float sc = (nu > 0.f) ? p.rsqrt_d / nu : 0.f;
-        const float2 sc2 = f2(sc, sc);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = __fmul2_rn(v[i], sc2);
+        const float sc = (nu > 0.f) ? p.rsqrt_d / nu : 0.f;   // y = sc * (H D x)
 
         // ---- quantize, residual ----
         constexpr int NW = 4 * (B > 0 ? B : 1);
@@ -198,30 +195,66 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 #pragma unroll
         for (int i = 0; i < NW; ++i) cw[i] = 0u;
         float2 rr2 = f2(0.f, 0.f);
+        if constexpr (B <= 2) {
+            // Symmetric codebooks with 2 or 4 levels, decided on the unscaled coordinate:
+            // sign plane N (1 = negative) and, for 4 levels, plane M (1 = |y| below t_2).
+            // Cells (B = 2): y < -t2 | -t2 <= y < 0 | 0 <= y < t2 | t2 <= y.
+            const float T2 = (B == 2 && nu > 0.f) ? p.t[2] / sc : INFINITY;
+            const float cs = (nu > 0.f) ? p.c[B == 2 ? 2 : 1] : 0.f;
+            const float cb = (nu > 0.f) ? p.c[B == 2 ? 3 : 1] : 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            float r[2];
+            for (int g = 0; g < 4; ++g) {
+                uint32_t np = 0u, mp = 0u;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float y = e ? v[i].y : v[i].x;
-                const int j = 2 * i + e;
-                uint32_t code;
-                float cv;
-                if constexpr (B == 2) {
-                    // symmetric 4-level codebook: sign and |y| >= t_2
-                    // cells: y < t0 = -t2 | t0 <= y < 0 | 0 <= y < t2 | t2 <= y (upper cell on a tie)
-                    const uint32_t neg = __float_as_uint(y) >> 31;
-                    const bool big = (y >= p.t[2]) | (y < p.t[0]);
-                    const float mag = big ? p.c[3] : p.c[2];
-                    code = ((neg ^ 1u) << 1) | ((uint32_t)big ^ neg);
-                    cv = __uint_as_float(__float_as_uint(mag) | (neg << 31));
-                } else if constexpr (B == 1) {
-                    const uint32_t neg = __float_as_uint(y) >> 31;
-                    code = neg ^ 1u;
-                    cv = __uint_as_float(__float_as_uint(p.c[1]) | (neg << 31));
+                for (int q = 15; q >= 0; --q) {
+                    const int i = g * 16 + q;
+                    float r[2];
+#pragma unroll
+                    for (int e = 1; e >= 0; --e) {
+                        const float y = e ? v[i].y : v[i].x;
+                        const uint32_t yb = __float_as_uint(y);
+                        np = __funnelshift_l(yb, np, 1);
+                        float mag = cs;
+                        if constexpr (B == 2) {
+                            const float dd = fabsf(y) - T2;
+                            mp = __funnelshift_l(__float_as_uint(dd), mp, 1);
+                            mag = (dd < 0.f) ? cs : cb;
+                        }
+                        const float smag = __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
+                        r[e] = fmaf(y, sc, -smag);
+                    }
+                    v[i] = f2(r[0], r[1]);
+                    rr2 = __ffma2_rn(v[i], v[i], rr2);
+                }
+                if constexpr (B == 1) {
+                    cw[g] = ~np;                       // code = 1 for y >= 0
                 } else {
-                    code = 0;
-                    cv = p.c[0];
+                    const uint32_t hi_bit = ~np;              // bit 1: y >= 0
+                    const uint32_t lo_bit = ~(np ^ mp);       // bit 0: negative XOR small, inverted
+                    auto spread = [](uint32_t x) {
+                        x &= 0xffffu;
+                        x = (x | (x << 8)) & 0x00ff00ffu;
+                        x = (x | (x << 4)) & 0x0f0f0f0fu;
+                        x = (x | (x << 2)) & 0x33333333u;
+                        x = (x | (x << 1)) & 0x55555555u;
+                        return x;
+                    };
+                    cw[2 * g] = spread(lo_bit) | (spread(hi_bit) << 1);
+                    cw[2 * g + 1] = spread(lo_bit >> 16) | (spread(hi_bit >> 16) << 1);
+                }
+            }
+        } else {
+            const float2 sc2 = f2(sc, sc);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = __fmul2_rn(v[i], sc2);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                float r[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float y = e ? v[i].y : v[i].x;
+                    uint32_t code = 0;
+                    float cv = p.c[0];
 #pragma unroll
                     for (int k = 0; k < (1 << B) - 1; ++k) {
                         if (y >= p.t[k]) {
@@ -229,12 +262,12 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                             cv = p.c[k + 1];
                         }
                     }
+                    put_code<B>(cw, 2 * i + e, code);
+                    r[e] = (nu > 0.f) ? (y - cv) : 0.f;
                 }
-                put_code<B>(cw, j, code);
-                r[e] = (nu > 0.f) ? (y - cv) : 0.f;
+                v[i] = f2(r[0], r[1]);
+                rr2 = __ffma2_rn(v[i], v[i], rr2);
             }
-            v[i] = f2(r[0], r[1]);
-            rr2 = __ffma2_rn(v[i], v[i], rr2);
         }
         const int64_t row = tile * kTile + tid;
         if (row < p.n) {
@@ -292,10 +325,10 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                 uint32_t acc[32];
                 ptx::tmem_ld32(t_lane + q * 32, acc);
                 ptx::tmem_wait_ld();
-                uint32_t word = 0u;
+                uint32_t neg = 0u;   // sign bits, collected so that bit j is column j
 #pragma unroll
-                for (int j = 0; j < 32; ++j) word |= (__uint_as_float(acc[j]) >= 0.f ? 1u : 0u) << j;
-                zw[q] = word;
+                for (int j = 31; j >= 0; --j) neg = __funnelshift_l(acc[j], neg, 1);
+                zw[q] = (nu > 0.f) ? ~neg : 0xffffffffu;   // r = 0 -> S r = 0 -> all signs +1
             }
             ptx::tc_fence_before();
             if (row < p.n) *reinterpret_cast<uint4*>(p.qjl + row * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
@@ -334,10 +367,14 @@ EncodeTiledFn encode_tiled_fn() {
 }
 
 int sm_count() {
-    int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return sms > 0 ? sms : 148;
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
 }
 
 template <int B, bool PROD>
@@ -373,8 +410,14 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
     }
     const size_t smem = sizeof(TcSmem) + 1024;
     auto kern = encode_tc_kernel<B, PROD>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return (int)e;
+    static int attr_set_for_device = -1;   // per instantiation
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_set_for_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_set_for_device = dev;
+    }
     const int64_t ntiles = (n + kTile - 1) / kTile;
     const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * 2);
     kern<<<grid, kTile, smem, stream>>>(tmap, p);

@@ -9,6 +9,7 @@
 // (fp32 accumulate), the RHT is an in-register / shuffle / shared-memory butterfly.
 // The specialised tensor-core encoder for d = 128 lives in encode_tc.cu.
 #include "common.cuh"
+#include "prep.cuh"
 
 namespace tq {
 namespace {
@@ -243,56 +244,6 @@ dequant_kernel(const DevState st, const uint8_t* __restrict__ codes, const uint8
     }
 }
 
-// ------------------------------------------------------------------------------------
-// Query preparation inside a block: qp = Pi q and u = S qp for `count` queries
-// (rows of q with stride d, fp32 or bf16) into shared memory [count][d].
-// ------------------------------------------------------------------------------------
-__device__ void prep_queries(const DevState& st, const void* q, int qdtype, int count,
-                             float* qs, float* qp, float* u) {
-    const int d = st.d;
-    for (int i = threadIdx.x; i < count * d; i += blockDim.x)
-        qs[i] = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + i)
-                                   : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + i));
-    __syncthreads();
-    if (st.rot == TQ_ROT_RHT) {
-        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
-            const int j = i % d;
-            qp[i] = rht_neg(st, j) ? -qs[i] : qs[i];
-        }
-        __syncthreads();
-        for (int h = 1; h < d; h <<= 1) {
-            for (int p = threadIdx.x; p < count * d / 2; p += blockDim.x) {
-                const int qi = p / (d / 2), pr = p % (d / 2);
-                const int j = (pr / h) * 2 * h + (pr % h);
-                float* v = qp + qi * d;
-                const float a = v[j], b = v[j + h];
-                v[j] = a + b;
-                v[j + h] = a - b;
-            }
-            __syncthreads();
-        }
-        for (int i = threadIdx.x; i < count * d; i += blockDim.x) qp[i] *= st.rsqrt_d;
-    } else {
-        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
-            const int qi = i / d, j = i % d;
-            float a = 0.f;
-            for (int k = 0; k < d; ++k) a = fmaf(mat_elem(st.piT, st.mat_dtype, (int64_t)k * d + j), qs[qi * d + k], a);
-            qp[i] = a;
-        }
-    }
-    __syncthreads();
-    if (st.mode == TQ_PROD) {
-        for (int i = threadIdx.x; i < count * d; i += blockDim.x) {
-            const int qi = i / d, j = i % d;
-            float a = 0.f;
-            for (int k = 0; k < d; ++k) a = fmaf(mat_elem(st.sT, st.mat_dtype, (int64_t)k * d + j), qp[qi * d + k], a);
-            u[i] = a;
-        }
-    }
-    __syncthreads();
-}
-
-
 // The two sums of an estimate for up to QT queries against one key:
 //   a1 = sum_j qp_j c[idx_j],  a2 = sum_j u_j (2 z_j - 1).
 template <int QT>
@@ -358,7 +309,7 @@ score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t 
     const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
     for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * d) * qelem,
+    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * d) * qelem,
                  qdtype, nqt, qs, qp, u);
     for (int64_t key = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; key < n;
          key += (int64_t)gridDim.x * blockDim.x) {
@@ -405,7 +356,7 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
     for (int i = threadIdx.x; i < ks.L; i += blockDim.x) kc[i] = ks.c[i];
     for (int i = threadIdx.x; i < vs.L; i += blockDim.x) vc[i] = vs.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u);
+    prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u);
 
     const int64_t t_begin = (int64_t)split * chunk;
     const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
@@ -579,7 +530,7 @@ search_block_kernel(const DevState st, const void* __restrict__ q, int qdtype, i
     const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
     for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries(st, reinterpret_cast<const unsigned char*>(q) + (size_t)(q0 * d) * qelem, qdtype, nqt, qs, qp, u);
+    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)(q0 * d) * qelem, qdtype, nqt, qs, qp, u);
     const int64_t k0 = (int64_t)blockIdx.x * block_keys;
     for (int local = threadIdx.x; local < block_keys; local += blockDim.x) {
         const int64_t key = k0 + local;
@@ -729,9 +680,16 @@ int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl,
     }
 }
 
+bool score_lut_supported(const DevState& st);
+int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
+                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                     void* stream);
+
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
                  void* stream) {
+    if (score_lut_supported(st))
+        return launch_score_lut(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, stream);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t smem = score_smem_bytes(st.d);
     if (smem > 48 * 1024) cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

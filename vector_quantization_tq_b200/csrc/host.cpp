@@ -495,7 +495,7 @@ int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int6
     const bool prod = st->p.mode == TQ_PROD;
     if (!q || !scores || !norms || (st->b_mse > 0 && !codes) || (prod && (!qjl || !rnorms)))
         return TQ_EINVAL;
-    if (!aligned16(q)) return TQ_EINVAL;
+    if (!aligned16(q) || (codes && !aligned16(codes)) || (prod && !aligned16(qjl))) return TQ_EINVAL;
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
     return cuda_status((cudaError_t)launch_score(st->dev, q, qdtype, groups, nq, codes, prod ? qjl : nullptr,
