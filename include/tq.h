@@ -216,6 +216,26 @@ int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int 
                      const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                      float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * tq_attend_decode without a workspace argument, for callers that cannot allocate device
+ * memory: runtimes that hand all device memory to their own pool allocator and forbid
+ * other allocations, and latency-critical decode loops where an allocation's cost or
+ * possible failure is not acceptable. (No counterpart on the reference pages: this is an
+ * interface convenience around the decode step above, with the same arguments and result.)
+ * The split partials go to a fixed device array of 4 MiB inside the library, which every
+ * GPU that loads the library holds until the process exits; the entry point itself
+ * allocates nothing. Calls that would need more than 4 MiB of partials
+ * (H * splits * (d + 2) * 4 bytes, see tq_attend_workspace) return TQ_EUNSUPPORTED.
+ * All calls on a device share the array and it keeps the last call's contents, so calls
+ * whose work overlaps on the GPU (concurrent streams or threads) race and must be
+ * serialised by the caller. The first call on each device looks up the array's device
+ * address with that device current; make that first call before any stream capture.
+ */
+int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H,
+                             int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                             const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                             float scale, float* out, void* stream);
+
 /* Workspace bytes that tq_search_topk needs. */
 int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes);
 

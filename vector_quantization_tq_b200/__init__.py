@@ -22,7 +22,7 @@ __all__ = [
     "MSE", "PROD", "ROT_DENSE", "ROT_RHT", "F32", "BF16",
     "build_codebook", "draw_gaussian", "draw_signs", "haar_rotation",
     "State", "quantize_mse", "quantize_prod", "dequant", "score",
-    "attend_workspace", "attend_decode", "search_workspace", "search_topk",
+    "attend_workspace", "attend_decode", "attend_decode_noalloc", "search_workspace", "search_topk",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -85,6 +85,7 @@ _SIGS = {
     "tq_score": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
     "tq_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
     "tq_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _SZ, _P]),
+    "tq_attend_decode_noalloc": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P]),
     "tq_search_workspace": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_SZ)]),
     "tq_search_topk": (_I, [_P, _P, _I, _I64, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
 }
@@ -317,6 +318,21 @@ def attend_decode(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms, vcodes
     _check(_lib.tq_attend_decode(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, _ptr(kcodes), _ptr(kqjl),
                                  _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "tq_attend_decode")
+
+
+def attend_decode_noalloc(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale: float,
+                          out, H=None, T=None, stream=None):
+    """tq_attend_decode with the library's fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory (runtimes whose own pool owns all device
+    memory, latency-critical loops that must not allocate). Calls that overlap on the GPU
+    share the library's fixed scratch and race; see tq.h.
+    """
+    H = q.shape[0] if H is None else H
+    T = knorms.numel() // H if T is None else T
+    _check(_lib.tq_attend_decode_noalloc(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, _ptr(kcodes),
+                                         _ptr(kqjl), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
+                                         float(scale), _ptr(out), _stream(stream)), "tq_attend_decode_noalloc")
 
 
 def search_workspace(st: State, nq: int, n: int, k: int) -> int:

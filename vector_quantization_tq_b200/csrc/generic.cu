@@ -8,6 +8,8 @@
 // The rotation and QJL products are CUDA-core FMA loops over the stored matrices
 // (fp32 accumulate), the RHT is an in-register / shuffle / shared-memory butterfly.
 // The specialised tensor-core encoder for d = 128 lives in encode_tc.cu.
+#include <mutex>
+
 #include "common.cuh"
 #include "prep.cuh"
 
@@ -738,6 +740,43 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
     if (e != cudaSuccess) return (int)e;
     attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, out);
     return (int)cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------
+// Decode attention without a caller-supplied workspace.
+//
+// For callers that cannot allocate device memory (runtimes that hand all device memory to
+// their own pool allocator, or latency-critical decode loops where an allocation's cost or
+// possible failure is not acceptable): the split partials live
+// in a fixed, file-scope device array instead of a workspace. Every GPU that loads the
+// library holds this array until the process exits. All calls share it and it keeps the
+// last call's contents; nothing in it needs to start at zero (each partial record is
+// written before the combine step reads it). Calls whose work overlaps on the GPU (other
+// streams, other threads) race on it and must be serialised by the caller.
+// ------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_attend_scratch[kAttendStaticScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+int attend_static_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    if (dev < 0 || dev >= kMaxDevices) return (int)cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        // The array's name is a host-side stand-in: its device address must be looked up,
+        // once per device, with that device current.
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attend_scratch);
+        if (e != cudaSuccess) return (int)e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return 0;
 }
 
 namespace {

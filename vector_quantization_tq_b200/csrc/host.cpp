@@ -533,6 +533,32 @@ int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int 
                                                   workspace, ws_bytes, stream));
 }
 
+int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int64_t T,
+                             const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+                             const uint8_t* vcodes, const float* vnorms, float scale, float* out, void* stream) {
+    if (!ks || !vs || H < 0 || T < 0) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (vs->p.mode != TQ_MSE || ks->p.d != vs->p.d || ks->p.device != vs->p.device) return TQ_EINVAL;
+    if (!std::isfinite(scale)) return TQ_EINVAL;
+    if (H == 0) return TQ_OK;
+    if (T == 0) return TQ_EINVAL;
+    const bool prod = ks->p.mode == TQ_PROD;
+    if (!q || !out || !knorms || !vnorms || (ks->b_mse > 0 && !kcodes) || !vcodes ||
+        (prod && (!kqjl || !krnorms)))
+        return TQ_EINVAL;
+    if (!aligned16(q) || !aligned16(out)) return TQ_EINVAL;
+    const size_t need = attend_workspace_bytes(ks->dev, H, T);
+    if (need > kAttendStaticScratchBytes) return TQ_EUNSUPPORTED;   // beyond the fixed 4 MiB array
+    DeviceGuard g(ks->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    void* scratch = nullptr;
+    int e = attend_static_scratch(&scratch);
+    if (e != 0) return cuda_status((cudaError_t)e);
+    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, kcodes, prod ? kqjl : nullptr,
+                                                  knorms, prod ? krnorms : nullptr, vcodes, vnorms, scale, out,
+                                                  scratch, kAttendStaticScratchBytes, stream));
+}
+
 int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes) {
     if (!st || !bytes || nq < 0 || n < 0 || k < 1 || k > 64) return TQ_EINVAL;
     *bytes = search_workspace_bytes(st->dev, nq, n, k);

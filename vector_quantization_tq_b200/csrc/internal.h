@@ -12,6 +12,9 @@ namespace tq {
 
 constexpr int kMaxLevels = 256;      // 2^b_mse with b_mse <= 8
 constexpr int kMaxDim = 2048;        // largest d the kernels accept
+constexpr int kMaxDevices = 64;
+// Size of the fixed device array behind tq_attend_decode_noalloc (4 MiB).
+constexpr size_t kAttendStaticScratchBytes = (size_t)4 << 20;
 
 // Everything a kernel needs about a state, passed by value as a kernel parameter
 // (lives in the constant bank: uniform reads of the codebook are broadcasts).
@@ -75,6 +78,7 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
                   int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
                   const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,
                   float* out, void* ws, size_t ws_bytes, void* stream);
+int attend_static_scratch(void** out);
 size_t search_workspace_bytes(const DevState& st, int64_t nq, int64_t n, int k);
 int launch_search(const DevState& st, const void* q, int qdtype, int64_t nq,
                   const uint8_t* codes, const uint8_t* qjl, const float* norms,
