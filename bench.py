@@ -121,6 +121,59 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# Decode attention over a compressed cache (32 heads x 131072 tokens, d = 128): keys prod
+# b=4 (48 B codes + 16 B QJL + 8 B norms), values mse b=4 (64 B codes + 4 B norm).
+DEC_H, DEC_T = 32, 131072
+DEC_BYTES_PER_TOKEN = (48 + 16 + 8) + (64 + 4)
+
+
+def measure_decode(tq, torch, dev, stream, steps: int, warmup: int, peak: float):
+    """Time tq_attend_decode on the decode-step workload (seeded synthetic cache, built on the GPU)."""
+    d = D
+    ks = tq.State(d, 4, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0),
+                  s=synth.gaussian_matrix(d, synth.SEED_S))
+    vs = tq.State(d, 4, tq.MSE, tq.ROT_DENSE, tq.F32, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0))
+    n = DEC_H * DEC_T
+    kc, kz, kn, kr = ks.empty_planes(n, dev)
+    vc, _, vn, _ = vs.empty_planes(n, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(12345)
+    for h in range(DEC_H):
+        sl = slice(h * DEC_T, (h + 1) * DEC_T)
+        k = torch.randn(DEC_T, d, generator=g, device=dev)
+        v = torch.randn(DEC_T, d, generator=g, device=dev)
+        k /= k.norm(dim=1, keepdim=True)
+        v /= v.norm(dim=1, keepdim=True)
+        tq.quantize_prod(ks, k, kc[sl], kz[sl], kn[sl], kr[sl], stream=stream)
+        tq.quantize_mse(vs, v, vc[sl], vn[sl], stream=stream)
+    q = torch.randn(DEC_H, d, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((DEC_H, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.attend_workspace(ks, vs, DEC_H, DEC_T), dtype=torch.uint8, device=dev)
+    scale = 1.0 / d ** 0.5
+
+    def run():
+        tq.attend_decode(ks, vs, q, kc, kz, kn, kr, vc, vn, scale, out, ws, H=DEC_H, T=DEC_T, stream=stream)
+
+    for _ in range(max(3, warmup)):
+        run()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    gbs = DEC_BYTES_PER_TOKEN * n / (ms / 1e3) / 1e9
+    ks.close()
+    vs.close()
+    return {"workload": "decode attention, 32 heads x 131072 tokens, d=128, K prod b=4, V mse b=4, one bf16 "
+                        "query per head", "ms": ms, "gkeys_s": n / (ms / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "algorithmic_bytes_per_launch": DEC_BYTES_PER_TOKEN * n},
+            "gpu_launches_per_step": 2}
+
+
 def oracle_sample(heads: int, seed: int):
     """The oracle (fp64 numpy) on `heads` heads of the workload; returns (vectors, seconds, threads)."""
     from oracle import quantizer as OQ
@@ -182,6 +235,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=HEADS, help="smaller batch for profiling runs")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -305,6 +359,9 @@ def main():
                          f"estimate, {dt:.2f} s wall"}
 
     peak, peak_kind = measured_peaks()
+    decode = None
+    if not args.no_decode:
+        decode = measure_decode(tq, torch, dev, stream, args.steps, args.warmup, peak)
     enc_gbs = ENC_BYTES_PER_VEC * nvec / (enc_ms / 1e3) / 1e9
     sc_gbs = SCORE_BYTES_PER_KEY * nvec / (sc_ms / 1e3) / 1e9
     traffic = stored_traffic("encode_prod_d128")
@@ -335,6 +392,7 @@ def main():
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
+        "decode_attention": decode,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -1,0 +1,260 @@
+// Fused decode attention over a compressed KV cache, d = 128 (one query per head).
+//
+// Per head h: s_t = scale * <q_h, k~_t>, p = softmax(s), out_h = sum_t p_t v~_t, with
+// v~_t = ||v_t|| Pi_V^T c_V[idx_t]. The standard attention form is the PolarQuant review's
+// (attention over a quantized cache); the score is TurboQuant's inner-product estimate
+// (Jump2Paper review, Theorem 2): <q, k~> = ||k|| (sum_j q'_j c[idx_j] + ||r|| sqrt(pi/2)/d
+// sum_j u_j (2 z_j - 1)), q' = Pi_K q, u = S q'.
+//
+// Flash-decoding split over tokens: block (split, h) walks tiles of 256 tokens with an
+// online softmax and writes (m, l, acc[d]) for the combine launch, which merges the splits
+// and applies Pi_V^T once per head. Inside a tile:
+//   A. one thread per token scores it through per-query tables over packed code groups
+//      (16- or 64-entry tables in shared memory, as in the LUT scorer);
+//   B. the block updates the running max and sum and forms w_t = p_t ||v_t||;
+//   C. one warp per token accumulates w_t c_V[idx_tj] into the rotated-domain value sum,
+//      each lane owning 4 coordinates (a 2-byte slice of the token's 4-bit code row).
+// Only the compressed bytes are read: 72 B (keys, prod b=4) + 68 B (values, mse b=4) per
+// token and head.
+#include "common.cuh"
+#include "prep.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+template <int B>
+struct KGroups {
+    static constexpr int G = (B == 3) ? 6 : 4;
+    static constexpr int CPG = G / B;
+    static constexpr int E = 1 << G;
+    static constexpr int NG = kD * B / G;
+};
+
+template <int BK, bool KPROD, int BV>
+__global__ void __launch_bounds__(kThreads)
+attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__ q, int qdtype, int64_t T,
+                  int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
+                  const float* __restrict__ knorms, const float* __restrict__ krnorms,
+                  const uint8_t* __restrict__ vcodes, const float* __restrict__ vnorms, float scale,
+                  float* __restrict__ part) {
+    using KG = KGroups<BK>;
+    constexpr int NQ = kD / 4;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float* ctab = reinterpret_cast<float*>(smem_raw);           // kMaxLevels (K centroids)
+    float* vc = ctab + kMaxLevels;                               // 16 (V centroids), padded to 32
+    float* qs = vc + 32;                                         // kD
+    float* qp = qs + kD;                                         // kD
+    float* u = qp + kD;                                          // kD
+    float* tm = u + kD;                                          // NG * E
+    float* tz = tm + KG::NG * KG::E;                             // NQ * 16
+    float* wt = tz + NQ * 16;                                    // kThreads
+    float* red = wt + kThreads;                                  // 32
+    float* accw = red + 32;                                      // kWarps * kD
+    unsigned char* stage = reinterpret_cast<unsigned char*>(accw + kWarps * kD);
+
+    const int h = blockIdx.y;
+    const int split = blockIdx.x;
+    const int nsplit = gridDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < ks.L; i += kThreads) ctab[i] = ks.c[i];
+    if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
+    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
+    prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * kD * qelem, qdtype, 1, qs, qp, u,
+                     stage);
+    for (int i = threadIdx.x; i < KG::NG * KG::E; i += kThreads) {
+        const int k = i / KG::E, e = i % KG::E;
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < KG::CPG; ++c) a = fmaf(qp[k * KG::CPG + c], ctab[(e >> (BK * c)) & ((1 << BK) - 1)], a);
+        tm[i] = a;
+    }
+    if constexpr (KPROD) {
+        for (int i = threadIdx.x; i < NQ * 16; i += kThreads) {
+            const int k = i / 16, e = i % 16;
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = u[4 * k + c];
+                a += ((e >> c) & 1) ? v : -v;
+            }
+            tz[i] = a;
+        }
+    }
+    __syncthreads();
+
+    const int64_t t_begin = (int64_t)split * chunk;
+    const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
+    const int64_t hT = (int64_t)h * T;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};       // coordinates 4*lane .. 4*lane+3, this warp's tokens
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads) {
+        const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
+        // ---- A: score of token t0 + threadIdx.x ----
+        float s = -INFINITY;
+        if ((int)threadIdx.x < cnt) {
+            const int64_t gk = hT + t0 + threadIdx.x;
+            constexpr int CW = kD * BK / 32;
+            uint32_t w[CW];
+            const uint4* src = reinterpret_cast<const uint4*>(kcodes + gk * (kD * BK / 8));
+#pragma unroll
+            for (int i = 0; i < CW / 4; ++i) {
+                const uint4 v = __ldg(src + i);
+                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+            }
+            float a1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < KG::NG; ++k) {
+                const int bit = k * KG::G;
+                const int wi = bit >> 5, sh = bit & 31;
+                uint32_t e;
+                if (sh + KG::G <= 32) e = (w[wi] >> sh) & (KG::E - 1);
+                else e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (KG::E - 1);
+                a1 += tm[k * KG::E + e];
+            }
+            float a2 = 0.f, g2 = 0.f;
+            if constexpr (KPROD) {
+                const uint4 zv = __ldg(reinterpret_cast<const uint4*>(kqjl + gk * (kD / 8)));
+                const uint32_t z[4] = {zv.x, zv.y, zv.z, zv.w};
+#pragma unroll
+                for (int k = 0; k < NQ; ++k) a2 += tz[k * 16 + ((z[k >> 3] >> ((k & 7) * 4)) & 15u)];
+                g2 = __ldg(krnorms + gk) * ks.qjl_scale;
+            }
+            s = scale * __ldg(knorms + gk) * fmaf(g2, a2, a1);
+        }
+        // ---- B: online softmax bookkeeping ----
+        const float wm = warp_max(s);
+        if (lane == 0) red[warp] = wm;
+        __syncthreads();
+        float tmax = red[0];
+#pragma unroll
+        for (int i = 1; i < kWarps; ++i) tmax = fmaxf(tmax, red[i]);
+        const float m_new = fmaxf(m_run, tmax);
+        const float alpha = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
+        const float p = ((int)threadIdx.x < cnt) ? __expf(s - m_new) : 0.f;
+        const float ps = warp_sum(p);
+        __syncthreads();   // everyone has read red[] (max) before it is reused
+        if (lane == 0) red[warp] = ps;
+        if ((int)threadIdx.x < cnt) wt[threadIdx.x] = p * __ldg(vnorms + hT + t0 + threadIdx.x);
+        __syncthreads();
+        float tsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kWarps; ++i) tsum += red[i];
+        l_run = l_run * alpha + tsum;
+        m_run = m_new;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] *= alpha;
+        // ---- C: value sum, one warp per token, 4 coordinates per lane ----
+        for (int t = warp; t < cnt; t += kWarps) {
+            const uint8_t* row = vcodes + (hT + t0 + t) * (kD * BV / 8);
+            const float wv = wt[t];
+            uint32_t bits;
+            if constexpr (BV == 4) {
+                bits = __ldg(reinterpret_cast<const uint16_t*>(row) + lane);
+            } else if constexpr (BV == 2) {
+                bits = __ldg(row + lane);
+            } else {
+                const int b0 = lane * 4 * BV;
+                const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row);
+                const int wi = b0 >> 5, sh = b0 & 31;
+                uint64_t win = __ldg(r32 + wi);
+                if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)__ldg(r32 + wi + 1) << 32;
+                bits = (uint32_t)(win >> sh);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[c] = fmaf(wv, vc[(bits >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
+        }
+        __syncthreads();   // wt / red reused by the next tile
+    }
+    // ---- reduce the warps' value sums and write the split record ----
+#pragma unroll
+    for (int c = 0; c < 4; ++c) accw[warp * kD + 4 * lane + c] = acc[c];
+    __syncthreads();
+    float* rec = part + ((int64_t)h * nsplit + split) * (kD + 2);
+    for (int j = threadIdx.x; j < kD; j += kThreads) {
+        float a = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kWarps; ++w2) a += accw[w2 * kD + j];
+        rec[2 + j] = a;
+    }
+    if (threadIdx.x == 0) {
+        rec[0] = m_run;
+        rec[1] = l_run;
+    }
+}
+
+template <int BK, bool KPROD, int BV>
+size_t smem_bytes() {
+    using KG = KGroups<BK>;
+    return (size_t)(kMaxLevels + 32 + 3 * kD + KG::NG * KG::E + (kD / 4) * 16 + kThreads + 32 + kWarps * kD) *
+               sizeof(float) + kPrepStageBytes;
+}
+
+template <int BK, bool KPROD, int BV>
+int launch_t(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+             int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+             const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
+    auto kern = attend_lut_kernel<BK, KPROD, BV>;
+    const size_t smem = smem_bytes<BK, KPROD, BV>();
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+    }
+    dim3 grid((unsigned)nsplit, (unsigned)H);
+    kern<<<grid, kThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
+                                      scale, part);
+    return (int)cudaGetLastError();
+}
+
+template <int BK, bool KPROD>
+int launch_v(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+             int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+             const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
+    switch (vs.b_mse) {
+        case 2: return launch_t<BK, KPROD, 2>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                              vcodes, vnorms, scale, part, s);
+        case 3: return launch_t<BK, KPROD, 3>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                              vcodes, vnorms, scale, part, s);
+        case 4: return launch_t<BK, KPROD, 4>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                              vcodes, vnorms, scale, part, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+template <bool KPROD>
+int launch_k(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+             int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+             const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
+    switch (ks.b_mse) {
+        case 2: return launch_v<2, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                          vcodes, vnorms, scale, part, s);
+        case 3: return launch_v<3, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                          vcodes, vnorms, scale, part, s);
+        case 4: return launch_v<4, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                          vcodes, vnorms, scale, part, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool attend_lut_supported(const DevState& ks, const DevState& vs) {
+    return ks.d == kD && vs.d == kD && ks.b_mse >= 2 && ks.b_mse <= 4 && vs.b_mse >= 2 && vs.b_mse <= 4;
+}
+
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
+                            int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
+                            const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                            float scale, float* part, void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    if (kqjl) return launch_k<true>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes,
+                                    vnorms, scale, part, s);
+    return launch_k<false>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
+                           scale, part, s);
+}
+
+}  // namespace tq

@@ -350,6 +350,529 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
 }
 
+// ------------------------------------------------------------------------------------
+// Two threads per vector (b_mse = 1 or 2): 256 threads per 128-vector tile. Warp w serves
+// vectors 32*(w%4) .. +31 (its TMEM lane quadrant) and coordinates 64*(w/4) .. +63. Both
+// threads of a vector read the whole bf16 row, so the stride-64 butterfly stage is taken
+// at load time (y_j = x_j +- x_{j+64}) and the remaining six stages stay in registers.
+// Halving the per-thread state keeps registers under 128, so two CTAs (16 warps) fit
+// on an SM; the two halves meet only through ||r||^2 (shared memory) and the MMA.
+// ------------------------------------------------------------------------------------
+struct __align__(1024) TcSmem2 {
+    uint8_t x[2][2][kTile * 128];   // [stage][half]: 128 rows x 128 bytes, 128B-swizzled
+    uint8_t s[kD * kD * 2];         // S as the B operand: K-major core matrices
+    float rr[2][kTile];             // per half: partial ||r||^2
+    uint64_t bar_x[2];
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int pad;
+};
+
+__device__ __forceinline__ uint32_t spread16(uint32_t x) {
+    x &= 0xffffu;
+    x = (x | (x << 8)) & 0x00ff00ffu;
+    x = (x | (x << 4)) & 0x0f0f0f0fu;
+    x = (x | (x << 2)) & 0x33333333u;
+    x = (x | (x << 1)) & 0x55555555u;
+    return x;
+}
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(2 * kTile, 2)
+encode_tc2_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
+    static_assert(B == 1 || B == 2, "two-thread layout covers 1- and 2-bit codes");
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem2& sm = *reinterpret_cast<TcSmem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int vrow = quad * 32 + (tid & 31);   // vector within the tile = TMEM lane
+    const int64_t ntiles = (p.n + kTile - 1) / kTile;
+
+    if (tid == 0) {
+        ptx::prefetch_tmap(&tmap);
+        ptx::mbar_init(&sm.bar_x[0], 1);
+        ptx::mbar_init(&sm.bar_x[1], 1);
+        ptx::mbar_init(&sm.bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    if constexpr (PROD) {
+        if (warp == 0) {
+            ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
+            ptx::tmem_relinquish();
+        }
+        for (int i = tid; i < kD * 16; i += 2 * kTile) {
+            const int row = i >> 4, c = i & 15;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.s + row * kD + c * 8));
+            *reinterpret_cast<uint4*>(sm.s + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
+        }
+        ptx::fence_proxy_async_smem();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = PROD ? sm.tmem_base : 0u;
+    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+
+    auto issue = [&](int stg, int64_t tile) {
+        ptx::mbar_arrive_expect_tx(&sm.bar_x[stg], 2 * kTile * 128);
+        ptx::tma_load_2d(sm.x[stg][0], &tmap, 0, (int)(tile * kTile), &sm.bar_x[stg]);
+        ptx::tma_load_2d(sm.x[stg][1], &tmap, 64, (int)(tile * kTile), &sm.bar_x[stg]);
+    };
+    uint32_t pending = 0u, xphase = 0u, mphase = 0u;
+    const int64_t t0 = blockIdx.x;
+    if (t0 < ntiles) {
+        if (tid == 0) issue(0, t0);
+        pending |= 1u;
+    }
+    if (t0 + gridDim.x < ntiles) {
+        if (tid == 0) issue(1, t0 + gridDim.x);
+        pending |= 2u;
+    }
+    bool failed = false;
+    const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
+    const uint32_t s_addr = ptx::smem_addr(sm.s);
+    const float2 hs = half ? f2(-1.f, -1.f) : f2(1.f, 1.f);
+
+    int it = 0;
+    for (int64_t tile = t0; tile < ntiles; tile += gridDim.x, ++it) {
+        const int stg = it & 1;
+        const bool ok = ptx::mbar_wait(&sm.bar_x[stg], (xphase >> stg) & 1u);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        xphase ^= 1u << stg;
+        pending &= ~(1u << stg);
+        // ---- read x_j and x_{j+64} (8 at a time), signs, fp32, stride-64 stage ----
+        float2 v[32];
+        float2 ss = f2(0.f, 0.f);
+        {
+            const uint8_t* b0 = sm.x[stg][0] + vrow * 128;
+            const uint8_t* b1 = sm.x[stg][1] + vrow * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int off = (c ^ (vrow & 7)) << 4;
+                const uint4 qa = *reinterpret_cast<const uint4*>(b0 + off);
+                const uint4 qb = *reinterpret_cast<const uint4*>(b1 + off);
+                const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+                const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t ua = wa[e] ^ p.sgn[4 * c + e];
+                    const uint32_t ub = wb[e] ^ p.sgn[32 + 4 * c + e];
+                    const float2 xa = f2(__uint_as_float(ua << 16), __uint_as_float(ua & 0xffff0000u));
+                    const float2 xb = f2(__uint_as_float(ub << 16), __uint_as_float(ub & 0xffff0000u));
+                    ss = __ffma2_rn(xa, xa, ss);
+                    ss = __ffma2_rn(xb, xb, ss);
+                    v[4 * c + e] = __ffma2_rn(xb, hs, xa);
+                }
+            }
+        }
+        __syncthreads();   // both halves have read the stage: refill it
+        const int64_t nxt = tile + 2 * (int64_t)gridDim.x;
+        if (nxt < ntiles) {
+            if (tid == 0) issue(stg, nxt);
+            pending |= 1u << stg;
+        }
+        const float nu = sqrtf(ss.x + ss.y);
+        // ---- remaining butterfly stages (strides 1..32) on the local 64 values ----
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float a = v[i].x, b = v[i].y;
+            v[i] = f2(a + b, a - b);
+        }
+#pragma unroll
+        for (int k = 1; k < 32; k <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if ((i & k) == 0) {
+                    const float2 a = v[i], b = v[i + k];
+                    v[i] = __fadd2_rn(a, b);
+                    v[i + k] = __ffma2_rn(b, f2(-1.f, -1.f), a);
+                }
+            }
+        }
+        const float sc = (nu > 0.f) ? p.rsqrt_d / nu : 0.f;
+        // ---- quantize on the unscaled coordinate; residual ----
+        const float T2 = (B == 2 && nu > 0.f) ? p.t[2] / sc : INFINITY;
+        const float cs = (nu > 0.f) ? p.c[B == 2 ? 2 : 1] : 0.f;
+        const float cb = (nu > 0.f) ? p.c[B == 2 ? 3 : 1] : 0.f;
+        uint32_t cw[2 * B];
+        float2 rr2 = f2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            uint32_t np = 0u, mp = 0u;
+#pragma unroll
+            for (int q = 15; q >= 0; --q) {
+                const int i = g * 16 + q;
+                float r[2];
+#pragma unroll
+                for (int e = 1; e >= 0; --e) {
+                    const float y = e ? v[i].y : v[i].x;
+                    const uint32_t yb = __float_as_uint(y);
+                    np = __funnelshift_l(yb, np, 1);
+                    float mag = cs;
+                    if constexpr (B == 2) {
+                        const float dd = fabsf(y) - T2;
+                        mp = __funnelshift_l(__float_as_uint(dd), mp, 1);
+                        mag = (dd < 0.f) ? cs : cb;
+                    }
+                    const float smag = __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
+                    r[e] = fmaf(y, sc, -smag);
+                }
+                v[i] = f2(r[0], r[1]);
+                rr2 = __ffma2_rn(v[i], v[i], rr2);
+            }
+            if constexpr (B == 1) {
+                cw[g] = ~np;
+            } else {
+                const uint32_t hb = ~np, lb = ~(np ^ mp);
+                cw[2 * g] = spread16(lb) | (spread16(hb) << 1);
+                cw[2 * g + 1] = spread16(lb >> 16) | (spread16(hb >> 16) << 1);
+            }
+        }
+        const int64_t row = tile * kTile + vrow;
+        if (row < p.n) {
+            if constexpr (B == 2)
+                *reinterpret_cast<uint4*>(p.codes + row * 32 + half * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            else
+                *reinterpret_cast<uint2*>(p.codes + row * 16 + half * 8) = make_uint2(cw[0], cw[1]);
+            if (half == 0) p.norms[row] = nu;
+        }
+        if constexpr (PROD) {
+            sm.rr[half][vrow] = rr2.x + rr2.y;
+#pragma unroll
+            for (int part = 0; part < 1; ++part) {
+                uint32_t hi[32], lo[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float2 r = v[q];
+                    const __nv_bfloat162 h = __float22bfloat162_rn(r);
+                    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+                    const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
+                    const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), r);
+                    const __nv_bfloat162 lb = __float22bfloat162_rn(l);
+                    hi[q] = hb;
+                    lo[q] = *reinterpret_cast<const uint32_t*>(&lb);
+                }
+                ptx::tmem_st32(t_lane + 128 + half * 32, hi);
+                ptx::tmem_st32(t_lane + 192 + half * 32, lo);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (half == 0 && row < p.n) p.rnorms[row] = sqrtf(sm.rr[0][vrow] + sm.rr[1][vrow]);
+            if (tid == 0) {
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 128 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 192 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, 1u);
+                ptx::mma_commit(&sm.bar_mma);
+            }
+            const bool mok = ptx::mbar_wait(&sm.bar_mma, mphase);
+            if (__syncthreads_or(!mok)) {
+                failed = true;
+                break;
+            }
+            mphase ^= 1u;
+            ptx::tc_fence_after();
+            uint32_t zw[2];
+            {
+                uint32_t a0[32], a1[32];
+                ptx::tmem_ld32(t_lane + half * 64, a0);
+                ptx::tmem_ld32(t_lane + half * 64 + 32, a1);
+                ptx::tmem_wait_ld();
+                uint32_t n0 = 0u, n1 = 0u;
+#pragma unroll
+                for (int j = 31; j >= 0; --j) {
+                    n0 = __funnelshift_l(a0[j], n0, 1);
+                    n1 = __funnelshift_l(a1[j], n1, 1);
+                }
+                zw[0] = (nu > 0.f) ? ~n0 : 0xffffffffu;
+                zw[1] = (nu > 0.f) ? ~n1 : 0xffffffffu;
+            }
+            ptx::tc_fence_before();
+            if (row < p.n) *reinterpret_cast<uint2*>(p.qjl + row * 16 + half * 8) = make_uint2(zw[0], zw[1]);
+        }
+    }
+    if (failed) {
+        if (tid == 0) atomicExch(&g_tq_device_error, 1);
+        for (int s2 = 0; s2 < 2; ++s2)
+            if ((pending >> s2) & 1u) (void)ptx::mbar_wait(&sm.bar_x[s2], (xphase >> s2) & 1u);
+        if (PROD) (void)ptx::mbar_wait(&sm.bar_mma, mphase, 100000000ull);
+    }
+    __syncthreads();
+    if constexpr (PROD) {
+        if (warp == 0) {
+            ptx::tc_fence_after();
+            ptx::tmem_dealloc(tmem, kTmemCols);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Rotation on the tensor core (b_mse = 1 or 2). The randomized Hadamard transform is the
+// dense product y = (H diag(eps)) x: with x bf16 (exact) and H diag(eps) = +-1 (exact in
+// bf16), one K = 128 MMA straight from the 128B-swizzled TMA tile gives H D x in fp32 in
+// TMEM, with exact products and fp32 sums as in the register butterfly. The threads then
+// only read y back, quantize, split the residual and read the signs of S r.
+// Two threads per vector as in encode_tc2_kernel; TMEM columns [0,128) hold y and then
+// S r, [128,256) the residual operand (hi, lo).
+// ------------------------------------------------------------------------------------
+struct __align__(1024) TcSmem3 {
+    uint8_t x[2][kTile * 128];      // [half]: 128 rows x 128 bytes, 128B-swizzled
+    uint8_t hd[kD * kD * 2];        // H diag(eps) as the B operand: K-major core matrices
+    uint8_t s[kD * kD * 2];         // S as the B operand
+    float ssq[2][kTile];            // per half: partial ||H D x||^2
+    float rsq[2][kTile];            // per half: partial ||r||^2
+    uint64_t bar_x;
+    uint64_t bar_h;
+    uint64_t bar_s;
+    uint32_t tmem_base;
+    int pad;
+};
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(2 * kTile, 2)
+encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
+    static_assert(B == 1 || B == 2, "two-thread layout covers 1- and 2-bit codes");
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem3& sm = *reinterpret_cast<TcSmem3*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int vrow = quad * 32 + (tid & 31);
+    const int64_t ntiles = (p.n + kTile - 1) / kTile;
+
+    if (tid == 0) {
+        ptx::prefetch_tmap(&tmap);
+        ptx::mbar_init(&sm.bar_x, 1);
+        ptx::mbar_init(&sm.bar_h, 1);
+        ptx::mbar_init(&sm.bar_s, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    // H diag(eps): entry (n, k) = (-1)^popcount(n & k) * eps_k, at chunk k/8 of row n.
+    for (int i = tid; i < kD * kD; i += 2 * kTile) {
+        const int n = i >> 7, k = i & 127;
+        const uint32_t neg = (__popc(n & k) & 1) ^ ((p.sgn[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u);
+        const uint16_t v = neg ? 0xBF80u : 0x3F80u;
+        *reinterpret_cast<uint16_t*>(sm.hd + (k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) = v;
+    }
+    if constexpr (PROD) {
+        for (int i = tid; i < kD * 16; i += 2 * kTile) {
+            const int row = i >> 4, c = i & 15;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.s + row * kD + c * 8));
+            *reinterpret_cast<uint4*>(sm.s + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+
+    auto issue = [&](int64_t tile) {
+        ptx::mbar_arrive_expect_tx(&sm.bar_x, 2 * kTile * 128);
+        ptx::tma_load_2d(sm.x[0], &tmap, 0, (int)(tile * kTile), &sm.bar_x);
+        ptx::tma_load_2d(sm.x[1], &tmap, 64, (int)(tile * kTile), &sm.bar_x);
+    };
+    bool pending = false;
+    const int64_t t0 = blockIdx.x;
+    if (t0 < ntiles) {
+        if (tid == 0) issue(t0);
+        pending = true;
+    }
+    uint32_t xph = 0u, hph = 0u, sph = 0u;
+    bool failed = false;
+    const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
+    const uint32_t s_addr = ptx::smem_addr(sm.s);
+    const uint32_t hd_addr = ptx::smem_addr(sm.hd);
+    const uint32_t x_addr0 = ptx::smem_addr(sm.x[0]);
+    const uint32_t x_addr1 = ptx::smem_addr(sm.x[1]);
+
+    for (int64_t tile = t0; tile < ntiles; tile += gridDim.x) {
+        const bool ok = ptx::mbar_wait(&sm.bar_x, xph);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        xph ^= 1u;
+        pending = false;
+        // ---- y = (H D) x on the tensor core ----
+        if (tid == 0) {
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a = ((kk < 4) ? x_addr0 : x_addr1) + (kk & 3) * 32;
+                ptx::mma_ss(tmem, ptx::smem_desc_kmajor_sw128(a),
+                            ptx::smem_desc_kmajor(hd_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(&sm.bar_h);
+        }
+        const bool hok = ptx::mbar_wait(&sm.bar_h, hph);
+        if (__syncthreads_or(!hok)) {
+            failed = true;
+            break;
+        }
+        hph ^= 1u;
+        ptx::tc_fence_after();
+        const int64_t nxt = tile + gridDim.x;
+        if (nxt < ntiles) {   // the MMA has read the tile: refill the buffer
+            if (tid == 0) issue(nxt);
+            pending = true;
+        }
+        float2 v[32];
+        {
+            uint32_t a0[32], a1[32];
+            ptx::tmem_ld32(t_lane + half * 64, a0);
+            ptx::tmem_ld32(t_lane + half * 64 + 32, a1);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                v[i] = f2(__uint_as_float(a0[2 * i]), __uint_as_float(a0[2 * i + 1]));
+                v[16 + i] = f2(__uint_as_float(a1[2 * i]), __uint_as_float(a1[2 * i + 1]));
+            }
+        }
+        float2 ss = f2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = __ffma2_rn(v[i], v[i], ss);
+        sm.ssq[half][vrow] = ss.x + ss.y;
+        ptx::tc_fence_before();
+        __syncthreads();
+        // ||H D x||^2 = d ||x||^2
+        const float nu = sqrtf(sm.ssq[0][vrow] + sm.ssq[1][vrow]) * p.rsqrt_d;
+        const float sc = (nu > 0.f) ? p.rsqrt_d / nu : 0.f;
+        const float T2 = (B == 2 && nu > 0.f) ? p.t[2] / sc : INFINITY;
+        const float cs = (nu > 0.f) ? p.c[B == 2 ? 2 : 1] : 0.f;
+        const float cb = (nu > 0.f) ? p.c[B == 2 ? 3 : 1] : 0.f;
+        uint32_t cw[2 * B];
+        float2 rr2 = f2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            uint32_t np = 0u, mp = 0u;
+#pragma unroll
+            for (int q = 15; q >= 0; --q) {
+                const int i = g * 16 + q;
+                float r[2];
+#pragma unroll
+                for (int e = 1; e >= 0; --e) {
+                    const float y = e ? v[i].y : v[i].x;
+                    const uint32_t yb = __float_as_uint(y);
+                    np = __funnelshift_l(yb, np, 1);
+                    float mag = cs;
+                    if constexpr (B == 2) {
+                        const float dd = fabsf(y) - T2;
+                        mp = __funnelshift_l(__float_as_uint(dd), mp, 1);
+                        mag = (dd < 0.f) ? cs : cb;
+                    }
+                    const float smag = __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
+                    r[e] = fmaf(y, sc, -smag);
+                }
+                v[i] = f2(r[0], r[1]);
+                rr2 = __ffma2_rn(v[i], v[i], rr2);
+            }
+            if constexpr (B == 1) {
+                cw[g] = ~np;
+            } else {
+                const uint32_t hb = ~np, lb = ~(np ^ mp);
+                cw[2 * g] = spread16(lb) | (spread16(hb) << 1);
+                cw[2 * g + 1] = spread16(lb >> 16) | (spread16(hb >> 16) << 1);
+            }
+        }
+        const int64_t row = tile * kTile + vrow;
+        if (row < p.n) {
+            if constexpr (B == 2)
+                *reinterpret_cast<uint4*>(p.codes + row * 32 + half * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            else
+                *reinterpret_cast<uint2*>(p.codes + row * 16 + half * 8) = make_uint2(cw[0], cw[1]);
+            if (half == 0) p.norms[row] = nu;
+        }
+        if constexpr (PROD) {
+            sm.rsq[half][vrow] = rr2.x + rr2.y;
+            {
+                uint32_t hi[32], lo[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float2 r = v[q];
+                    const __nv_bfloat162 h = __float22bfloat162_rn(r);
+                    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+                    const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
+                    const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), r);
+                    const __nv_bfloat162 lb = __float22bfloat162_rn(l);
+                    hi[q] = hb;
+                    lo[q] = *reinterpret_cast<const uint32_t*>(&lb);
+                }
+                ptx::tmem_st32(t_lane + 128 + half * 32, hi);
+                ptx::tmem_st32(t_lane + 192 + half * 32, lo);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (half == 0 && row < p.n) p.rnorms[row] = sqrtf(sm.rsq[0][vrow] + sm.rsq[1][vrow]);
+            if (tid == 0) {
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 128 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem, tmem + 192 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, 1u);
+                ptx::mma_commit(&sm.bar_s);
+            }
+            const bool sok = ptx::mbar_wait(&sm.bar_s, sph);
+            if (__syncthreads_or(!sok)) {
+                failed = true;
+                break;
+            }
+            sph ^= 1u;
+            ptx::tc_fence_after();
+            uint32_t zw[2];
+            {
+                uint32_t a0[32], a1[32];
+                ptx::tmem_ld32(t_lane + half * 64, a0);
+                ptx::tmem_ld32(t_lane + half * 64 + 32, a1);
+                ptx::tmem_wait_ld();
+                uint32_t n0 = 0u, n1 = 0u;
+#pragma unroll
+                for (int j = 31; j >= 0; --j) {
+                    n0 = __funnelshift_l(a0[j], n0, 1);
+                    n1 = __funnelshift_l(a1[j], n1, 1);
+                }
+                zw[0] = (nu > 0.f) ? ~n0 : 0xffffffffu;
+                zw[1] = (nu > 0.f) ? ~n1 : 0xffffffffu;
+            }
+            if (row < p.n) *reinterpret_cast<uint2*>(p.qjl + row * 16 + half * 8) = make_uint2(zw[0], zw[1]);
+        }
+        ptx::tc_fence_before();
+    }
+    if (failed) {
+        if (tid == 0) atomicExch(&g_tq_device_error, 1);
+        if (pending) (void)ptx::mbar_wait(&sm.bar_x, xph);
+        (void)ptx::mbar_wait(&sm.bar_h, hph, 100000000ull);
+        if (PROD) (void)ptx::mbar_wait(&sm.bar_s, sph, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -408,8 +931,9 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
         const bool n1 = (st.signs[(2 * i + 1) >> 5] >> ((2 * i + 1) & 31)) & 1u;
         p.sgn[i] = (n0 ? 0x8000u : 0u) | (n1 ? 0x80000000u : 0u);
     }
-    const size_t smem = sizeof(TcSmem) + 1024;
-    auto kern = encode_tc_kernel<B, PROD>;
+    constexpr bool kTwo = (B == 1 || B == 2);
+    const size_t smem = (kTwo ? sizeof(TcSmem3) : sizeof(TcSmem)) + 1024;
+    auto kern = kTwo ? encode_tc3_kernel<(B <= 2 ? B : 2), PROD> : encode_tc_kernel<B, PROD>;
     static int attr_set_for_device = -1;   // per instantiation
     int dev = 0;
     cudaGetDevice(&dev);
@@ -420,7 +944,7 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
     }
     const int64_t ntiles = (n + kTile - 1) / kTile;
     const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * 2);
-    kern<<<grid, kTile, smem, stream>>>(tmap, p);
+    kern<<<grid, kTwo ? 2 * kTile : kTile, smem, stream>>>(tmap, p);
     return (int)cudaGetLastError();
 }
 

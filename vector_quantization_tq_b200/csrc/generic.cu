@@ -293,7 +293,7 @@ __device__ __forceinline__ void score_sums(const DevState& st, const float* ctab
 constexpr int kScoreQT = 8;
 constexpr int kScoreThreads = 256;
 
-size_t score_smem_bytes(int d) { return (size_t)(kMaxLevels + 3 * kScoreQT * d) * sizeof(float); }
+size_t score_smem_bytes(int d) { return (size_t)(kMaxLevels + 3 * kScoreQT * d) * sizeof(float) + kPrepStageBytes; }
 
 __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t nq,
@@ -306,13 +306,14 @@ score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t 
     float* qs = ctab + kMaxLevels;
     float* qp = qs + kScoreQT * d;
     float* u = qp + kScoreQT * d;
+    unsigned char* stage = reinterpret_cast<unsigned char*>(u + kScoreQT * d);
     const int64_t grp = blockIdx.z;
     const int64_t q0 = (int64_t)blockIdx.y * kScoreQT;
     const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
     for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
     prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * d) * qelem,
-                 qdtype, nqt, qs, qp, u);
+                 qdtype, nqt, qs, qp, u, stage);
     for (int64_t key = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; key < n;
          key += (int64_t)gridDim.x * blockDim.x) {
         const int64_t gk = grp * n + key;
@@ -333,7 +334,7 @@ constexpr int kAttMaxJ = kMaxDim / kAttThreads;   // coordinates per thread when
 
 size_t attend_smem_bytes(int d) {
     const int accs = (d > kAttThreads) ? d : kAttThreads;
-    return (size_t)(2 * kMaxLevels + 3 * d + kAttThreads + 32 + accs) * sizeof(float);
+    return (size_t)(2 * kMaxLevels + 3 * d + kAttThreads + 32 + accs) * sizeof(float) + kPrepStageBytes;
 }
 
 __global__ void __launch_bounds__(kAttThreads)
@@ -355,10 +356,12 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
     float* wt = u + d;                                    // kAttThreads weights p_t * ||v_t||
     float* red = wt + kAttThreads;                        // 32
     float* accs = red + 32;                               // max(d, kAttThreads)
+    unsigned char* stage = reinterpret_cast<unsigned char*>(accs + (d > kAttThreads ? d : kAttThreads));
     for (int i = threadIdx.x; i < ks.L; i += blockDim.x) kc[i] = ks.c[i];
     for (int i = threadIdx.x; i < vs.L; i += blockDim.x) vc[i] = vs.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u);
+    prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u,
+                     stage);
 
     const int64_t t_begin = (int64_t)split * chunk;
     const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
@@ -527,12 +530,14 @@ search_block_kernel(const DevState st, const void* __restrict__ q, int qdtype, i
     float* u = qp + kScoreQT * d;
     float* rv = u + kScoreQT * d;                                   // 8
     int64_t* ri = reinterpret_cast<int64_t*>(rv + 8);               // 8
-    float* sv = reinterpret_cast<float*>(ri + 8);                   // kScoreQT * block_keys
+    unsigned char* stage = reinterpret_cast<unsigned char*>(ri + 8);  // kPrepStageBytes
+    float* sv = reinterpret_cast<float*>(stage + kPrepStageBytes);  // kScoreQT * block_keys
     const int64_t q0 = (int64_t)blockIdx.y * kScoreQT;
     const int nqt = (int)(nq - q0 < kScoreQT ? nq - q0 : kScoreQT);
     for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)(q0 * d) * qelem, qdtype, nqt, qs, qp, u);
+    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)(q0 * d) * qelem, qdtype, nqt, qs, qp, u,
+                     stage);
     const int64_t k0 = (int64_t)blockIdx.x * block_keys;
     for (int local = threadIdx.x; local < block_keys; local += blockDim.x) {
         const int64_t key = k0 + local;
@@ -715,6 +720,12 @@ int attend_splits(int H, int64_t T) {
 }
 }  // namespace
 
+bool attend_lut_supported(const DevState& ks, const DevState& vs);
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
+                            int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
+                            const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                            float scale, float* part, void* stream);
+
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T) {
     if (H <= 0 || T <= 0) return 0;
     const int sp = attend_splits(H, T);
@@ -730,13 +741,19 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
     const int64_t chunk = (T + sp - 1) / sp;
     const int nsplit = (int)((T + chunk - 1) / chunk);
     float* part = reinterpret_cast<float*>(ws);
-    const size_t smem = attend_smem_bytes(ks.d);
-    if (smem > 48 * 1024)
-        cudaFuncSetAttribute(attend_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dim3 grid((unsigned)nsplit, (unsigned)H);
-    attend_split_kernel<<<grid, kAttThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms, krnorms,
-                                                         vcodes, vnorms, scale, part);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (attend_lut_supported(ks, vs)) {
+        e = (cudaError_t)launch_attend_lut_split(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms,
+                                                 krnorms, vcodes, vnorms, scale, part, stream);
+    } else {
+        const size_t smem = attend_smem_bytes(ks.d);
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(attend_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        dim3 grid((unsigned)nsplit, (unsigned)H);
+        attend_split_kernel<<<grid, kAttThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms,
+                                                             krnorms, vcodes, vnorms, scale, part);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return (int)e;
     attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, out);
     return (int)cudaGetLastError();

@@ -47,6 +47,7 @@ score_lut_kernel(const DevState st, const void* __restrict__ q, int qdtype, int6
     float* u = qp + QT * D;                                     // QT*D
     float* tm = u + QT * D;                                     // QT*NG*E
     float* tz = tm + QT * NG * Gr::E;                           // QT*NQ*16 (prod)
+    unsigned char* stage = reinterpret_cast<unsigned char*>(tz + (PROD ? QT * NQ * 16 : 0));
 
     const int64_t grp = blockIdx.z;
     const int64_t q0 = (int64_t)blockIdx.y * QT;
@@ -54,7 +55,7 @@ score_lut_kernel(const DevState st, const void* __restrict__ q, int qdtype, int6
     for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
     prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * D) * qelem, qdtype,
-                     nqt, qs, qp, u);
+                     nqt, qs, qp, u, stage);
     // tables (queries beyond nqt get zero tables; their scores are not stored)
     for (int i = threadIdx.x; i < QT * NG * Gr::E; i += blockDim.x) {
         const int qi = i / (NG * Gr::E);
@@ -148,7 +149,7 @@ template <int D, int B, bool PROD, int QT>
 size_t lut_smem() {
     using Gr = Groups<B>;
     return (size_t)(kMaxLevels + 3 * QT * D + QT * (D * B / Gr::G) * Gr::E + (PROD ? QT * (D / 4) * 16 : 0)) *
-           sizeof(float);
+               sizeof(float) + kPrepStageBytes;
 }
 
 int sm_count_lut() {

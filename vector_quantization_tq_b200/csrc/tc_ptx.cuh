@@ -165,6 +165,20 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t lb
     return d;
 }
 
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: the layout a TMA tile load
+// with CU_TENSOR_MAP_SWIZZLE_128B writes (rows of 128 bytes, 8-row atoms of 1024 bytes,
+// 16-byte chunks XOR-ed with the row index). Advancing along K inside an atom is done by
+// adding the byte offset to the start address.
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                  // leading byte offset (unused for this layout): 16 B
+    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;                  // layout type: 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor for kind::f16: bf16 A and B (K-major), fp32 D, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                    // D format fp32
