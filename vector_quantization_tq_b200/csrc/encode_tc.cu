@@ -696,7 +696,7 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         pending = true;
     }
     uint32_t xph = 0u, hph = 0u, sph = 0u;
-    bool failed = false;
+    bool failed = false, hmma_pending = false, smma_pending = false;
     const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
     const uint32_t s_addr = ptx::smem_addr(sm.s);
     const uint32_t hd_addr = ptx::smem_addr(sm.hd);
@@ -704,30 +704,32 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     const uint32_t x_addr1 = ptx::smem_addr(sm.x[1]);
 
     for (int64_t tile = t0; tile < ntiles; tile += gridDim.x) {
-        const bool ok = ptx::mbar_wait(&sm.bar_x, xph);
+        // One thread waits for the tile, runs y = (H D) x on the tensor core and waits for
+        // it; the others park on the block barrier instead of spinning.
+        bool ok = true;
+        if (tid == 0) {
+            ok = ptx::mbar_wait(&sm.bar_x, xph);
+            if (ok) {
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = ((kk < 4) ? x_addr0 : x_addr1) + (kk & 3) * 32;
+                    ptx::mma_ss(tmem, ptx::smem_desc_kmajor_sw128(a),
+                                ptx::smem_desc_kmajor(hd_addr + kk * 2 * 2048, 2048, 128), idesc,
+                                kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(&sm.bar_h);
+                ok = ptx::mbar_wait(&sm.bar_h, hph);
+                if (!ok) hmma_pending = true;
+            }
+        }
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
         }
         xph ^= 1u;
-        pending = false;
-        // ---- y = (H D) x on the tensor core ----
-        if (tid == 0) {
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = ((kk < 4) ? x_addr0 : x_addr1) + (kk & 3) * 32;
-                ptx::mma_ss(tmem, ptx::smem_desc_kmajor_sw128(a),
-                            ptx::smem_desc_kmajor(hd_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit(&sm.bar_h);
-        }
-        const bool hok = ptx::mbar_wait(&sm.bar_h, hph);
-        if (__syncthreads_or(!hok)) {
-            failed = true;
-            break;
-        }
         hph ^= 1u;
+        pending = false;
         ptx::tc_fence_after();
         const int64_t nxt = tile + gridDim.x;
         if (nxt < ntiles) {   // the MMA has read the tile: refill the buffer
@@ -822,6 +824,7 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             ptx::tc_fence_before();
             __syncthreads();
             if (half == 0 && row < p.n) p.rnorms[row] = sqrtf(sm.rsq[0][vrow] + sm.rsq[1][vrow]);
+            bool sok = true;
             if (tid == 0) {
                 ptx::tc_fence_after();
 #pragma unroll
@@ -833,8 +836,9 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                     ptx::mma_ts(tmem, tmem + 192 + kk * 8,
                                 ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, 1u);
                 ptx::mma_commit(&sm.bar_s);
+                sok = ptx::mbar_wait(&sm.bar_s, sph);
+                if (!sok) smma_pending = true;
             }
-            const bool sok = ptx::mbar_wait(&sm.bar_s, sph);
             if (__syncthreads_or(!sok)) {
                 failed = true;
                 break;
@@ -862,9 +866,11 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
     if (failed) {
         if (tid == 0) atomicExch(&g_tq_device_error, 1);
-        if (pending) (void)ptx::mbar_wait(&sm.bar_x, xph);
-        (void)ptx::mbar_wait(&sm.bar_h, hph, 100000000ull);
-        if (PROD) (void)ptx::mbar_wait(&sm.bar_s, sph, 100000000ull);
+        if (tid == 0) {
+            if (pending) (void)ptx::mbar_wait(&sm.bar_x, xph);
+            if (hmma_pending) (void)ptx::mbar_wait(&sm.bar_h, hph, 100000000ull);
+            if (smma_pending) (void)ptx::mbar_wait(&sm.bar_s, sph, 100000000ull);
+        }
     }
     __syncthreads();
     if (warp == 0) {
