@@ -173,6 +173,8 @@ CASES = [
     (256, 4, tq.PROD, tq.ROT_DENSE, tq.F32), (512, 3, tq.MSE, tq.ROT_RHT, tq.F32),
     (1536, 2, tq.PROD, tq.ROT_DENSE, tq.BF16), (128, 1, tq.PROD, tq.ROT_DENSE, tq.F32),
     (128, 6, tq.MSE, tq.ROT_DENSE, tq.F32), (2048, 1, tq.PROD, tq.ROT_RHT, tq.BF16),
+    (512, 2, tq.PROD, tq.ROT_DENSE, tq.BF16), (1536, 3, tq.MSE, tq.ROT_DENSE, tq.BF16),
+    (1024, 4, tq.PROD, tq.ROT_DENSE, tq.BF16),
 ]
 
 
@@ -289,6 +291,23 @@ def test_tc_encoder(b, mode, n, pad):
     xd = dev_bf16(buf)[:, :d]
     enc = pair.encode(synth.bf16_from_bits(bits))
     gpu, gplanes = gpu_encode(pair, xd, n)
+    tq.device_status(0)
+    bad = check_codes(pair, gpu, enc)
+    xt_o = pair.decode(enc)
+    xt_g = gpu_dequant(pair, gplanes, n)
+    assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2
+
+
+# --------------------------------------------------------------------------------------
+# The dense tensor-core encoder (d >= 512, Pi and S bf16, bf16 input): several M tiles and
+# a ragged tail, more than one pass of its internal chunking.
+# --------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,b,mode,n", [(1536, 2, 1, 5000), (512, 3, 1, 70000), (1536, 1, 0, 300)])
+def test_dense_gemm_encoder(d, b, mode, n):
+    pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.BF16)
+    bits, _ = synth.mixture_vectors(n, d, seed=57)
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    gpu, gplanes = gpu_encode(pair, dev_bf16(bits), n)
     tq.device_status(0)
     bad = check_codes(pair, gpu, enc)
     xt_o = pair.decode(enc)

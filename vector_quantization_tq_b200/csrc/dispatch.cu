@@ -11,8 +11,33 @@ bool encode_tc_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
 int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl,
                      float* norms, float* rnorms, void* stream);
 
+bool encode_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
+size_t encode_gemm_ws_bytes(int d, int64_t n);
+int launch_encode_gemm(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl,
+                       float* norms, float* rnorms, void* ws, void* stream);
+
+// Vectors per pass of the dense tensor-core encoder; bounds its stream-ordered workspace
+// (a bf16 residual pair per coordinate: 65536 x 1536 x 4 B = 384 MiB at d = 1536).
+constexpr int64_t kGemmChunk = 65536;
+
 int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
                   uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+    if (encode_gemm_supported(st, dtype, n, ld)) {
+        cudaStream_t s = (cudaStream_t)stream;
+        const int64_t chunk = n < kGemmChunk ? n : kGemmChunk;
+        void* ws = nullptr;
+        cudaError_t e = cudaMallocAsync(&ws, encode_gemm_ws_bytes(st.d, chunk), s);
+        if (e != cudaSuccess) return (int)e;
+        int rc = 0;
+        for (int64_t c0 = 0; c0 < n && rc == 0; c0 += chunk) {
+            const int64_t cn = (n - c0 < chunk) ? n - c0 : chunk;
+            rc = launch_encode_gemm(st, reinterpret_cast<const uint16_t*>(x) + c0 * ld, cn, ld,
+                                    codes + c0 * st.code_bytes, qjl ? qjl + c0 * st.qjl_bytes : nullptr,
+                                    norms + c0, rnorms ? rnorms + c0 : nullptr, ws, stream);
+        }
+        e = cudaFreeAsync(ws, s);
+        return rc ? rc : (int)e;
+    }
     if (encode_tc_supported(st, dtype, n, ld))
         return launch_encode_tc(st, x, n, ld, codes, qjl, norms, rnorms, stream);
     return launch_encode_generic(st, x, dtype, n, ld, codes, qjl, norms, rnorms, stream);

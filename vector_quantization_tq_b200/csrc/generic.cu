@@ -611,6 +611,17 @@ search_merge_kernel(int64_t ncand, int k, const float* __restrict__ cand_v, cons
     }
 }
 
+}  // namespace
+
+int launch_search_merge(int64_t nq, int64_t ncand, int k, const float* cand_v, const int64_t* cand_i, int64_t* idx,
+                        float* vals, void* stream) {
+    search_merge_kernel<<<(unsigned)nq, kSearchThreads, 0, (cudaStream_t)stream>>>(ncand, k, cand_v, cand_i, idx,
+                                                                                   vals);
+    return (int)cudaGetLastError();
+}
+
+namespace {
+
 // ------------------------------------------------------------------------------------
 // launch helpers
 // ------------------------------------------------------------------------------------
@@ -810,18 +821,31 @@ int64_t search_blocks(int64_t n, int d) {
 }
 }  // namespace
 
+bool search_tc_supported(const DevState& st, int qdtype, int k);
+size_t search_tc_ws_bytes(const DevState& st, int64_t nq, int64_t n, int k);
+int launch_search_tc(const DevState& st, const void* q, int qdtype, int64_t nq, const uint8_t* codes,
+                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int k, int64_t* idx,
+                     float* vals, void* ws, void* stream);
+
 size_t search_workspace_bytes(const DevState& st, int64_t nq, int64_t n, int k) {
     if (nq <= 0 || n <= 0) return 0;
     const size_t nc = (size_t)nq * search_blocks(n, st.d) * k;
     size_t b = nc * sizeof(float);
     b = (b + 255) & ~(size_t)255;
-    return b + nc * sizeof(int64_t);
+    b += nc * sizeof(int64_t);
+    if (search_tc_supported(st, TQ_BF16, k)) {
+        const size_t t = search_tc_ws_bytes(st, nq, n, k);
+        if (t > b) b = t;
+    }
+    return b;
 }
 
 int launch_search(const DevState& st, const void* q, int qdtype, int64_t nq, const uint8_t* codes,
                   const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int k, int64_t* idx,
                   float* vals, void* ws, size_t ws_bytes, void* stream) {
     (void)ws_bytes;
+    if (search_tc_supported(st, qdtype, k) && nq <= (1 << 20))
+        return launch_search_tc(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, k, idx, vals, ws, stream);
     cudaStream_t s = (cudaStream_t)stream;
     const int bk = search_block_keys(st.d);
     const int64_t nblk = search_blocks(n, st.d);
