@@ -236,6 +236,21 @@ int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void*
                              const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                              float scale, float* out, void* stream);
 
+/*
+ * Distortion and inner-product error statistics of reconstructions, for the distortion /
+ * bias sweep (Jump2Paper review: Theorem 1 gives D_mse = E||x - x~||^2; Theorem 2 gives an
+ * unbiased <q, x~> for prod; the motivation paragraph gives the 2/pi slope of the 1-bit MSE
+ * quantizer). Inputs fp32 row-major: x and xt [n][d] (original and reconstruction, e.g. from
+ * tq_dequant), q [nq][d]. Writes 6 fp64 sums to the device buffer `out`:
+ *   out[0] = sum_i ||x_i - xt_i||^2     out[1] = sum_i ||x_i||^2
+ *   out[2] = sum_{q,i} e                out[3] = sum e^2          with a = <q, x_i>,
+ *   out[4] = sum a b                    out[5] = sum a^2               b = <q, xt_i>, e = b - a.
+ * `out` is zeroed first on `stream`. d <= 256 (TQ_EUNSUPPORTED above). The fp64 sums are
+ * accumulated with atomics, so their last bits can vary from run to run.
+ */
+int tq_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,
+                void* stream, int device);
+
 /* Workspace bytes that tq_search_topk needs. */
 int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes);
 

@@ -313,3 +313,37 @@ def test_dense_gemm_encoder(d, b, mode, n):
     xt_o = pair.decode(enc)
     xt_g = gpu_dequant(pair, gplanes, n)
     assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2
+
+
+# --------------------------------------------------------------------------------------
+# Tensor-core search (1-bit prod codes, dense Pi and S bf16): several query tiles and key
+# tiles with ragged tails; top-k against the oracle's estimates.
+# --------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,n,nq,k,qf32", [(512, 10000, 200, 10, False), (1536, 5000, 37, 16, True),
+                                            (512, 300, 5, 7, False)])
+def test_search_topk_tensor_core(d, n, nq, k, qf32):
+    pair = Pair(tq, d, 2, tq.PROD, tq.ROT_DENSE, tq.BF16)
+    bits, _ = synth.mixture_vectors(n, d, seed=61, centres=32)
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    xt = pair.decode(enc)
+    qbits, _ = synth.mixture_vectors(nq, d, seed=62, centres=32, centre_seed=61)
+    qv = synth.bf16_from_bits(qbits)
+    est = OQ.estimate(qv, xt)
+    oidx, ovals = OA.topk(est, k)
+    planes = planes_to_dev(pair.packed(enc))
+    qd = dev_f32(qv) if qf32 else dev_bf16(qbits)
+    idx = torch.empty((nq, k), dtype=torch.int64, device="cuda")
+    vals = torch.empty((nq, k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(tq.search_workspace(pair.st, nq, n, k), dtype=torch.uint8, device="cuda")
+    tq.search_topk(pair.st, qd, *planes, k, idx, vals, ws)
+    torch.cuda.synchronize()
+    tq.device_status(0)
+    gi, gv = host(idx), host(vals)
+    for i in range(nq):
+        assert len(set(gi[i].tolist())) == k
+        np.testing.assert_allclose(gv[i], est[i, gi[i]], atol=ABS_SCORE)
+        assert np.all(np.diff(gv[i]) <= ABS_SCORE)
+        kth = ovals[i, -1]
+        for j in range(k):
+            if gi[i, j] not in oidx[i]:
+                assert est[i, gi[i, j]] >= kth - ABS_SCORE

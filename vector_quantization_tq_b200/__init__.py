@@ -22,7 +22,7 @@ __all__ = [
     "MSE", "PROD", "ROT_DENSE", "ROT_RHT", "F32", "BF16",
     "build_codebook", "draw_gaussian", "draw_signs", "haar_rotation",
     "State", "quantize_mse", "quantize_prod", "dequant", "score",
-    "attend_workspace", "attend_decode", "attend_decode_noalloc", "search_workspace", "search_topk",
+    "attend_workspace", "attend_decode", "attend_decode_noalloc", "ip_stats", "search_workspace", "search_topk",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,7 @@ _SIGS = {
     "tq_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
     "tq_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _SZ, _P]),
     "tq_attend_decode_noalloc": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P]),
+    "tq_ip_stats": (_I, [_P, _P, _I64, _I, _P, _I64, _P, _P, _I]),
     "tq_search_workspace": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_SZ)]),
     "tq_search_topk": (_I, [_P, _P, _I, _I64, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
 }
@@ -333,6 +334,13 @@ def attend_decode_noalloc(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms
     _check(_lib.tq_attend_decode_noalloc(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, _ptr(kcodes),
                                          _ptr(kqjl), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
                                          float(scale), _ptr(out), _stream(stream)), "tq_attend_decode_noalloc")
+
+
+def ip_stats(x, xt, q, out, device: int = 0, stream=None):
+    """Six fp64 sums (see tq.h) of reconstruction and inner-product errors into `out` (device)."""
+    n, d = x.shape
+    _check(_lib.tq_ip_stats(_ptr(x), _ptr(xt), n, d, _ptr(q), q.shape[0], _ptr(out), _stream(stream), device),
+           "tq_ip_stats")
 
 
 def search_workspace(st: State, nq: int, n: int, k: int) -> int:

@@ -559,6 +559,17 @@ int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void*
                                                   scratch, kAttendStaticScratchBytes, stream));
 }
 
+int tq_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,
+                void* stream, int device) {
+    if (n < 0 || nq < 0 || d < 1 || !out || device < 0) return TQ_EINVAL;
+    if (d > 256) return TQ_EUNSUPPORTED;
+    if (n > 0 && (!x || !xt)) return TQ_EINVAL;
+    if (nq > 0 && !q) return TQ_EINVAL;
+    DeviceGuard g(device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_ip_stats(x, xt, n, d, q, nq, out, stream));
+}
+
 int tq_search_workspace(const tq_state* st, int64_t nq, int64_t n, int k, size_t* bytes) {
     if (!st || !bytes || nq < 0 || n < 0 || k < 1 || k > 64) return TQ_EINVAL;
     *bytes = search_workspace_bytes(st->dev, nq, n, k);

@@ -73,6 +73,8 @@ int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, 
                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
                  const float* rnorms, int64_t n, float* scores, void* stream);
 int read_device_error(int* flag);
+int launch_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,
+                    void* stream);
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
                   int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
