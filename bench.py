@@ -41,6 +41,24 @@ SCORE_BYTES_PER_KEY = (BITS - 1) * D // 8 + D // 8 + 8 + 4
 WORKLOAD = "turboquant_prod b=3 RHT prefill encode of KV keys [1,32,32768,128] bf16 + one decode query per head scored"
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank quantizes its own batch (weak scaling): a distinct data seed per rank."""
+    return synth.SEED_DATA + 100 * rank
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, in millions."""
+    return units_per_rank * world / (ms / 1e3) / 1e6
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -48,6 +66,15 @@ def measured_peaks():
             m = json.load(f)
         return float(m["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Measured dense bf16 peak (burst: the kernels are timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
 
 
 def stored_traffic(kernel_key: str):
@@ -174,6 +201,61 @@ def measure_decode(tq, torch, dev, stream, steps: int, warmup: int, peak: float)
             "gpu_launches_per_step": 2}
 
 
+# Embedding search (1,000,000 vectors, d = 1536, prod b = 2, dense Pi and S bf16, 1000 queries):
+# algorithmic flops: encode 4 d^2 per vector (Pi x and S r); search 4 d per (query, key).
+C5_N, C5_D, C5_NQ, C5_K = 1_000_000, 1536, 1000, 10
+
+
+def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: float):
+    """Time the dense tensor-core encode and the top-10 search on the embedding-search shape."""
+    d = C5_D
+    st = tq.State(d, 2, tq.PROD, tq.ROT_DENSE, tq.BF16, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0),
+                  s=synth.gaussian_matrix(d, synth.SEED_S))
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    mu = torch.randn(256, d, generator=g, device=dev)
+    mu /= mu.norm(dim=1, keepdim=True)
+    lab = torch.randint(0, 256, (C5_N,), generator=g, device=dev)
+    x = mu[lab] + 0.3 * torch.randn(C5_N, d, generator=g, device=dev) / d ** 0.5
+    x = (x / x.norm(dim=1, keepdim=True)).to(torch.bfloat16)
+    qlab = torch.randint(0, 256, (C5_NQ,), generator=g, device=dev)
+    qv = mu[qlab] + 0.3 * torch.randn(C5_NQ, d, generator=g, device=dev) / d ** 0.5
+    qv = (qv / qv.norm(dim=1, keepdim=True)).to(torch.bfloat16)
+    codes, qjl, norms, rnorms = st.empty_planes(C5_N, dev)
+    idx = torch.empty((C5_NQ, C5_K), dtype=torch.int64, device=dev)
+    vals = torch.empty((C5_NQ, C5_K), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.search_workspace(st, C5_NQ, C5_N, C5_K), dtype=torch.uint8, device=dev)
+
+    def enc():
+        tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
+
+    def srch():
+        tq.search_topk(st, qv, codes, qjl, norms, rnorms, C5_K, idx, vals, ws, stream=stream)
+
+    out = {}
+    for name, fn, flops in (("encode", enc, 4.0 * d * d * C5_N), ("search", srch, 4.0 * d * C5_NQ * C5_N)):
+        for _ in range(max(2, min(warmup, 3))):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(2, min(steps, 5))
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / reps
+        tf = flops / (ms / 1e3) / 1e12
+        out[name] = {"ms": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": tflops_peak,
+                                            "unit": "TFLOP/s", "frac": tf / tflops_peak,
+                                            "algorithmic_flops_per_launch": flops}}
+    out["encode"]["mvec_s"] = C5_N / (out["encode"]["ms"] / 1e3) / 1e6
+    out["workload"] = ("embedding search: 1,000,000 x 1536 bf16 (Gaussian mixture, 256 centres), prod b=2, dense "
+                       "Pi and S bf16 (tensor cores), 1000 queries, top-10")
+    st.close()
+    return out
+
+
 def oracle_sample(heads: int, seed: int):
     """The oracle (fp64 numpy) on `heads` heads of the workload; returns (vectors, seconds, threads)."""
     from oracle import quantizer as OQ
@@ -236,6 +318,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=HEADS, help="smaller batch for profiling runs")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
+    ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -260,7 +343,7 @@ def main():
     st = tq.State(D, BITS, tq.PROD, tq.ROT_RHT, tq.BF16, device=local, signs=synth.rht_signs(D),
                   s=synth.gaussian_matrix(D, synth.SEED_S))
     # each rank its own batch (weak scaling)
-    seed = synth.SEED_DATA + 100 * rank
+    seed = rank_seed(rank)
     kbits = synth.kv_prefill_batch(HEADS, TOKENS, D, seed=seed, head_range=(0, heads)).reshape(nvec, D)
     qbits = synth.decode_queries(HEADS, D)[:heads]
     x = torch.from_numpy(kbits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -301,9 +384,7 @@ def main():
     sc_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     step_ms = total_ms / args.steps
     if world > 1:
-        t = torch.tensor([step_ms, enc_ms, sc_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, enc_ms, sc_ms = [float(v) for v in t.tolist()]
+        step_ms, enc_ms, sc_ms = max_over_ranks([step_ms, enc_ms, sc_ms], dist, dev)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -343,12 +424,10 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms = s0.elapsed_time(s1) / ne2e
         if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+            e2e_ms = max_over_ranks([e2e_ms], dist, dev)[0]
         h2d = hx.numel() * hx.element_size() + hq.numel() * hq.element_size()
         d2h = sum(t.numel() * t.element_size() for t in (hc, hz, hn, hr, hs))
-        e2e = {"value": nvec * world / (e2e_ms / 1e3) / 1e6, "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_rate(nvec, world, e2e_ms), "unit": "Mvec/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     cpu = None
@@ -362,12 +441,15 @@ def main():
     decode = None
     if not args.no_decode:
         decode = measure_decode(tq, torch, dev, stream, args.steps, args.warmup, peak)
+    c5 = None
+    if not args.no_c5:
+        c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak())
     enc_gbs = ENC_BYTES_PER_VEC * nvec / (enc_ms / 1e3) / 1e9
     sc_gbs = SCORE_BYTES_PER_KEY * nvec / (sc_ms / 1e3) / 1e9
     traffic = stored_traffic("encode_prod_d128")
     line = {
         "metric": METRIC,
-        "value": nvec * world / (step_ms / 1e3) / 1e6,
+        "value": job_rate(nvec, world, step_ms),
         "unit": "Mvec/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -393,6 +475,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": e2e,
         "decode_attention": decode,
+        "embedding_search": c5,
         "cpu_baseline": cpu,
     }
     if rank == 0:

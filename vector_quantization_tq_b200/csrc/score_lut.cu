@@ -30,62 +30,79 @@ struct Groups {
     static constexpr int E = 1 << G;                     // entries per table
 };
 
+template <int D, int B, bool PROD>
+struct LutShape {
+    using Gr = Groups<B>;
+    static constexpr int NG = D * B / Gr::G;        // MSE tables per query
+    static constexpr int NQ = D / 4;                // QJL tables per query
+    static constexpr int MSE = NG * Gr::E;          // floats
+    static constexpr int QJL = PROD ? NQ * 16 : 0;  // floats
+    static constexpr int SIZE = MSE + QJL;          // floats per query (a multiple of 4)
+};
+
+// One block per query: q' = Pi q, u = S q', then the tables, written to `luts`.
+template <int D, int B, bool PROD>
+__global__ void __launch_bounds__(kThreads)
+score_prep_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts) {
+    using Gr = Groups<B>;
+    using LS = LutShape<D, B, PROD>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float* ctab = reinterpret_cast<float*>(smem_raw);
+    float* qs = ctab + kMaxLevels;
+    float* qp = qs + D;
+    float* u = qp + D;
+    unsigned char* stage = reinterpret_cast<unsigned char*>(u + D);
+    const int64_t qi = blockIdx.x;   // flat query index (group-major)
+    for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
+    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
+    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)qi * D * qelem, qdtype, 1, qs, qp, u,
+                     stage);
+    float* out = luts + qi * LS::SIZE;
+    for (int i = threadIdx.x; i < LS::MSE; i += blockDim.x) {
+        const int k = i / Gr::E, e = i % Gr::E;
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < Gr::CPG; ++c)
+            a = fmaf(qp[k * Gr::CPG + c], ctab[(e >> (B * c)) & ((1 << B) - 1)], a);
+        out[i] = a;
+    }
+    if constexpr (PROD) {
+        for (int i = threadIdx.x; i < LS::QJL; i += blockDim.x) {
+            const int k = i / 16, e = i % 16;
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = u[4 * k + c];
+                a += ((e >> c) & 1) ? v : -v;
+            }
+            out[LS::MSE + i] = a;
+        }
+    }
+}
+
 template <int D, int B, bool PROD, int QT>
 __global__ void __launch_bounds__(kThreads)
-score_lut_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t nq,
+score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
                  const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
                  const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
                  int keys_per_block, float* __restrict__ scores) {
     using Gr = Groups<B>;
-    constexpr int NG = D * B / Gr::G;      // MSE tables per query
-    constexpr int NQ = D / 4;              // QJL tables per query
+    using LS = LutShape<D, B, PROD>;
+    constexpr int NG = LS::NG;
+    constexpr int NQ = LS::NQ;
     constexpr int CW = D * B / 32;         // code words per key
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float* ctab = reinterpret_cast<float*>(smem_raw);          // kMaxLevels
-    float* qs = ctab + kMaxLevels;                              // QT*D
-    float* qp = qs + QT * D;                                    // QT*D
-    float* u = qp + QT * D;                                     // QT*D
-    float* tm = u + QT * D;                                     // QT*NG*E
-    float* tz = tm + QT * NG * Gr::E;                           // QT*NQ*16 (prod)
-    unsigned char* stage = reinterpret_cast<unsigned char*>(tz + (PROD ? QT * NQ * 16 : 0));
+    float* tab = reinterpret_cast<float*>(smem_raw);   // QT x SIZE
 
     const int64_t grp = blockIdx.z;
     const int64_t q0 = (int64_t)blockIdx.y * QT;
     const int nqt = (int)((nq - q0) < QT ? (nq - q0) : QT);
-    for (int i = threadIdx.x; i < st.L; i += blockDim.x) ctab[i] = st.c[i];
-    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries_dev(st, reinterpret_cast<const unsigned char*>(q) + (size_t)((grp * nq + q0) * D) * qelem, qdtype,
-                     nqt, qs, qp, u, stage);
-    // tables (queries beyond nqt get zero tables; their scores are not stored)
-    for (int i = threadIdx.x; i < QT * NG * Gr::E; i += blockDim.x) {
-        const int qi = i / (NG * Gr::E);
-        const int k = (i / Gr::E) % NG;
-        const int e = i % Gr::E;
-        float a = 0.f;
-        if (qi < nqt) {
-#pragma unroll
-            for (int c = 0; c < Gr::CPG; ++c) {
-                const int j = k * Gr::CPG + c;
-                a = fmaf(qp[qi * D + j], ctab[(e >> (B * c)) & ((1 << B) - 1)], a);
-            }
-        }
-        tm[i] = a;
-    }
-    if constexpr (PROD) {
-        for (int i = threadIdx.x; i < QT * NQ * 16; i += blockDim.x) {
-            const int qi = i / (NQ * 16);
-            const int k = (i / 16) % NQ;
-            const int e = i % 16;
-            float a = 0.f;
-            if (qi < nqt) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float v = u[qi * D + 4 * k + c];
-                    a += ((e >> c) & 1) ? v : -v;
-                }
-            }
-            tz[i] = a;
-        }
+    {
+        const float4* src = reinterpret_cast<const float4*>(luts + (grp * nq + q0) * LS::SIZE);
+        float4* dst = reinterpret_cast<float4*>(tab);
+        for (int i = threadIdx.x; i < nqt * LS::SIZE / 4; i += kThreads) dst[i] = __ldg(src + i);
+        for (int i = nqt * LS::SIZE / 4 + threadIdx.x; i < QT * LS::SIZE / 4; i += kThreads)
+            dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
 
@@ -102,6 +119,18 @@ score_lut_kernel(const DevState st, const void* __restrict__ q, int qdtype, int6
                 w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
             }
         }
+        uint32_t z[PROD ? D / 32 : 1];
+        float g2 = 0.f;
+        if constexpr (PROD) {
+            const uint4* zs = reinterpret_cast<const uint4*>(qjl + gk * (D / 8));
+#pragma unroll
+            for (int i = 0; i < D / 128; ++i) {
+                const uint4 v = __ldg(zs + i);
+                z[4 * i] = v.x; z[4 * i + 1] = v.y; z[4 * i + 2] = v.z; z[4 * i + 3] = v.w;
+            }
+            g2 = __ldg(rnorms + gk) * st.qjl_scale;
+        }
+        const float nu = __ldg(norms + gk);
         float a1[QT];
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) a1[qi] = 0.f;
@@ -116,40 +145,28 @@ score_lut_kernel(const DevState st, const void* __restrict__ q, int qdtype, int6
                 e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (Gr::E - 1);
             }
 #pragma unroll
-            for (int qi = 0; qi < QT; ++qi) a1[qi] += tm[(qi * NG + k) * Gr::E + e];
+            for (int qi = 0; qi < QT; ++qi) a1[qi] += tab[qi * LS::SIZE + k * Gr::E + e];
         }
         float a2[QT];
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) a2[qi] = 0.f;
-        float g2 = 0.f;
         if constexpr (PROD) {
-            uint32_t z[D / 32];
-            const uint4* zs = reinterpret_cast<const uint4*>(qjl + gk * (D / 8));
-#pragma unroll
-            for (int i = 0; i < D / 128; ++i) {
-                const uint4 v = __ldg(zs + i);
-                z[4 * i] = v.x; z[4 * i + 1] = v.y; z[4 * i + 2] = v.z; z[4 * i + 3] = v.w;
-            }
 #pragma unroll
             for (int k = 0; k < NQ; ++k) {
                 const uint32_t e = (z[k >> 3] >> ((k & 7) * 4)) & 15u;
 #pragma unroll
-                for (int qi = 0; qi < QT; ++qi) a2[qi] += tz[(qi * NQ + k) * 16 + e];
+                for (int qi = 0; qi < QT; ++qi) a2[qi] += tab[qi * LS::SIZE + LS::MSE + k * 16 + e];
             }
-            g2 = __ldg(rnorms + gk) * st.qjl_scale;
         }
-        const float nu = __ldg(norms + gk);
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi)
             if (qi < nqt) scores[(grp * nq + q0 + qi) * n + key] = nu * fmaf(g2, a2[qi], a1[qi]);
     }
 }
 
-template <int D, int B, bool PROD, int QT>
-size_t lut_smem() {
-    using Gr = Groups<B>;
-    return (size_t)(kMaxLevels + 3 * QT * D + QT * (D * B / Gr::G) * Gr::E + (PROD ? QT * (D / 4) * 16 : 0)) *
-               sizeof(float) + kPrepStageBytes;
+template <int D, int B, bool PROD>
+size_t prep_smem() {
+    return (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
 }
 
 int sm_count_lut() {
@@ -167,25 +184,38 @@ template <int D, int B, bool PROD, int QT>
 int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
                cudaStream_t s) {
-    auto kern = score_lut_kernel<D, B, PROD, QT>;
-    const size_t smem = lut_smem<D, B, PROD, QT>();
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return (int)e;
-    }
+    using LS = LutShape<D, B, PROD>;
     const int64_t qtiles = (nq + QT - 1) / QT;
-    if (qtiles > 65535 || groups > 65535) return (int)cudaErrorInvalidConfiguration;
-    // Enough blocks for a few waves, at least 1024 keys per block so the table set-up
-    // stays small next to the scoring.
-    const int64_t want_blocks = (int64_t)sm_count_lut() * 8;
-    int64_t per = (n * qtiles * groups + want_blocks - 1) / want_blocks;
-    per = std::max<int64_t>(per, 1024);
-    per = (per + kThreads - 1) / kThreads * kThreads;
-    const int64_t kb = (n + per - 1) / per;
-    if (kb > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)kb, (unsigned)qtiles, (unsigned)groups);
-    kern<<<grid, kThreads, smem, s>>>(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, (int)per, scores);
-    return (int)cudaGetLastError();
+    if (qtiles > 65535 || groups > 65535 || groups * nq > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
+    // Per-query tables in a stream-ordered scratch buffer, built once per query.
+    float* luts = nullptr;
+    cudaError_t ce = cudaMallocAsync(reinterpret_cast<void**>(&luts), (size_t)groups * nq * LS::SIZE * sizeof(float), s);
+    if (ce != cudaSuccess) return (int)ce;
+    auto prep = score_prep_kernel<D, B, PROD>;
+    const size_t psmem = prep_smem<D, B, PROD>();
+    if (psmem > 48 * 1024) cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    prep<<<(unsigned)(groups * nq), kThreads, psmem, s>>>(st, q, qdtype, luts);
+    ce = cudaGetLastError();
+    if (ce == cudaSuccess) {
+        auto kern = score_lut_kernel<D, B, PROD, QT>;
+        const size_t smem = (size_t)QT * LS::SIZE * sizeof(float);
+        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        // A few waves of blocks; at least 1024 keys per block.
+        const int64_t want_blocks = (int64_t)sm_count_lut() * 8;
+        int64_t per = (n * qtiles * groups + want_blocks - 1) / want_blocks;
+        per = std::max<int64_t>(per, 1024);
+        per = (per + kThreads - 1) / kThreads * kThreads;
+        const int64_t kb = (n + per - 1) / per;
+        if (kb > (1ll << 31) - 1) {
+            ce = cudaErrorInvalidConfiguration;
+        } else {
+            dim3 grid((unsigned)kb, (unsigned)qtiles, (unsigned)groups);
+            kern<<<grid, kThreads, smem, s>>>(st, luts, nq, codes, qjl, norms, rnorms, n, (int)per, scores);
+            ce = cudaGetLastError();
+        }
+    }
+    cudaError_t fe = cudaFreeAsync(luts, s);
+    return (int)(ce != cudaSuccess ? ce : fe);
 }
 
 template <int D, int B, bool PROD>
