@@ -35,6 +35,32 @@ struct KGroups {
     static constexpr int NG = kD * B / G;
 };
 
+// Asynchronous global -> shared copies (16 bytes, L2 only; 4 bytes through L1).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// One tile of a head's compressed cache in shared memory.
+template <int BK, bool KPROD, int BV>
+struct TileBuf {
+    static constexpr int KROW = kD * BK / 8;   // bytes of key codes per token
+    static constexpr int VROW = kD * BV / 8;   // bytes of value codes per token
+    uint8_t kc[kThreads * KROW];
+    uint8_t kz[KPROD ? kThreads * 16 : 16];
+    uint8_t vc[kThreads * VROW];
+    float kn[kThreads];
+    float kr[kThreads];
+    float vn[kThreads];
+};
+
 template <int BK, bool KPROD, int BV>
 __global__ void __launch_bounds__(kThreads)
 attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__ q, int qdtype, int64_t T,
@@ -43,10 +69,12 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
                   const uint8_t* __restrict__ vcodes, const float* __restrict__ vnorms, float scale,
                   float* __restrict__ part) {
     using KG = KGroups<BK>;
+    using TB = TileBuf<BK, KPROD, BV>;
     constexpr int NQ = kD / 4;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float* ctab = reinterpret_cast<float*>(smem_raw);           // kMaxLevels (K centroids)
-    float* vc = ctab + kMaxLevels;                               // 16 (V centroids), padded to 32
+    TB* tb = reinterpret_cast<TB*>(smem_raw);                    // 2 stages
+    float* ctab = reinterpret_cast<float*>(tb + 2);             // kMaxLevels (K centroids)
+    float* vc = ctab + kMaxLevels;                               // 32 (V centroids)
     float* qs = vc + 32;                                         // kD
     float* qp = qs + kD;                                         // kD
     float* u = qp + kD;                                          // kD
@@ -55,12 +83,41 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
     float* wt = tz + NQ * 16;                                    // kThreads
     float* red = wt + kThreads;                                  // 32
     float* accw = red + 32;                                      // kWarps * kD
-    unsigned char* stage = reinterpret_cast<unsigned char*>(accw + kWarps * kD);
+    // the query preparation's staging buffer aliases tile buffer 1, first written in the loop
+    static_assert(sizeof(TB) >= kPrepStageBytes, "tile buffer too small to alias");
+    unsigned char* stage = reinterpret_cast<unsigned char*>(tb + 1);
 
     const int h = blockIdx.y;
     const int split = blockIdx.x;
     const int nsplit = gridDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t t_begin = (int64_t)split * chunk;
+    const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
+    const int64_t hT = (int64_t)h * T;
+
+    // Stage a tile (tokens t0 .. t0+255 of this head) into buffer `sb`; rows past the end of
+    // this split are not copied and not read.
+    auto stage_tile = [&](int sb, int64_t t0) {
+        TB& B = tb[sb];
+        const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
+        const uint8_t* kc = kcodes + (hT + t0) * TB::KROW;
+        for (int i = threadIdx.x; i < cnt * (TB::KROW / 16); i += kThreads) cp_async16(B.kc + i * 16, kc + i * 16);
+        const uint8_t* vcp = vcodes + (hT + t0) * TB::VROW;
+        for (int i = threadIdx.x; i < cnt * (TB::VROW / 16); i += kThreads) cp_async16(B.vc + i * 16, vcp + i * 16);
+        if ((int)threadIdx.x < cnt) {
+            const int64_t g = hT + t0 + threadIdx.x;
+            if constexpr (KPROD) {
+                cp_async16(B.kz + threadIdx.x * 16, kqjl + g * 16);
+                cp_async4(B.kr + threadIdx.x, krnorms + g);
+            }
+            cp_async4(B.kn + threadIdx.x, knorms + g);
+            cp_async4(B.vn + threadIdx.x, vnorms + g);
+        }
+    };
+
+    if (t_begin < t_end) stage_tile(0, t_begin);
+    cp_async_commit();
+
     for (int i = threadIdx.x; i < ks.L; i += kThreads) ctab[i] = ks.c[i];
     if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
     const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
@@ -87,23 +144,26 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
     }
     __syncthreads();
 
-    const int64_t t_begin = (int64_t)split * chunk;
-    const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
-    const int64_t hT = (int64_t)h * T;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};       // coordinates 4*lane .. 4*lane+3, this warp's tokens
     float m_run = -INFINITY, l_run = 0.f;
-    for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads) {
+    int it = 0;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads, ++it) {
         const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
+        const int sb = it & 1;
+        if (t0 + kThreads < t_end) stage_tile(sb ^ 1, t0 + kThreads);   // prefetch the next tile
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        const TB& B = tb[sb];
         // ---- A: score of token t0 + threadIdx.x ----
         float s = -INFINITY;
         if ((int)threadIdx.x < cnt) {
-            const int64_t gk = hT + t0 + threadIdx.x;
             constexpr int CW = kD * BK / 32;
             uint32_t w[CW];
-            const uint4* src = reinterpret_cast<const uint4*>(kcodes + gk * (kD * BK / 8));
+            const uint4* src = reinterpret_cast<const uint4*>(B.kc + threadIdx.x * TB::KROW);
 #pragma unroll
             for (int i = 0; i < CW / 4; ++i) {
-                const uint4 v = __ldg(src + i);
+                const uint4 v = src[i];
                 w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
             }
             float a1 = 0.f;
@@ -118,13 +178,13 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
             }
             float a2 = 0.f, g2 = 0.f;
             if constexpr (KPROD) {
-                const uint4 zv = __ldg(reinterpret_cast<const uint4*>(kqjl + gk * (kD / 8)));
+                const uint4 zv = *reinterpret_cast<const uint4*>(B.kz + threadIdx.x * 16);
                 const uint32_t z[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
                 for (int k = 0; k < NQ; ++k) a2 += tz[k * 16 + ((z[k >> 3] >> ((k & 7) * 4)) & 15u)];
-                g2 = __ldg(krnorms + gk) * ks.qjl_scale;
+                g2 = B.kr[threadIdx.x] * ks.qjl_scale;
             }
-            s = scale * __ldg(knorms + gk) * fmaf(g2, a2, a1);
+            s = scale * B.kn[threadIdx.x] * fmaf(g2, a2, a1);
         }
         // ---- B: online softmax bookkeeping ----
         const float wm = warp_max(s);
@@ -139,7 +199,7 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
         const float ps = warp_sum(p);
         __syncthreads();   // everyone has read red[] (max) before it is reused
         if (lane == 0) red[warp] = ps;
-        if ((int)threadIdx.x < cnt) wt[threadIdx.x] = p * __ldg(vnorms + hT + t0 + threadIdx.x);
+        if ((int)threadIdx.x < cnt) wt[threadIdx.x] = p * B.vn[threadIdx.x];
         __syncthreads();
         float tsum = 0.f;
 #pragma unroll
@@ -148,28 +208,46 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
         m_run = m_new;
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[c] *= alpha;
-        // ---- C: value sum, one warp per token, 4 coordinates per lane ----
-        for (int t = warp; t < cnt; t += kWarps) {
-            const uint8_t* row = vcodes + (hT + t0 + t) * (kD * BV / 8);
-            const float wv = wt[t];
-            uint32_t bits;
-            if constexpr (BV == 4) {
-                bits = __ldg(reinterpret_cast<const uint16_t*>(row) + lane);
-            } else if constexpr (BV == 2) {
-                bits = __ldg(row + lane);
-            } else {
-                const int b0 = lane * 4 * BV;
-                const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row);
-                const int wi = b0 >> 5, sh = b0 & 31;
-                uint64_t win = __ldg(r32 + wi);
-                if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)__ldg(r32 + wi + 1) << 32;
-                bits = (uint32_t)(win >> sh);
+        // ---- C: value sum, one warp per token, 4 coordinates per lane; 32 tokens per warp ----
+        const int ntok = (cnt - warp + kWarps - 1) / kWarps;   // tokens t = warp + 8 * i < cnt
+        // batches of 8 tokens: the 8 code slices are loaded before their FMAs
+#pragma unroll
+        for (int i0 = 0; i0 < kThreads / kWarps; i0 += 8) {
+            uint32_t bits[8];
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j;
+                const int t = warp + i * kWarps;
+                uint32_t b = 0;
+                float w = 0.f;
+                if (i < ntok) {
+                    const uint8_t* row = B.vc + t * TB::VROW;
+                    if constexpr (BV == 4) {
+                        b = reinterpret_cast<const uint16_t*>(row)[lane];
+                    } else if constexpr (BV == 2) {
+                        b = row[lane];
+                    } else {
+                        const int b0 = lane * 4 * BV;
+                        const int wi = b0 >> 5, sh = b0 & 31;
+                        const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row);
+                        uint64_t win = r32[wi];
+                        if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)r32[wi + 1] << 32;
+                        b = (uint32_t)(win >> sh);
+                    }
+                    w = wt[t];
+                }
+                bits[j] = b;
+                wv[j] = w;
             }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[c] = fmaf(wv, vc[(bits >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[c] = fmaf(wv[j], vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
         }
-        __syncthreads();   // wt / red reused by the next tile
+        __syncthreads();   // wt / red and the tile buffer are reused
     }
+    cp_async_wait0();
     // ---- reduce the warps' value sums and write the split record ----
 #pragma unroll
     for (int c = 0; c < 4; ++c) accw[warp * kD + 4 * lane + c] = acc[c];
@@ -190,8 +268,9 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
 template <int BK, bool KPROD, int BV>
 size_t smem_bytes() {
     using KG = KGroups<BK>;
-    return (size_t)(kMaxLevels + 32 + 3 * kD + KG::NG * KG::E + (kD / 4) * 16 + kThreads + 32 + kWarps * kD) *
-               sizeof(float) + kPrepStageBytes;
+    return 2 * sizeof(TileBuf<BK, KPROD, BV>) +
+           (size_t)(kMaxLevels + 32 + 3 * kD + KG::NG * KG::E + (kD / 4) * 16 + kThreads + 32 + kWarps * kD) *
+               sizeof(float);
 }
 
 template <int BK, bool KPROD, int BV>
@@ -242,8 +321,10 @@ int launch_k(const DevState& ks, const DevState& vs, const void* q, int qdtype, 
 
 }  // namespace
 
-bool attend_lut_supported(const DevState& ks, const DevState& vs) {
-    return ks.d == kD && vs.d == kD && ks.b_mse >= 2 && ks.b_mse <= 4 && vs.b_mse >= 2 && vs.b_mse <= 4;
+bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kcodes, const void* kqjl,
+                          const void* vcodes) {
+    const auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    return a16(kcodes) && a16(vcodes) && (kqjl == nullptr || a16(kqjl)) && ks.d == kD && vs.d == kD && ks.b_mse >= 2 && ks.b_mse <= 4 && vs.b_mse >= 2 && vs.b_mse <= 4;
 }
 
 int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,

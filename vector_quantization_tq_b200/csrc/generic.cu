@@ -731,7 +731,8 @@ int attend_splits(int H, int64_t T) {
 }
 }  // namespace
 
-bool attend_lut_supported(const DevState& ks, const DevState& vs);
+bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kcodes, const void* kqjl,
+                          const void* vcodes);
 int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
                             int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
@@ -753,7 +754,7 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
     const int nsplit = (int)((T + chunk - 1) / chunk);
     float* part = reinterpret_cast<float*>(ws);
     cudaError_t e;
-    if (attend_lut_supported(ks, vs)) {
+    if (attend_lut_supported(ks, vs, kcodes, kqjl, vcodes)) {
         e = (cudaError_t)launch_attend_lut_split(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms,
                                                  krnorms, vcodes, vnorms, scale, part, stream);
     } else {
