@@ -298,6 +298,22 @@ def test_tc_encoder(b, mode, n, pad):
     assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2
 
 
+# The pipelined encoder (b_mse 1 and 2) with several tiles per CTA: more tiles than the TMA
+# ring has stages on every SM, both residual buffers in use, and a ragged last tile.
+@pytest.mark.parametrize("b,mode", [(2, 1), (3, 1), (1, 0), (2, 0)])
+def test_tc_encoder_many_tiles(b, mode):
+    d, n = 128, 148 * 128 * 5 + 77
+    pair = Pair(tq, d, b, mode, tq.ROT_RHT, tq.BF16)
+    bits = synth.kv_prefill_batch(1, n, d, seed=41)[0]
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    gpu, gplanes = gpu_encode(pair, dev_bf16(bits), n)
+    tq.device_status(0)
+    bad = check_codes(pair, gpu, enc)
+    xt_o = pair.decode(enc)
+    xt_g = gpu_dequant(pair, gplanes, n)
+    assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2
+
+
 # --------------------------------------------------------------------------------------
 # The dense tensor-core encoder (d >= 512, Pi and S bf16, bf16 input): several M tiles and
 # a ragged tail, more than one pass of its internal chunking.

@@ -6,9 +6,12 @@
 // (Jump2Paper review, Theorem 2): <q, k~> = ||k|| (sum_j q'_j c[idx_j] + ||r|| sqrt(pi/2)/d
 // sum_j u_j (2 z_j - 1)), q' = Pi_K q, u = S q'.
 //
-// Flash-decoding split over tokens: block (split, h) walks tiles of 256 tokens with an
-// online softmax and writes (m, l, acc[d]) for the combine launch, which merges the splits
-// and applies Pi_V^T once per head. Inside a tile:
+// A table launch first builds, once per head, the lookup tables of q' = Pi_K q against the
+// key code groups and of u = S q' against the QJL nibbles (the scorer's tables).
+// Flash-decoding split over tokens: block (split, h) copies its head's tables, walks tiles
+// of 256 tokens (staged with cp.async, double-buffered) with an online softmax and writes
+// (m, l, acc[d]) for the combine launch, which merges the splits and applies Pi_V^T once
+// per head. Inside a tile:
 //   A. one thread per token scores it through per-query tables over packed code groups
 //      (16- or 64-entry tables in shared memory, as in the LUT scorer);
 //   B. the block updates the running max and sum and forms w_t = p_t ||v_t||;
@@ -17,7 +20,6 @@
 // Only the compressed bytes are read: 72 B (keys, prod b=4) + 68 B (values, mse b=4) per
 // token and head.
 #include "common.cuh"
-#include "prep.cuh"
 
 namespace tq {
 
@@ -29,8 +31,7 @@ constexpr int kWarps = kThreads / 32;
 
 template <int B>
 struct KGroups {
-    static constexpr int G = (B == 3) ? 6 : 4;
-    static constexpr int CPG = G / B;
+    static constexpr int G = (B == 3) ? 6 : 4;   // bits per table index (as in the scorer's tables)
     static constexpr int E = 1 << G;
     static constexpr int NG = kD * B / G;
 };
@@ -63,8 +64,7 @@ struct TileBuf {
 
 template <int BK, bool KPROD, int BV>
 __global__ void __launch_bounds__(kThreads)
-attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__ q, int qdtype, int64_t T,
-                  int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
+attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict__ luts, int64_t T, int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
                   const float* __restrict__ knorms, const float* __restrict__ krnorms,
                   const uint8_t* __restrict__ vcodes, const float* __restrict__ vnorms, float scale,
                   float* __restrict__ part) {
@@ -72,20 +72,14 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
     using TB = TileBuf<BK, KPROD, BV>;
     constexpr int NQ = kD / 4;
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    constexpr int LSIZE = KG::NG * KG::E + (KPROD ? NQ * 16 : 0);   // floats of one query's tables
     TB* tb = reinterpret_cast<TB*>(smem_raw);                    // 2 stages
-    float* ctab = reinterpret_cast<float*>(tb + 2);             // kMaxLevels (K centroids)
-    float* vc = ctab + kMaxLevels;                               // 32 (V centroids)
-    float* qs = vc + 32;                                         // kD
-    float* qp = qs + kD;                                         // kD
-    float* u = qp + kD;                                          // kD
-    float* tm = u + kD;                                          // NG * E
+    float* vc = reinterpret_cast<float*>(tb + 2);               // 32 (V centroids)
+    float* tm = vc + 32;                                         // NG * E
     float* tz = tm + KG::NG * KG::E;                             // NQ * 16
-    float* wt = tz + NQ * 16;                                    // kThreads
+    float* wt = tm + LSIZE;                                      // kThreads
     float* red = wt + kThreads;                                  // 32
     float* accw = red + 32;                                      // kWarps * kD
-    // the query preparation's staging buffer aliases tile buffer 1, first written in the loop
-    static_assert(sizeof(TB) >= kPrepStageBytes, "tile buffer too small to alias");
-    unsigned char* stage = reinterpret_cast<unsigned char*>(tb + 1);
 
     const int h = blockIdx.y;
     const int split = blockIdx.x;
@@ -115,34 +109,12 @@ attend_lut_kernel(const DevState ks, const DevState vs, const void* __restrict__
         }
     };
 
+    // this head's tables (q' against the K code groups, u against the QJL nibbles), built
+    // once per head by the table launch, arrive with the first tile
+    for (int i = threadIdx.x; i < LSIZE / 4; i += kThreads) cp_async16(tm + 4 * i, luts + (int64_t)h * LSIZE + 4 * i);
     if (t_begin < t_end) stage_tile(0, t_begin);
     cp_async_commit();
-
-    for (int i = threadIdx.x; i < ks.L; i += kThreads) ctab[i] = ks.c[i];
     if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
-    const size_t qelem = (qdtype == TQ_F32) ? 4 : 2;
-    prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * kD * qelem, qdtype, 1, qs, qp, u,
-                     stage);
-    for (int i = threadIdx.x; i < KG::NG * KG::E; i += kThreads) {
-        const int k = i / KG::E, e = i % KG::E;
-        float a = 0.f;
-#pragma unroll
-        for (int c = 0; c < KG::CPG; ++c) a = fmaf(qp[k * KG::CPG + c], ctab[(e >> (BK * c)) & ((1 << BK) - 1)], a);
-        tm[i] = a;
-    }
-    if constexpr (KPROD) {
-        for (int i = threadIdx.x; i < NQ * 16; i += kThreads) {
-            const int k = i / 16, e = i % 16;
-            float a = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float v = u[4 * k + c];
-                a += ((e >> c) & 1) ? v : -v;
-            }
-            tz[i] = a;
-        }
-    }
-    __syncthreads();
 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};       // coordinates 4*lane .. 4*lane+3, this warp's tokens
     float m_run = -INFINITY, l_run = 0.f;
@@ -269,12 +241,11 @@ template <int BK, bool KPROD, int BV>
 size_t smem_bytes() {
     using KG = KGroups<BK>;
     return 2 * sizeof(TileBuf<BK, KPROD, BV>) +
-           (size_t)(kMaxLevels + 32 + 3 * kD + KG::NG * KG::E + (kD / 4) * 16 + kThreads + 32 + kWarps * kD) *
-               sizeof(float);
+           (size_t)(32 + KG::NG * KG::E + (KPROD ? (kD / 4) * 16 : 0) + kThreads + 32 + kWarps * kD) * sizeof(float);
 }
 
 template <int BK, bool KPROD, int BV>
-int launch_t(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     auto kern = attend_lut_kernel<BK, KPROD, BV>;
@@ -284,36 +255,36 @@ int launch_t(const DevState& ks, const DevState& vs, const void* q, int qdtype, 
         if (e != cudaSuccess) return (int)e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)H);
-    kern<<<grid, kThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
-                                      scale, part);
+    kern<<<grid, kThreads, smem, s>>>(ks, vs, luts, T, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale,
+                                      part);
     return (int)cudaGetLastError();
 }
 
 template <int BK, bool KPROD>
-int launch_v(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+int launch_v(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     switch (vs.b_mse) {
-        case 2: return launch_t<BK, KPROD, 2>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 2: return launch_t<BK, KPROD, 2>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
-        case 3: return launch_t<BK, KPROD, 3>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 3: return launch_t<BK, KPROD, 3>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
-        case 4: return launch_t<BK, KPROD, 4>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 4: return launch_t<BK, KPROD, 4>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
         default: return (int)cudaErrorInvalidValue;
     }
 }
 
 template <bool KPROD>
-int launch_k(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int nsplit,
+int launch_k(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     switch (ks.b_mse) {
-        case 2: return launch_v<2, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 2: return launch_v<2, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
-        case 3: return launch_v<3, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 3: return launch_v<3, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
-        case 4: return launch_v<4, KPROD>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 4: return launch_v<4, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
         default: return (int)cudaErrorInvalidValue;
     }
@@ -327,14 +298,14 @@ bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kc
     return a16(kcodes) && a16(vcodes) && (kqjl == nullptr || a16(kqjl)) && ks.d == kD && vs.d == kD && ks.b_mse >= 2 && ks.b_mse <= 4 && vs.b_mse >= 2 && vs.b_mse <= 4;
 }
 
-int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T,
                             int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                             float scale, float* part, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    if (kqjl) return launch_k<true>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes,
+    if (kqjl) return launch_k<true>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes,
                                     vnorms, scale, part, s);
-    return launch_k<false>(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
+    return launch_k<false>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
                            scale, part, s);
 }
 

@@ -29,7 +29,9 @@
 
 namespace tq {
 
+namespace {
 __device__ int g_tq_device_error = 0;
+}  // namespace
 
 namespace {
 
@@ -879,6 +881,323 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
 }
 
+// ------------------------------------------------------------------------------------
+// Pipelined tensor-core encoder (b_mse = 1 or 2). One persistent CTA per SM owns all 512
+// TMEM columns. Warp 16 streams tiles of 128 vectors with TMA (kT4Stages deep) and issues
+// the MMAs; warps 0..15 quantize, four warps per group of 32 vectors (TMEM lane quadrant
+// warp % 4), each thread taking 32 of its vector's 128 coordinates. The tensor core runs
+// y = (H D) x for tile k+1 and S r for tile k-1 while the warps quantize tile k.
+// TMEM columns: Y [0,128) y; D [128,256) S r; HL0 [256,384), HL1 [384,512) the residual
+// operand of tiles k even / odd (hi in the first 64 columns, lo in the next 64).
+// Arithmetic per coordinate is that of encode_tc3_kernel: the same fp32 rotation sums, the
+// level decision |y| sc < t against the Lloyd-Max boundary, the bf16 hi + lo residual and
+// the sign of S r read from the fp32 accumulator.
+// ------------------------------------------------------------------------------------
+constexpr int kT4Stages = 3;
+constexpr int kT4Warps = 16;
+constexpr int kT4Threads = (kT4Warps + 1) * 32;
+constexpr uint32_t kT4Cols = 512;
+
+struct __align__(1024) TcSmem4 {
+    uint8_t x[kT4Stages][2][kTile * 128];   // [stage][half]: 128 rows x 128 bytes, 128B-swizzled
+    uint8_t hd[kD * kD * 2];                // H diag(eps), B operand (K-major core matrices)
+    uint8_t s[kD * kD * 2];                 // S, B operand
+    float ssq[2][4][kTile];                 // [tile parity][part]: partial ||H D x||^2
+    float rsq[2][4][kTile];                 // [tile parity][part]: partial ||r||^2
+    uint64_t bar_x[kT4Stages];              // tile landed
+    uint64_t bar_xfree[kT4Stages];          // the rotation MMA has read the stage
+    uint64_t bar_h;                         // y of the current tile is in TMEM
+    uint64_t bar_yfree;                     // all quantizing warps have read y
+    uint64_t bar_hl[2];                     // residual operand written and S r of the previous tile read
+    uint64_t bar_s;                         // S r is in TMEM
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(kT4Threads, 1)
+encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
+    static_assert(B == 1 || B == 2, "the pipelined encoder covers 1- and 2-bit codes");
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem4& sm = *reinterpret_cast<TcSmem4*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int* abort_flag = &sm.abort;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int64_t ntiles = (p.n + kTile - 1) / kTile;
+    const int64_t mytiles = (ntiles > (int64_t)blockIdx.x) ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+    if (tid == 0) {
+        ptx::prefetch_tmap(&tmap);
+        for (int i = 0; i < kT4Stages; ++i) {
+            ptx::mbar_init(&sm.bar_x[i], 1);
+            ptx::mbar_init(&sm.bar_xfree[i], 1);
+        }
+        ptx::mbar_init(&sm.bar_h, 1);
+        ptx::mbar_init(&sm.bar_yfree, kT4Warps);
+        ptx::mbar_init(&sm.bar_hl[0], kT4Warps);
+        ptx::mbar_init(&sm.bar_hl[1], kT4Warps);
+        ptx::mbar_init(&sm.bar_s, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&sm.tmem_base, kT4Cols);
+        ptx::tmem_relinquish();
+    }
+    // H diag(eps): entry (n, k) = (-1)^popcount(n & k) * eps_k, at chunk k/8 of row n.
+    for (int i = tid; i < kD * kD; i += kT4Threads) {
+        const int n = i >> 7, k = i & 127;
+        const uint32_t neg = (__popc(n & k) & 1) ^ ((p.sgn[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u);
+        *reinterpret_cast<uint16_t*>(sm.hd + (k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) =
+            neg ? 0xBF80u : 0x3F80u;
+    }
+    if constexpr (PROD) {
+        for (int i = tid; i < kD * 16; i += kT4Threads) {
+            const int row = i >> 4, c = i & 15;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.s + row * kD + c * 8));
+            *reinterpret_cast<uint4*>(sm.s + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == kT4Warps) {
+        // ---------------- producer: TMA + MMA issue (one thread) ----------------
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
+            const uint32_t s_addr = ptx::smem_addr(sm.s);
+            const uint32_t hd_addr = ptx::smem_addr(sm.hd);
+            uint32_t tma_pend = 0u, tma_par = 0u;   // per stage: load in flight / its phase parity
+            int h_st = -1;
+            uint32_t h_par = 0u;
+            bool s_issued = false;
+            uint32_t s_par = 0u;
+            auto load = [&](int64_t j) {
+                const int st = (int)(j % kT4Stages);
+                const int row0 = (int)((blockIdx.x + j * gridDim.x) * kTile);
+                ptx::mbar_arrive_expect_tx(&sm.bar_x[st], 2 * kTile * 128);
+                ptx::tma_load_2d(sm.x[st][0], &tmap, 0, row0, &sm.bar_x[st]);
+                ptx::tma_load_2d(sm.x[st][1], &tmap, 64, row0, &sm.bar_x[st]);
+                tma_pend |= 1u << st;
+                tma_par = (tma_par & ~(1u << st)) | ((uint32_t)((j / kT4Stages) & 1) << st);
+            };
+            auto issue_s = [&](int64_t j) -> bool {
+                if (!ptx::mbar_wait(&sm.bar_hl[j & 1], (uint32_t)(j >> 1) & 1u) || *abort_flag) return false;
+                ptx::tc_fence_after();
+                const uint32_t hl = tmem + 256u + (uint32_t)(j & 1) * 128u;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem + 128u, hl + kk * 8, ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128),
+                                idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem + 128u, hl + 64 + kk * 8,
+                                ptx::smem_desc_kmajor(s_addr + kk * 2 * 2048, 2048, 128), idesc, 1u);
+                ptx::mma_commit(&sm.bar_s);
+                s_issued = true;
+                s_par = (uint32_t)(j & 1);
+                return true;
+            };
+            for (int64_t j = 0; j < mytiles && j < kT4Stages; ++j) load(j);
+            bool ok = true;
+            for (int64_t k = 0; k < mytiles; ++k) {
+                const int st = (int)(k % kT4Stages);
+                const uint32_t xpar = (uint32_t)((k / kT4Stages) & 1);
+                ok = ptx::mbar_wait(&sm.bar_x[st], xpar);
+                if (!ok) break;
+                tma_pend &= ~(1u << st);
+                if (k > 0) {
+                    ok = ptx::mbar_wait(&sm.bar_yfree, (uint32_t)((k - 1) & 1)) && !*abort_flag;
+                    if (!ok) break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t xa0 = ptx::smem_addr(sm.x[st][0]), xa1 = ptx::smem_addr(sm.x[st][1]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ss(tmem, ptx::smem_desc_kmajor_sw128(((kk < 4) ? xa0 : xa1) + (kk & 3) * 32),
+                                ptx::smem_desc_kmajor(hd_addr + kk * 2 * 2048, 2048, 128), idesc, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&sm.bar_h);
+                ptx::mma_commit(&sm.bar_xfree[st]);
+                h_st = st;
+                h_par = xpar;
+                if (PROD && k > 0) {
+                    ok = issue_s(k - 1);
+                    if (!ok) break;
+                }
+                if (k + kT4Stages < mytiles) {
+                    ok = ptx::mbar_wait(&sm.bar_xfree[st], xpar);
+                    if (!ok) break;
+                    load(k + kT4Stages);
+                }
+            }
+            if (ok && PROD && mytiles > 0) ok = issue_s(mytiles - 1);
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(&g_tq_device_error, 1);
+            }
+            // Drain: every copy and MMA this thread started has finished before the CTA
+            // releases TMEM and shared memory.
+            for (int st = 0; st < kT4Stages; ++st)
+                if ((tma_pend >> st) & 1u) (void)ptx::mbar_wait(&sm.bar_x[st], (tma_par >> st) & 1u);
+            if (h_st >= 0) (void)ptx::mbar_wait(&sm.bar_xfree[h_st], h_par);
+            if (s_issued) (void)ptx::mbar_wait(&sm.bar_s, s_par);
+        }
+    } else {
+        // ---------------- quantizing warps ----------------
+        const int quad = warp & 3, part = warp >> 2;
+        const int vrow = quad * 32 + lane;
+        const int bar_id = 1 + quad;   // named barrier of the four warps sharing these vectors
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const float rsqrt_d = p.rsqrt_d;
+        const float t2 = p.t[2];
+        int64_t prev_row = -1;
+        bool prev_nz = false;
+        bool fail = false;
+        // Signs of S r (in D) for vector `srow`; [(S r)_j >= 0], all ones for a zero vector.
+        auto emit_signs = [&](uint32_t parity, int64_t srow, bool snz) -> bool {
+            bool sok = true;
+            if (lane == 0) sok = ptx::mbar_wait(&sm.bar_s, parity);
+            sok = __shfl_sync(0xffffffffu, sok ? 1 : 0, 0) != 0;
+            ptx::tc_fence_after();
+            uint32_t d[32];
+            ptx::tmem_ld32(t_lane + 128 + part * 32, d);
+            ptx::tmem_wait_ld();
+            uint32_t z0 = 0u, z1 = 0u;
+#pragma unroll
+            for (int j = 15; j >= 0; --j) {
+                z0 = __funnelshift_l(d[j], z0, 1);
+                z1 = __funnelshift_l(d[j + 16], z1, 1);
+            }
+            if (sok && srow < p.n)
+                *reinterpret_cast<uint32_t*>(p.qjl + srow * 16 + part * 4) = snz ? ~(z0 | (z1 << 16)) : 0xffffffffu;
+            return sok;
+        };
+        for (int64_t k = 0; k < mytiles; ++k) {
+            const int kb = (int)(k & 1);
+            const int64_t row = (blockIdx.x + k * gridDim.x) * kTile + vrow;
+            bool ok = true;
+            if (lane == 0) ok = ptx::mbar_wait(&sm.bar_h, (uint32_t)(k & 1));
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            ptx::tc_fence_after();
+            uint32_t a[32];
+            ptx::tmem_ld32(t_lane + part * 32, a);
+            ptx::tmem_wait_ld();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sm.bar_yfree);
+            float2 q0 = f2(0.f, 0.f), q1 = f2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 u0 = f2(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]));
+                const float2 u1 = f2(__uint_as_float(a[4 * i + 2]), __uint_as_float(a[4 * i + 3]));
+                q0 = __ffma2_rn(u0, u0, q0);
+                q1 = __ffma2_rn(u1, u1, q1);
+            }
+            sm.ssq[kb][part][vrow] = (q0.x + q0.y) + (q1.x + q1.y);
+            if (ptx::bar_sync_or(bar_id, 128, !ok || *abort_flag)) {
+                fail = true;
+                break;
+            }
+            // ||H D x||^2 = d ||x||^2
+            const float nu =
+                sqrtf((sm.ssq[kb][0][vrow] + sm.ssq[kb][1][vrow]) + (sm.ssq[kb][2][vrow] + sm.ssq[kb][3][vrow])) *
+                rsqrt_d;
+            const bool nz = nu > 0.f;
+            const float sc = nz ? rsqrt_d / nu : 0.f;
+            const float cs = nz ? p.c[B == 2 ? 2 : 1] : 0.f;   // inner level (b = 2) / the level (b = 1)
+            const float cb = nz ? p.c[B == 2 ? 3 : 1] : 0.f;   // outer level
+            const float dcb = cs - cb;
+            uint32_t np0 = 0u, np1 = 0u, mp0 = 0u, mp1 = 0u;
+            float r[32];
+#pragma unroll
+            for (int j = 15; j >= 0; --j) {
+#pragma unroll
+                for (int hh = 1; hh >= 0; --hh) {
+                    const int jj = j + 16 * hh;
+                    const uint32_t yb = a[jj];
+                    const float ay = fabsf(__uint_as_float(yb));
+                    uint32_t& np = hh ? np1 : np0;
+                    np = __funnelshift_l(yb, np, 1);   // bit jj: y < 0
+                    float mag = cs;
+                    if constexpr (B == 2) {
+                        uint32_t& mp = hh ? mp1 : mp0;
+                        const float dd = fmaf(-ay, sc, t2);                 // > 0: inner level
+                        const float st = __saturatef(dd * 0x1p126f);        // exactly 1 (inner) or 0
+                        mp = __funnelshift_l(__float_as_uint(0.5f - st), mp, 1);   // bit jj: inner
+                        mag = fmaf(st, dcb, cb);
+                    }
+                    const float ar = fmaf(ay, sc, -mag);
+                    r[jj] = __uint_as_float(__float_as_uint(ar) ^ (yb & 0x80000000u));
+                }
+            }
+            const uint32_t np = np0 | (np1 << 16);
+            if (row < p.n) {
+                if constexpr (B == 2) {
+                    const uint32_t mp = mp0 | (mp1 << 16);
+                    const uint32_t hb = ~np, lb = ~(np ^ mp);
+                    *reinterpret_cast<uint2*>(p.codes + row * 32 + part * 8) =
+                        make_uint2(spread16(lb) | (spread16(hb) << 1), spread16(lb >> 16) | (spread16(hb >> 16) << 1));
+                } else {
+                    *reinterpret_cast<uint32_t*>(p.codes + row * 16 + part * 4) = ~np;
+                }
+                if (part == 0) p.norms[row] = nu;
+            }
+            if constexpr (PROD) {
+                float2 e0 = f2(0.f, 0.f), e1 = f2(0.f, 0.f);
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 rp = f2(r[2 * i], r[2 * i + 1]);
+                    if (i & 1) e1 = __ffma2_rn(rp, rp, e1);
+                    else e0 = __ffma2_rn(rp, rp, e0);
+                    const __nv_bfloat162 h = __float22bfloat162_rn(rp);
+                    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+                    const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
+                    const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), rp);
+                    const __nv_bfloat162 lb = __float22bfloat162_rn(l);
+                    hi[i] = hb;
+                    lo[i] = *reinterpret_cast<const uint32_t*>(&lb);
+                }
+                sm.rsq[kb][part][vrow] = (e0.x + e0.y) + (e1.x + e1.y);
+                const uint32_t hl = t_lane + 256u + (uint32_t)kb * 128u;
+                ptx::tmem_st16(hl + part * 16, hi);
+                ptx::tmem_st16(hl + 64 + part * 16, lo);
+                ptx::tmem_wait_st();
+                bool sok = true;
+                if (k > 0) sok = emit_signs((uint32_t)((k - 1) & 1), prev_row, prev_nz);   // previous tile
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sm.bar_hl[kb]);
+                if (ptx::bar_sync_or(bar_id, 128, !sok || *abort_flag)) {
+                    fail = true;
+                    break;
+                }
+                if (part == 0 && row < p.n)
+                    p.rnorms[row] = sqrtf((sm.rsq[kb][0][vrow] + sm.rsq[kb][1][vrow]) +
+                                          (sm.rsq[kb][2][vrow] + sm.rsq[kb][3][vrow]));
+                prev_row = row;
+                prev_nz = nz;
+            }
+        }
+        if constexpr (PROD) {
+            if (!fail && mytiles > 0 && !emit_signs((uint32_t)((mytiles - 1) & 1), prev_row, prev_nz)) fail = true;
+        }
+        if (fail) {
+            *abort_flag = 1;
+            if (lane == 0) atomicExch(&g_tq_device_error, 1);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kT4Cols);
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -938,8 +1257,8 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
         p.sgn[i] = (n0 ? 0x8000u : 0u) | (n1 ? 0x80000000u : 0u);
     }
     constexpr bool kTwo = (B == 1 || B == 2);
-    const size_t smem = (kTwo ? sizeof(TcSmem3) : sizeof(TcSmem)) + 1024;
-    auto kern = kTwo ? encode_tc3_kernel<(B <= 2 ? B : 2), PROD> : encode_tc_kernel<B, PROD>;
+    const size_t smem = (kTwo ? sizeof(TcSmem4) : sizeof(TcSmem)) + 1024;
+    auto kern = kTwo ? encode_tc4_kernel<(B <= 2 ? B : 2), PROD> : encode_tc_kernel<B, PROD>;
     static int attr_set_for_device = -1;   // per instantiation
     int dev = 0;
     cudaGetDevice(&dev);
@@ -949,8 +1268,8 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
         attr_set_for_device = dev;
     }
     const int64_t ntiles = (n + kTile - 1) / kTile;
-    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * 2);
-    kern<<<grid, kTwo ? 2 * kTile : kTile, smem, stream>>>(tmap, p);
+    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * (kTwo ? 1 : 2));
+    kern<<<grid, kTwo ? kT4Threads : kTile, smem, stream>>>(tmap, p);
     return (int)cudaGetLastError();
 }
 
@@ -984,6 +1303,8 @@ int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, u
     }
 }
 
+// Reads and clears the error words of all kernels with bounded waits (one word per
+// translation unit: the library is built without relocatable device code).
 int read_device_error(int* flag) {
     int v = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_tq_device_error, sizeof(int));
@@ -993,7 +1314,12 @@ int read_device_error(int* flag) {
         e = cudaMemcpyToSymbol(g_tq_device_error, &zero, sizeof(int));
         if (e != cudaSuccess) return (int)e;
     }
-    *flag = v;
+    int g = 0, s = 0;
+    int rc = take_device_error_gemm(&g);
+    if (rc) return rc;
+    rc = take_device_error_search(&s);
+    if (rc) return rc;
+    *flag = v | g | s;
     return 0;
 }
 

@@ -20,7 +20,9 @@
 
 namespace tq {
 
-extern __device__ int g_tq_device_error;
+namespace {
+__device__ int g_tq_device_error = 0;
+}  // namespace
 
 namespace {
 
@@ -371,6 +373,19 @@ int launch_gemm_f32(const void* A, int64_t lda, const void* B, int64_t ldb, int 
     p.c = C;
     p.ldc = ldc;
     return run_gemm<256, kStoreF32>(A, lda, B, ldb, p, (cudaStream_t)stream);
+}
+
+int take_device_error_gemm(int* flag) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tq_device_error, sizeof(int));
+    if (e != cudaSuccess) return (int)e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_tq_device_error, &zero, sizeof(int));
+        if (e != cudaSuccess) return (int)e;
+    }
+    *flag = v;
+    return 0;
 }
 
 }  // namespace tq

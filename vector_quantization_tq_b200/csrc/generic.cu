@@ -733,15 +733,22 @@ int attend_splits(int H, int64_t T) {
 
 bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kcodes, const void* kqjl,
                           const void* vcodes);
-int launch_attend_lut_split(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T,
                             int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                             float scale, float* part, void* stream);
 
+size_t attend_part_bytes(const DevState& ks, int H, int64_t T) {
+    const int sp = attend_splits(H, T);
+    return ((size_t)H * sp * (ks.d + 2) * sizeof(float) + 255) & ~(size_t)255;
+}
+
+// Split partials, then (d = 128, 2- to 4-bit key codes) the per-head query tables.
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T) {
     if (H <= 0 || T <= 0) return 0;
-    const int sp = attend_splits(H, T);
-    return (size_t)H * sp * (ks.d + 2) * sizeof(float);
+    size_t b = attend_part_bytes(ks, H, T);
+    if (ks.d == 128 && ks.b_mse >= 2 && ks.b_mse <= 4) b += (size_t)H * query_table_floats(ks) * sizeof(float);
+    return b;
 }
 
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
@@ -755,8 +762,11 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
     float* part = reinterpret_cast<float*>(ws);
     cudaError_t e;
     if (attend_lut_supported(ks, vs, kcodes, kqjl, vcodes)) {
-        e = (cudaError_t)launch_attend_lut_split(ks, vs, q, qdtype, H, T, nsplit, chunk, kcodes, kqjl, knorms,
-                                                 krnorms, vcodes, vnorms, scale, part, stream);
+        float* luts = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ws) + attend_part_bytes(ks, H, T));
+        e = (cudaError_t)launch_query_tables128(ks, q, qdtype, H, luts, stream);
+        if (e == cudaSuccess)
+            e = (cudaError_t)launch_attend_lut_split(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                                     vcodes, vnorms, scale, part, stream);
     } else {
         const size_t smem = attend_smem_bytes(ks.d);
         if (smem > 48 * 1024)

@@ -73,9 +73,15 @@ int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, 
                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
                  const float* rnorms, int64_t n, float* scores, void* stream);
 int read_device_error(int* flag);
+int take_device_error_gemm(int* flag);
+int take_device_error_search(int* flag);
 int launch_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,
                     void* stream);
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
+// Per-query lookup tables of the d = 128 scorers (rotated query against code groups, and
+// QJL nibbles): floats per query, and a launch building them for `count` query rows.
+size_t query_table_floats(const DevState& st);
+int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, void* stream);
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
                   int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
                   const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,

@@ -80,6 +80,169 @@ score_prep_kernel(const DevState st, const void* __restrict__ q, int qdtype, flo
     }
 }
 
+// d = 128: the same preparation with the d x d matrices staged whole in shared memory,
+// every load of a thread in flight at once, the RHT butterfly done by one warp with
+// shuffles, and the matrix-vector products split over all 256 threads.
+constexpr int kD128 = 128;
+
+__device__ __forceinline__ void stage_matrix128(const void* M, int dtype, unsigned char* dst) {
+    const uint4* src = reinterpret_cast<const uint4*>(M);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    if (dtype == TQ_F32) {
+        uint4 v[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) v[r] = __ldg(src + threadIdx.x + r * kThreads);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) d4[threadIdx.x + r * kThreads] = v[r];
+    } else {
+        uint4 v[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) v[r] = __ldg(src + threadIdx.x + r * kThreads);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) d4[threadIdx.x + r * kThreads] = v[r];
+    }
+}
+
+// out[j] = sum_k MT[k][j] in[k] (MT staged row-major 128 x 128); threads (j, half) each sum
+// 64 rows, `part` holds the halves.
+__device__ __forceinline__ void matvec128(const unsigned char* MT, int dtype, const float* in, float* part,
+                                          float* out) {
+    const int j = threadIdx.x & (kD128 - 1), h = threadIdx.x >> 7;
+    float a0 = 0.f, a1 = 0.f;
+    if (dtype == TQ_F32) {
+        const float* m = reinterpret_cast<const float*>(MT) + h * 64 * kD128 + j;
+#pragma unroll 16
+        for (int k = 0; k < 64; k += 2) {
+            a0 = fmaf(m[k * kD128], in[h * 64 + k], a0);
+            a1 = fmaf(m[(k + 1) * kD128], in[h * 64 + k + 1], a1);
+        }
+    } else {
+        const uint16_t* m = reinterpret_cast<const uint16_t*>(MT) + h * 64 * kD128 + j;
+#pragma unroll 16
+        for (int k = 0; k < 64; k += 2) {
+            a0 = fmaf(bf16_bits_to_float(m[k * kD128]), in[h * 64 + k], a0);
+            a1 = fmaf(bf16_bits_to_float(m[(k + 1) * kD128]), in[h * 64 + k + 1], a1);
+        }
+    }
+    part[h * kD128 + j] = a0 + a1;
+    __syncthreads();
+    if (threadIdx.x < kD128) out[threadIdx.x] = part[threadIdx.x] + part[kD128 + threadIdx.x];
+    __syncthreads();
+}
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(kThreads)
+tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts) {
+    using Gr = Groups<B>;
+    using LS = LutShape<kD128, B, PROD>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const size_t mbytes = (size_t)kD128 * kD128 * (st.mat_dtype == TQ_F32 ? 4 : 2);
+    unsigned char* m0 = smem_raw;              // Pi^T (dense rotation)
+    unsigned char* m1 = smem_raw + mbytes;     // S^T
+    float* ctab = reinterpret_cast<float*>(smem_raw + 2 * mbytes);
+    float* qs = ctab + kMaxLevels;
+    float* qp = qs + kD128;
+    float* u = qp + kD128;
+    float* part = u + kD128;                   // 2 x 128
+    const int64_t qi = blockIdx.x;
+    const bool dense = st.rot != TQ_ROT_RHT;
+    if (dense) stage_matrix128(st.piT, st.mat_dtype, m0);
+    if (PROD) stage_matrix128(st.sT, st.mat_dtype, m1);
+    for (int i = threadIdx.x; i < st.L; i += kThreads) ctab[i] = st.c[i];
+    if (threadIdx.x < kD128) {
+        const int i = threadIdx.x;
+        qs[i] = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + qi * kD128 + i)
+                                   : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + qi * kD128 + i));
+    }
+    __syncthreads();
+    if (dense) {
+        matvec128(m0, st.mat_dtype, qs, part, qp);
+    } else {
+        if (threadIdx.x < 32) {
+            // lane l holds elements 4l .. 4l+3; stages h = 1, 2 in registers, h >= 4 across lanes
+            const int l = threadIdx.x;
+            float v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = rht_neg(st, 4 * l + i) ? -qs[4 * l + i] : qs[4 * l + i];
+#pragma unroll
+            for (int h = 1; h < 4; h <<= 1) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if ((i & h) == 0) {
+                        const float a = v[i], b = v[i + h];
+                        v[i] = a + b;
+                        v[i + h] = a - b;
+                    }
+                }
+            }
+#pragma unroll
+            for (int hl = 1; hl < 32; hl <<= 1) {
+                const bool upper = (l & hl) != 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[i], hl);
+                    v[i] = upper ? o - v[i] : v[i] + o;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qp[4 * l + i] = v[i] * st.rsqrt_d;
+        }
+        __syncthreads();
+    }
+    if (PROD) matvec128(m1, st.mat_dtype, qp, part, u);
+    float* out = luts + qi * LS::SIZE;
+    for (int i = threadIdx.x; i < LS::MSE; i += kThreads) {
+        const int k = i / Gr::E, e = i % Gr::E;
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < Gr::CPG; ++c)
+            a = fmaf(qp[k * Gr::CPG + c], ctab[(e >> (B * c)) & ((1 << B) - 1)], a);
+        out[i] = a;
+    }
+    if constexpr (PROD) {
+        for (int i = threadIdx.x; i < LS::QJL; i += kThreads) {
+            const int k = i / 16, e = i % 16;
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = u[4 * k + c];
+                a += ((e >> c) & 1) ? v : -v;
+            }
+            out[LS::MSE + i] = a;
+        }
+    }
+}
+
+size_t tables128_smem(const DevState& st) {
+    const size_t mbytes = (size_t)kD128 * kD128 * (st.mat_dtype == TQ_F32 ? 4 : 2);
+    return 2 * mbytes + (size_t)(kMaxLevels + 5 * kD128) * sizeof(float);
+}
+
+// Tables of `count` queries (rows of q) into luts[count][SIZE].
+template <int D, int B, bool PROD>
+int launch_tables(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, cudaStream_t s) {
+    if (count <= 0) return 0;
+    if (count > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
+    if constexpr (D == kD128) {
+        auto k = tables128_kernel<B, PROD>;
+        const size_t smem = tables128_smem(st);
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return (int)e;
+        }
+        k<<<(unsigned)count, kThreads, smem, s>>>(st, q, qdtype, luts);
+    } else {
+        auto k = score_prep_kernel<D, B, PROD>;
+        const size_t smem = (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return (int)e;
+        }
+        k<<<(unsigned)count, kThreads, smem, s>>>(st, q, qdtype, luts);
+    }
+    return (int)cudaGetLastError();
+}
+
 template <int D, int B, bool PROD, int QT>
 __global__ void __launch_bounds__(kThreads)
 score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
@@ -164,10 +327,6 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
     }
 }
 
-template <int D, int B, bool PROD>
-size_t prep_smem() {
-    return (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
-}
 
 int sm_count_lut() {
     static int sms = 0;
@@ -191,11 +350,7 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
     float* luts = nullptr;
     cudaError_t ce = cudaMallocAsync(reinterpret_cast<void**>(&luts), (size_t)groups * nq * LS::SIZE * sizeof(float), s);
     if (ce != cudaSuccess) return (int)ce;
-    auto prep = score_prep_kernel<D, B, PROD>;
-    const size_t psmem = prep_smem<D, B, PROD>();
-    if (psmem > 48 * 1024) cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-    prep<<<(unsigned)(groups * nq), kThreads, psmem, s>>>(st, q, qdtype, luts);
-    ce = cudaGetLastError();
+    ce = (cudaError_t)launch_tables<D, B, PROD>(st, q, qdtype, groups * nq, luts, s);
     if (ce == cudaSuccess) {
         auto kern = score_lut_kernel<D, B, PROD, QT>;
         const size_t smem = (size_t)QT * LS::SIZE * sizeof(float);
@@ -247,7 +402,36 @@ int launch_lut_b(const DevState& st, const void* q, int qdtype, int64_t groups, 
     }
 }
 
+template <bool PROD>
+int launch_tables128_b(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, cudaStream_t s) {
+    switch (st.b_mse) {
+        case 1: return launch_tables<128, 1, PROD>(st, q, qdtype, count, luts, s);
+        case 2: return launch_tables<128, 2, PROD>(st, q, qdtype, count, luts, s);
+        case 3: return launch_tables<128, 3, PROD>(st, q, qdtype, count, luts, s);
+        case 4: return launch_tables<128, 4, PROD>(st, q, qdtype, count, luts, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
+
+size_t query_table_floats(const DevState& st) {
+    const bool prod = st.mode == TQ_PROD;
+    switch (st.b_mse) {
+        case 1: return prod ? LutShape<128, 1, true>::SIZE : LutShape<128, 1, false>::SIZE;
+        case 2: return prod ? LutShape<128, 2, true>::SIZE : LutShape<128, 2, false>::SIZE;
+        case 3: return prod ? LutShape<128, 3, true>::SIZE : LutShape<128, 3, false>::SIZE;
+        case 4: return prod ? LutShape<128, 4, true>::SIZE : LutShape<128, 4, false>::SIZE;
+        default: return 0;
+    }
+}
+
+int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, void* stream) {
+    if (st.d != 128) return (int)cudaErrorInvalidValue;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (st.mode == TQ_PROD) return launch_tables128_b<true>(st, q, qdtype, count, luts, s);
+    return launch_tables128_b<false>(st, q, qdtype, count, luts, s);
+}
 
 bool score_lut_supported(const DevState& st) {
     return (st.d == 128 || st.d == 256) && st.b_mse >= 1 && st.b_mse <= 4;

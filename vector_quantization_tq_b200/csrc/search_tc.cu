@@ -23,7 +23,9 @@
 
 namespace tq {
 
-extern __device__ int g_tq_device_error;
+namespace {
+__device__ int g_tq_device_error = 0;
+}  // namespace
 
 namespace {
 
@@ -458,6 +460,19 @@ int launch_search_tc(const DevState& st, const void* q, int qdtype, int64_t nq, 
     search_tc_kernel<<<grid, kThreads, smem, s>>>(tm, p);
     if ((e = (int)cudaGetLastError())) return e;
     return launch_search_merge(nq, (int64_t)cy * k, k, cand_v, cand_i, idx, vals, stream);
+}
+
+int take_device_error_search(int* flag) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tq_device_error, sizeof(int));
+    if (e != cudaSuccess) return (int)e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_tq_device_error, &zero, sizeof(int));
+        if (e != cudaSuccess) return (int)e;
+    }
+    *flag = v;
+    return 0;
 }
 
 }  // namespace tq
