@@ -138,25 +138,30 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                 const uint4 v = src[i];
                 w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
             }
-            float a1 = 0.f;
+            float a1[1] = {0.f};
+            if constexpr (KG::G == 4) {
 #pragma unroll
-            for (int k = 0; k < KG::NG; ++k) {
-                const int bit = k * KG::G;
-                const int wi = bit >> 5, sh = bit & 31;
-                uint32_t e;
-                if (sh + KG::G <= 32) e = (w[wi] >> sh) & (KG::E - 1);
-                else e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (KG::E - 1);
-                a1 += tm[k * KG::E + e];
+                for (int wi = 0; wi < CW; ++wi) add_nibbles<1, 0>(w[wi], tm + 8 * wi * 16, a1);
+            } else {
+#pragma unroll
+                for (int k = 0; k < KG::NG; ++k) {
+                    const int bit = k * KG::G;
+                    const int wi = bit >> 5, sh = bit & 31;
+                    uint32_t e;
+                    if (sh + KG::G <= 32) e = (w[wi] >> sh) & (KG::E - 1);
+                    else e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (KG::E - 1);
+                    a1[0] += tm[k * KG::E + e];
+                }
             }
-            float a2 = 0.f, g2 = 0.f;
+            float a2[1] = {0.f}, g2 = 0.f;
             if constexpr (KPROD) {
                 const uint4 zv = *reinterpret_cast<const uint4*>(B.kz + threadIdx.x * 16);
                 const uint32_t z[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-                for (int k = 0; k < NQ; ++k) a2 += tz[k * 16 + ((z[k >> 3] >> ((k & 7) * 4)) & 15u)];
+                for (int wi = 0; wi < 4; ++wi) add_nibbles<1, 0>(z[wi], tz + 8 * wi * 16, a2);
                 g2 = B.kr[threadIdx.x] * ks.qjl_scale;
             }
-            s = scale * B.kn[threadIdx.x] * fmaf(g2, a2, a1);
+            s = scale * B.kn[threadIdx.x] * fmaf(g2, a2[0], a1[0]);
         }
         // ---- B: online softmax bookkeeping ----
         const float wm = warp_max(s);
@@ -213,9 +218,27 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                 wv[j] = w;
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 8; ++j) {
+                const char* cbase = reinterpret_cast<const char*>(vc);
+                if constexpr (BV == 4) {
+                    // byte offsets 4 e of the four nibbles: 0 and 2 from `lo`, 1 and 3 from `hi`
+                    const uint32_t lo = (bits[j] << 2) & 0x3C3Cu, hi = (bits[j] >> 2) & 0x3C3Cu;
+                    acc[0] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (lo & 0xFFu)), acc[0]);
+                    acc[1] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (hi & 0xFFu)), acc[1]);
+                    acc[2] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (lo >> 8)), acc[2]);
+                    acc[3] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (hi >> 8)), acc[3]);
+                } else if constexpr (BV == 2) {
+                    const uint32_t b8 = bits[j];
+                    acc[0] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 << 2) & 0xCu)), acc[0]);
+                    acc[1] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (b8 & 0xCu)), acc[1]);
+                    acc[2] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 >> 2) & 0xCu)), acc[2]);
+                    acc[3] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 >> 4) & 0xCu)), acc[3]);
+                } else {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[c] = fmaf(wv[j], vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
+                    for (int c = 0; c < 4; ++c)
+                        acc[c] = fmaf(wv[j], vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
+                }
+            }
         }
         __syncthreads();   // wt / red and the tile buffer are reused
     }

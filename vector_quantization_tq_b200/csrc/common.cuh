@@ -132,4 +132,26 @@ __device__ __forceinline__ uint32_t extract_code(const uint32_t* __restrict__ ro
     return (uint32_t)(win >> sh) & ((1u << b) - 1u);
 }
 
+
+// Table lookups over the 8 nibbles of a packed word: acc[qi] += sum_m T_m[e_m], e_m the
+// m-th nibble of w and T_m the 16-entry float table at t0 + 16 m (query qi's tables
+// `stride` floats further on). Two masks put the nibbles, times 4, into bytes; a lookup is
+// then one byte permute and one shared-memory load.
+template <int QT, int STRIDE>
+__device__ __forceinline__ void add_nibbles(uint32_t w, const float* t0, float (&acc)[QT]) {
+    const uint32_t lo4 = (w << 2) & 0x3C3C3C3Cu;   // nibbles 0, 2, 4, 6
+    const uint32_t hi4 = (w >> 2) & 0x3C3C3C3Cu;   // nibbles 1, 3, 5, 7
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const uint32_t o0 = __byte_perm(lo4, 0u, 0x4440u | m);
+        const uint32_t o1 = __byte_perm(hi4, 0u, 0x4440u | m);
+#pragma unroll
+        for (int qi = 0; qi < QT; ++qi) {
+            const char* t = reinterpret_cast<const char*>(t0 + qi * STRIDE + 2 * m * 16);
+            acc[qi] += *reinterpret_cast<const float*>(t + o0);
+            acc[qi] += *reinterpret_cast<const float*>(t + 64 + o1);
+        }
+    }
+}
+
 }  // namespace tq

@@ -894,16 +894,21 @@ encode_tc3_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 // the sign of S r read from the fp32 accumulator.
 // ------------------------------------------------------------------------------------
 constexpr int kT4Stages = 3;
-constexpr int kT4Warps = 16;
-constexpr int kT4Threads = (kT4Warps + 1) * 32;
 constexpr uint32_t kT4Cols = 512;
+constexpr int kT4P = 2;   // threads per vector (each takes 128 / kT4P coordinates)
+template <int P>
+struct T4 {
+    static constexpr int kWarps = 4 * P;                // quantizing warps
+    static constexpr int kThreads = (kWarps + 1) * 32;  // + the TMA / MMA warp
+    static constexpr int kC = kD / P;                   // coordinates per thread
+};
 
 struct __align__(1024) TcSmem4 {
     uint8_t x[kT4Stages][2][kTile * 128];   // [stage][half]: 128 rows x 128 bytes, 128B-swizzled
     uint8_t hd[kD * kD * 2];                // H diag(eps), B operand (K-major core matrices)
     uint8_t s[kD * kD * 2];                 // S, B operand
     float ssq[2][4][kTile];                 // [tile parity][part]: partial ||H D x||^2
-    float rsq[2][4][kTile];                 // [tile parity][part]: partial ||r||^2
+    float rsq[2][4][kTile];                 // [tile parity][part]: partial ||r||^2 (up to 4 parts)
     uint64_t bar_x[kT4Stages];              // tile landed
     uint64_t bar_xfree[kT4Stages];          // the rotation MMA has read the stage
     uint64_t bar_h;                         // y of the current tile is in TMEM
@@ -914,10 +919,12 @@ struct __align__(1024) TcSmem4 {
     int abort;
 };
 
-template <int B, bool PROD>
-__global__ void __launch_bounds__(kT4Threads, 1)
+template <int B, bool PROD, int P>
+__global__ void __launch_bounds__(T4<P>::kThreads, 1)
 encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     static_assert(B == 1 || B == 2, "the pipelined encoder covers 1- and 2-bit codes");
+    static_assert(P == 2 || P == 4, "two or four threads per vector");
+    constexpr int kWarps = T4<P>::kWarps, kThreads = T4<P>::kThreads, C = T4<P>::kC, NCH = C / 32;
     extern __shared__ uint8_t smem_raw[];
     TcSmem4& sm = *reinterpret_cast<TcSmem4*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int* abort_flag = &sm.abort;
@@ -933,9 +940,9 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             ptx::mbar_init(&sm.bar_xfree[i], 1);
         }
         ptx::mbar_init(&sm.bar_h, 1);
-        ptx::mbar_init(&sm.bar_yfree, kT4Warps);
-        ptx::mbar_init(&sm.bar_hl[0], kT4Warps);
-        ptx::mbar_init(&sm.bar_hl[1], kT4Warps);
+        ptx::mbar_init(&sm.bar_yfree, kWarps);
+        ptx::mbar_init(&sm.bar_hl[0], kWarps);
+        ptx::mbar_init(&sm.bar_hl[1], kWarps);
         ptx::mbar_init(&sm.bar_s, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -945,14 +952,14 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         ptx::tmem_relinquish();
     }
     // H diag(eps): entry (n, k) = (-1)^popcount(n & k) * eps_k, at chunk k/8 of row n.
-    for (int i = tid; i < kD * kD; i += kT4Threads) {
+    for (int i = tid; i < kD * kD; i += kThreads) {
         const int n = i >> 7, k = i & 127;
         const uint32_t neg = (__popc(n & k) & 1) ^ ((p.sgn[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u);
         *reinterpret_cast<uint16_t*>(sm.hd + (k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) =
             neg ? 0xBF80u : 0x3F80u;
     }
     if constexpr (PROD) {
-        for (int i = tid; i < kD * 16; i += kT4Threads) {
+        for (int i = tid; i < kD * 16; i += kThreads) {
             const int row = i >> 4, c = i & 15;
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.s + row * kD + c * 8));
             *reinterpret_cast<uint4*>(sm.s + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
@@ -964,7 +971,7 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == kT4Warps) {
+    if (warp == kWarps) {
         // ---------------- producer: TMA + MMA issue (one thread) ----------------
         if (lane == 0) {
             const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
@@ -1047,32 +1054,41 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
     } else {
         // ---------------- quantizing warps ----------------
+        // warp w: lane quadrant w % 4 (vectors 32 (w % 4) ..), part w / 4 (coordinates
+        // C part .. C part + C - 1 of each of those vectors)
         const int quad = warp & 3, part = warp >> 2;
         const int vrow = quad * 32 + lane;
-        const int bar_id = 1 + quad;   // named barrier of the four warps sharing these vectors
+        const int bar_id = 1 + quad;   // named barrier of the P warps sharing these vectors
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const float rsqrt_d = p.rsqrt_d;
         const float t2 = p.t[2];
         int64_t prev_row = -1;
         bool prev_nz = false;
         bool fail = false;
-        // Signs of S r (in D) for vector `srow`; [(S r)_j >= 0], all ones for a zero vector.
+        // Signs of S r (in D) for vector `srow`: [(S r)_j >= 0], all ones for a zero vector.
         auto emit_signs = [&](uint32_t parity, int64_t srow, bool snz) -> bool {
             bool sok = true;
             if (lane == 0) sok = ptx::mbar_wait(&sm.bar_s, parity);
             sok = __shfl_sync(0xffffffffu, sok ? 1 : 0, 0) != 0;
             ptx::tc_fence_after();
-            uint32_t d[32];
-            ptx::tmem_ld32(t_lane + 128 + part * 32, d);
-            ptx::tmem_wait_ld();
-            uint32_t z0 = 0u, z1 = 0u;
+            uint32_t zw[NCH];
 #pragma unroll
-            for (int j = 15; j >= 0; --j) {
-                z0 = __funnelshift_l(d[j], z0, 1);
-                z1 = __funnelshift_l(d[j + 16], z1, 1);
+            for (int ch = 0; ch < NCH; ++ch) {
+                uint32_t d[32];
+                ptx::tmem_ld32(t_lane + 128 + part * C + ch * 32, d);
+                ptx::tmem_wait_ld();
+                uint32_t z0 = 0u, z1 = 0u;
+#pragma unroll
+                for (int j = 15; j >= 0; --j) {
+                    z0 = __funnelshift_l(d[j], z0, 1);
+                    z1 = __funnelshift_l(d[j + 16], z1, 1);
+                }
+                zw[ch] = snz ? ~(z0 | (z1 << 16)) : 0xffffffffu;
             }
-            if (sok && srow < p.n)
-                *reinterpret_cast<uint32_t*>(p.qjl + srow * 16 + part * 4) = snz ? ~(z0 | (z1 << 16)) : 0xffffffffu;
+            if (sok && srow < p.n) {
+                uint8_t* dst = p.qjl + srow * 16 + part * (C / 8);
+                if constexpr (NCH == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(zw[0], zw[1]);
+                else *reinterpret_cast<uint32_t*>(dst) = zw[0];
+            }
             return sok;
         };
         for (int64_t k = 0; k < mytiles; ++k) {
@@ -1082,75 +1098,97 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             if (lane == 0) ok = ptx::mbar_wait(&sm.bar_h, (uint32_t)(k & 1));
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             ptx::tc_fence_after();
-            uint32_t a[32];
-            ptx::tmem_ld32(t_lane + part * 32, a);
+            uint32_t a[C];
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch) {
+                uint32_t (&ac)[32] = *reinterpret_cast<uint32_t(*)[32]>(a + ch * 32);
+                ptx::tmem_ld32(t_lane + part * C + ch * 32, ac);
+            }
             ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&sm.bar_yfree);
             float2 q0 = f2(0.f, 0.f), q1 = f2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < C / 4; ++i) {
                 const float2 u0 = f2(__uint_as_float(a[4 * i]), __uint_as_float(a[4 * i + 1]));
                 const float2 u1 = f2(__uint_as_float(a[4 * i + 2]), __uint_as_float(a[4 * i + 3]));
                 q0 = __ffma2_rn(u0, u0, q0);
                 q1 = __ffma2_rn(u1, u1, q1);
             }
             sm.ssq[kb][part][vrow] = (q0.x + q0.y) + (q1.x + q1.y);
-            if (ptx::bar_sync_or(bar_id, 128, !ok || *abort_flag)) {
+            if (ptx::bar_sync_or(bar_id, 32 * P, !ok || *abort_flag)) {
                 fail = true;
                 break;
             }
-            // ||H D x||^2 = d ||x||^2
-            const float nu =
-                sqrtf((sm.ssq[kb][0][vrow] + sm.ssq[kb][1][vrow]) + (sm.ssq[kb][2][vrow] + sm.ssq[kb][3][vrow])) *
-                rsqrt_d;
-            const bool nz = nu > 0.f;
-            const float sc = nz ? rsqrt_d / nu : 0.f;
+            // ||H D x||^2 = d ||x||^2; the normalised rotated coordinate is y / ||H D x||
+            float ssq = sm.ssq[kb][0][vrow] + sm.ssq[kb][1][vrow];
+            if constexpr (P == 4) ssq += sm.ssq[kb][2][vrow] + sm.ssq[kb][3][vrow];
+            const bool nz = ssq > 0.f;
+            const float sc = nz ? rsqrtf(ssq) : 0.f;
             const float cs = nz ? p.c[B == 2 ? 2 : 1] : 0.f;   // inner level (b = 2) / the level (b = 1)
             const float cb = nz ? p.c[B == 2 ? 3 : 1] : 0.f;   // outer level
             const float dcb = cs - cb;
-            uint32_t np0 = 0u, np1 = 0u, mp0 = 0u, mp1 = 0u;
-            float r[32];
+            // Code bits in chains of 16 coordinates: np (y < 0), mp (inner level). Coordinates
+            // go in pairs through f32x2 arithmetic: ys = y sc; inner iff ys^2 < t2^2; the residual
+            // is r = ys - sign(y) c, c the inner or outer level.
+            uint32_t np[C / 16], mp[C / 16];
 #pragma unroll
-            for (int j = 15; j >= 0; --j) {
+            for (int g = 0; g < C / 16; ++g) np[g] = mp[g] = 0u;
+            float2 r2[C / 2];
+            const float2 sc2 = f2(sc, sc);
+            const float2 nt2 = f2(-t2 * t2, -t2 * t2);
+            const float2 dcb2 = f2(dcb, dcb), cb2 = f2(cb, cb);
 #pragma unroll
-                for (int hh = 1; hh >= 0; --hh) {
-                    const int jj = j + 16 * hh;
-                    const uint32_t yb = a[jj];
-                    const float ay = fabsf(__uint_as_float(yb));
-                    uint32_t& np = hh ? np1 : np0;
-                    np = __funnelshift_l(yb, np, 1);   // bit jj: y < 0
-                    float mag = cs;
+            for (int i = 7; i >= 0; --i) {
+#pragma unroll
+                for (int g = C / 16 - 1; g >= 0; --g) {
+                    const int pi = 8 * g + i;   // coordinates 2 pi, 2 pi + 1
+                    const uint32_t yb0 = a[2 * pi], yb1 = a[2 * pi + 1];
+                    const float2 ys = __fmul2_rn(f2(__uint_as_float(yb0), __uint_as_float(yb1)), sc2);
+                    np[g] = __funnelshift_l(yb1, np[g], 1);   // bit: y < 0
+                    np[g] = __funnelshift_l(yb0, np[g], 1);
+                    float2 mag = cb2;
                     if constexpr (B == 2) {
-                        uint32_t& mp = hh ? mp1 : mp0;
-                        const float dd = fmaf(-ay, sc, t2);                 // > 0: inner level
-                        const float st = __saturatef(dd * 0x1p126f);        // exactly 1 (inner) or 0
-                        mp = __funnelshift_l(__float_as_uint(0.5f - st), mp, 1);   // bit jj: inner
-                        mag = fmaf(st, dcb, cb);
+                        const float2 dd = __ffma2_rn(ys, ys, nt2);   // < 0: inner level
+                        mp[g] = __funnelshift_l(__float_as_uint(dd.y), mp[g], 1);
+                        mp[g] = __funnelshift_l(__float_as_uint(dd.x), mp[g], 1);
+                        // exactly 1 (inner) or 0: a nonzero dd is far above the subnormal range
+                        const float2 st = f2(__saturatef(dd.x * -0x1p126f), __saturatef(dd.y * -0x1p126f));
+                        mag = __ffma2_rn(st, dcb2, cb2);
                     }
-                    const float ar = fmaf(ay, sc, -mag);
-                    r[jj] = __uint_as_float(__float_as_uint(ar) ^ (yb & 0x80000000u));
+                    // -sign(y) c
+                    const float2 nsm = f2(__uint_as_float(__float_as_uint(mag.x) | (~yb0 & 0x80000000u)),
+                                          __uint_as_float(__float_as_uint(mag.y) | (~yb1 & 0x80000000u)));
+                    r2[pi] = __fadd2_rn(ys, nsm);
                 }
             }
-            const uint32_t np = np0 | (np1 << 16);
             if (row < p.n) {
-                if constexpr (B == 2) {
-                    const uint32_t mp = mp0 | (mp1 << 16);
-                    const uint32_t hb = ~np, lb = ~(np ^ mp);
-                    *reinterpret_cast<uint2*>(p.codes + row * 32 + part * 8) =
-                        make_uint2(spread16(lb) | (spread16(hb) << 1), spread16(lb >> 16) | (spread16(hb >> 16) << 1));
-                } else {
-                    *reinterpret_cast<uint32_t*>(p.codes + row * 16 + part * 4) = ~np;
+                uint32_t cw[B * C / 32];
+#pragma unroll
+                for (int h2 = 0; h2 < C / 32; ++h2) {
+                    const uint32_t n32 = np[2 * h2] | (np[2 * h2 + 1] << 16);
+                    if constexpr (B == 2) {
+                        const uint32_t m32 = mp[2 * h2] | (mp[2 * h2 + 1] << 16);
+                        const uint32_t hb = ~n32, lb = ~(n32 ^ m32);
+                        cw[2 * h2] = spread16(lb) | (spread16(hb) << 1);
+                        cw[2 * h2 + 1] = spread16(lb >> 16) | (spread16(hb >> 16) << 1);
+                    } else {
+                        cw[h2] = ~n32;
+                    }
                 }
-                if (part == 0) p.norms[row] = nu;
+                uint8_t* dst = p.codes + row * (B * 16) + part * (B * C / 8);
+                if constexpr (B * C / 32 == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                else if constexpr (B * C / 32 == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(cw[0], cw[1]);
+                else *reinterpret_cast<uint32_t*>(dst) = cw[0];
+                if (part == 0) p.norms[row] = sqrtf(ssq) * p.rsqrt_d;
             }
             if constexpr (PROD) {
                 float2 e0 = f2(0.f, 0.f), e1 = f2(0.f, 0.f);
-                uint32_t hi[16], lo[16];
+                uint32_t hi[C / 2], lo[C / 2];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 rp = f2(r[2 * i], r[2 * i + 1]);
+                for (int i = 0; i < C / 2; ++i) {
+                    const float2 rp = r2[i];
                     if (i & 1) e1 = __ffma2_rn(rp, rp, e1);
                     else e0 = __ffma2_rn(rp, rp, e0);
                     const __nv_bfloat162 h = __float22bfloat162_rn(rp);
@@ -1163,21 +1201,28 @@ encode_tc4_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                 }
                 sm.rsq[kb][part][vrow] = (e0.x + e0.y) + (e1.x + e1.y);
                 const uint32_t hl = t_lane + 256u + (uint32_t)kb * 128u;
-                ptx::tmem_st16(hl + part * 16, hi);
-                ptx::tmem_st16(hl + 64 + part * 16, lo);
+                if constexpr (C / 2 == 32) {
+                    ptx::tmem_st32(hl + part * 32, hi);
+                    ptx::tmem_st32(hl + 64 + part * 32, lo);
+                } else {
+                    ptx::tmem_st16(hl + part * 16, *reinterpret_cast<uint32_t(*)[16]>(hi));
+                    ptx::tmem_st16(hl + 64 + part * 16, *reinterpret_cast<uint32_t(*)[16]>(lo));
+                }
                 ptx::tmem_wait_st();
                 bool sok = true;
                 if (k > 0) sok = emit_signs((uint32_t)((k - 1) & 1), prev_row, prev_nz);   // previous tile
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&sm.bar_hl[kb]);
-                if (ptx::bar_sync_or(bar_id, 128, !sok || *abort_flag)) {
+                if (ptx::bar_sync_or(bar_id, 32 * P, !sok || *abort_flag)) {
                     fail = true;
                     break;
                 }
-                if (part == 0 && row < p.n)
-                    p.rnorms[row] = sqrtf((sm.rsq[kb][0][vrow] + sm.rsq[kb][1][vrow]) +
-                                          (sm.rsq[kb][2][vrow] + sm.rsq[kb][3][vrow]));
+                if (part == 0 && row < p.n) {
+                    float rs = sm.rsq[kb][0][vrow] + sm.rsq[kb][1][vrow];
+                    if constexpr (P == 4) rs += sm.rsq[kb][2][vrow] + sm.rsq[kb][3][vrow];
+                    p.rnorms[row] = sqrtf(rs);
+                }
                 prev_row = row;
                 prev_nz = nz;
             }
@@ -1258,7 +1303,7 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
     }
     constexpr bool kTwo = (B == 1 || B == 2);
     const size_t smem = (kTwo ? sizeof(TcSmem4) : sizeof(TcSmem)) + 1024;
-    auto kern = kTwo ? encode_tc4_kernel<(B <= 2 ? B : 2), PROD> : encode_tc_kernel<B, PROD>;
+    auto kern = kTwo ? encode_tc4_kernel<(B <= 2 ? B : 2), PROD, kT4P> : encode_tc_kernel<B, PROD>;
     static int attr_set_for_device = -1;   // per instantiation
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1269,7 +1314,7 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
     }
     const int64_t ntiles = (n + kTile - 1) / kTile;
     const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * (kTwo ? 1 : 2));
-    kern<<<grid, kTwo ? kT4Threads : kTile, smem, stream>>>(tmap, p);
+    kern<<<grid, kTwo ? T4<kT4P>::kThreads : kTile, smem, stream>>>(tmap, p);
     return (int)cudaGetLastError();
 }
 

@@ -294,32 +294,31 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
             g2 = __ldg(rnorms + gk) * st.qjl_scale;
         }
         const float nu = __ldg(norms + gk);
-        float a1[QT];
+        float a1[QT], a2[QT];
 #pragma unroll
-        for (int qi = 0; qi < QT; ++qi) a1[qi] = 0.f;
+        for (int qi = 0; qi < QT; ++qi) a1[qi] = a2[qi] = 0.f;
+        if constexpr (Gr::G == 4) {
+            // 16-entry tables: the 8 nibbles of a word, pre-scaled to byte offsets 4 e
 #pragma unroll
-        for (int k = 0; k < NG; ++k) {
-            const int bit = k * Gr::G;
-            const int wi = bit >> 5, sh = bit & 31;
-            uint32_t e;
-            if (sh + Gr::G <= 32) {
-                e = (w[wi] >> sh) & (Gr::E - 1);
-            } else {
-                e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (Gr::E - 1);
+            for (int wi = 0; wi < CW; ++wi) add_nibbles<QT, LS::SIZE>(w[wi], tab + 8 * wi * 16, a1);
+        } else {
+#pragma unroll
+            for (int k = 0; k < NG; ++k) {
+                const int bit = k * Gr::G;
+                const int wi = bit >> 5, sh = bit & 31;
+                uint32_t e;
+                if (sh + Gr::G <= 32) {
+                    e = (w[wi] >> sh) & (Gr::E - 1);
+                } else {
+                    e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (Gr::E - 1);
+                }
+#pragma unroll
+                for (int qi = 0; qi < QT; ++qi) a1[qi] += tab[qi * LS::SIZE + k * Gr::E + e];
             }
-#pragma unroll
-            for (int qi = 0; qi < QT; ++qi) a1[qi] += tab[qi * LS::SIZE + k * Gr::E + e];
         }
-        float a2[QT];
-#pragma unroll
-        for (int qi = 0; qi < QT; ++qi) a2[qi] = 0.f;
         if constexpr (PROD) {
 #pragma unroll
-            for (int k = 0; k < NQ; ++k) {
-                const uint32_t e = (z[k >> 3] >> ((k & 7) * 4)) & 15u;
-#pragma unroll
-                for (int qi = 0; qi < QT; ++qi) a2[qi] += tab[qi * LS::SIZE + LS::MSE + k * 16 + e];
-            }
+            for (int wi = 0; wi < NQ / 8; ++wi) add_nibbles<QT, LS::SIZE>(z[wi], tab + LS::MSE + 8 * wi * 16, a2);
         }
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi)
