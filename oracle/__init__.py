@@ -14,9 +14,11 @@ What it computes (each function cites the passage it follows):
   quantizer  TurboQuant_mse and TurboQuant_prod encode / decode, bit packing,
              inner-product estimate <q, x~>
   attention  decode attention over reconstructed K and V, top-k by estimate
+  mixed      outlier-channel split: two channel groups, each its own quantizer at its
+             own bit width; merge, effective width, outlier-channel choice
 
 Every function is pinned by a `-m "not gpu"` test against values the pages print,
 closed forms, textbook special cases or brute force (tests/test_oracle_*.py).
 No function is "parity unpinned".
 """
-from . import attention, codebook, quantizer, rotation  # noqa: F401
+from . import attention, codebook, mixed, quantizer, rotation  # noqa: F401
