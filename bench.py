@@ -79,23 +79,21 @@ def tensor_peak():
 
 def stored_traffic(kernel_key: str):
     """Per-launch DRAM bytes from the committed ncu summary, if it matches the current source."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
     try:
-        with open(p) as f:
-            t = json.load(f)
-        ent = t.get(kernel_key)
-        if not ent:
-            return None
         import hashlib
-        src = os.path.join(ROOT, ent["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h != ent["source_sha"]:
-            return None
-        return float(ent["dram_bytes_per_launch"])
+        for line in open(p):
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) == 5 and cells[0] == kernel_key:
+                src = os.path.join(ROOT, cells[2])
+                if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != cells[3]:
+                    return None
+                return float(cells[4])
     except Exception:
         return None
+    return None
 
 
 class ClockSampler:
@@ -199,6 +197,58 @@ def measure_decode(tq, torch, dev, stream, steps: int, warmup: int, peak: float)
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "algorithmic_bytes_per_launch": DEC_BYTES_PER_TOKEN * n},
             "gpu_launches_per_step": 2}
+
+
+# Outlier-channel split of the same KV key batch: the 32 channels of largest mean square
+# (over the first 32,768 keys) at prod b=3, the other 96 at prod b=2 (dense Pi, fp32 state).
+# Per vector: 256 B in; out 8 + 4 + 8 B (outer codes, QJL, norms) + 12 + 12 + 8 B (inner).
+SPLIT_M, SPLIT_BO, SPLIT_BR = 32, 3, 2
+SPLIT_BYTES_PER_VEC = 2 * D + (SPLIT_M * (SPLIT_BO - 1) // 8 + SPLIT_M // 8 + 8) + \
+    ((D - SPLIT_M) * (SPLIT_BR - 1) // 8 + (D - SPLIT_M) // 8 + 8)
+
+
+def measure_split(tq, torch, x, q, heads, dev, stream, steps: int, warmup: int, peak: float):
+    """Time tq_split_quantize and tq_split_score on the prefill batch (x, q already on the device)."""
+    nvec = x.shape[0]
+    ms = torch.mean(x[:TOKENS].float() ** 2, dim=0)
+    ch = np.sort(torch.argsort(ms, descending=True)[:SPLIT_M].cpu().numpy())
+    so = tq.State(SPLIT_M, SPLIT_BO, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, seed_pi=20, seed_s=21)
+    sr = tq.State(D - SPLIT_M, SPLIT_BR, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, seed_pi=22, seed_s=23)
+    sp = tq.Split(so, sr, ch)
+    po, pr = sp.empty_planes(nvec, dev)
+    scores = torch.empty((heads, 1, TOKENS), dtype=torch.float32, device=dev)
+
+    def enc():
+        tq.split_quantize(sp, x, po, pr, stream=stream)
+
+    def sc():
+        tq.split_score(sp, q, po, pr, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+
+    out = {}
+    for name, fn in (("encode", enc), ("score", sc)):
+        for _ in range(max(3, warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        out[name] = e0.elapsed_time(e1) / steps
+    gbs = SPLIT_BYTES_PER_VEC * nvec / (out["encode"] / 1e3) / 1e9
+    res = {"workload": f"outlier-channel split of the KV key batch: {SPLIT_M} channels at prod b={SPLIT_BO}, "
+                       f"{D - SPLIT_M} at prod b={SPLIT_BR} (dense Pi, fp32 state), "
+                       f"{SPLIT_M * SPLIT_BO + (D - SPLIT_M) * SPLIT_BR} bits per vector of codes",
+           "effective_bits": (SPLIT_M * SPLIT_BO + (D - SPLIT_M) * SPLIT_BR) / D,
+           "ms": out, "quantize_mvec_s": nvec / (out["encode"] / 1e3) / 1e6,
+           "score_gkeys_s": nvec / (out["score"] / 1e3) / 1e9,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                        "algorithmic_bytes_per_launch": SPLIT_BYTES_PER_VEC * nvec}}
+    sp.close()
+    so.close()
+    sr.close()
+    return res
 
 
 # Embedding search (1,000,000 vectors, d = 1536, prod b = 2, dense Pi and S bf16, 1000 queries):
@@ -319,6 +369,7 @@ def main():
     ap.add_argument("--heads", type=int, default=HEADS, help="smaller batch for profiling runs")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
     ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
+    ap.add_argument("--no-split", action="store_true", help="skip the outlier-channel split measurement")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -441,6 +492,9 @@ def main():
     decode = None
     if not args.no_decode:
         decode = measure_decode(tq, torch, dev, stream, args.steps, args.warmup, peak)
+    split = None
+    if not args.no_split:
+        split = measure_split(tq, torch, x, q, heads, dev, stream, args.steps, args.warmup, peak)
     c5 = None
     if not args.no_c5:
         c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak())
@@ -471,11 +525,12 @@ def main():
                      "traffic": traffic, "kernel": "encode (tq_quantize_prod)",
                      "algorithmic_bytes_per_launch": ENC_BYTES_PER_VEC * nvec, "peak_kind": peak_kind},
         "score_roofline": {"bound": "hbm", "achieved": sc_gbs, "peak": peak, "unit": "GB/s", "frac": sc_gbs / peak},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,   # encoder; query tables + scorer
         "clocks": clk.summary(),
         "e2e": e2e,
         "decode_attention": decode,
         "embedding_search": c5,
+        "outlier_split": split,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -265,6 +265,97 @@ int tq_search_topk(const tq_state* st, const void* q, int qdtype, int64_t nq,
                    const float* rnorms, int64_t n, int k, int64_t* idx, float* vals,
                    void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Decode step with grouped queries: H query heads, G of them per KV head (H % G == 0;
+ * query head h reads KV head h / G). The planes of KV head g are rows g*Tcap .. g*Tcap+T-1
+ * (Tcap >= T: a cache with room to grow); q [H][d], out fp32 [H][d]. Workspace as
+ * tq_attend_workspace(ks, vs, H, T). G = 1 and Tcap = T is tq_attend_decode.
+ */
+int tq_attend_decode_grouped(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int G,
+                             int64_t T, int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl,
+                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                             float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Streaming decode step (the "online" setting: one new token per step): encode the new key
+ * and value of every KV head (k_new, v_new: [H/G][d], dtype kvdtype, contiguous) into row T
+ * of that head's planes (0 <= T < Tcap), then run tq_attend_decode_grouped over the T + 1
+ * tokens. Both launches go on `stream` in that order. Workspace as
+ * tq_attend_workspace(ks, vs, H, T + 1).
+ */
+int tq_attend_append_decode(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int G,
+                            const void* k_new, const void* v_new, int kvdtype, int64_t T, int64_t Tcap,
+                            uint8_t* kcodes, uint8_t* kqjl, float* knorms, float* krnorms, uint8_t* vcodes,
+                            float* vnorms, float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- outlier-channel split ------------------------------------------------------------
+ * TurboQuant review (Jump2Paper), experiment settings ("KV bit settings": 2.5 and 3.5 bits
+ * with outlier and non-outlier channels separated; "outlier handling": 32 of 128 channels at
+ * 3 bits, 96 at 2 bits). A split quantizes the m channels listed in `channels` with the
+ * state `outer` (dimension m) and the other d - m channels, in ascending order, with `inner`
+ * (dimension d - m): two independent quantizers, each with its own rotation, codebook, QJL
+ * matrix and norms. The reconstruction puts each group back into its channels, so an
+ * estimate <q, x~> is the sum of the two groups' estimates.
+ */
+typedef struct tq_split tq_split;
+
+/* Device planes of one channel group (qjl and rnorms NULL for an MSE state). */
+typedef struct tq_planes {
+    uint8_t* codes;
+    uint8_t* qjl;
+    float* norms;
+    float* rnorms;
+} tq_planes;
+
+/*
+ * Create a split of d = outer.d + inner.d channels. h_channels: host array of m = outer.d
+ * distinct channel indices in [0, d), ascending. Both states must have the same mode and
+ * device; the split keeps pointers to them (they must outlive it) and a device copy of the
+ * two channel maps. TQ_EINVAL on any mismatch.
+ */
+int tq_split_create(const tq_state* outer, const tq_state* inner, const int32_t* h_channels, int m,
+                    tq_split** out);
+
+/* Free a split (NULL is allowed). */
+void tq_split_destroy(tq_split* sp);
+
+/*
+ * Quantize n rows x [n][ld] (dtype TQ_F32/TQ_BF16, row stride ld >= d elements, 16-byte
+ * aligned base and stride): the outer group into `outer`'s planes [n], the inner group into
+ * `inner`'s planes [n]. Plane pointers 16-byte aligned, as for tq_quantize_*.
+ */
+int tq_split_quantize(const tq_split* sp, const void* x, int dtype, int64_t n, int64_t ld,
+                      const tq_planes* outer, const tq_planes* inner, void* stream);
+
+/* Reconstruct rows out fp32 [n][d] (16-byte aligned) from both groups' planes. */
+int tq_split_dequant(const tq_split* sp, const tq_planes* outer, const tq_planes* inner, int64_t n,
+                     float* out, void* stream);
+
+/*
+ * Estimates as tq_score (queries [groups][nq][d], planes [groups][n], scores fp32
+ * [groups][nq][n]), summed over the two groups. The queries' channel groups are gathered
+ * into a stream-ordered scratch buffer.
+ */
+int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups, int64_t nq,
+                   const tq_planes* outer, const tq_planes* inner, int64_t n, float* scores,
+                   void* stream);
+
+/* Workspace bytes that tq_split_attend_decode needs for H heads and T tokens. */
+int tq_split_attend_workspace(const tq_split* ks, const tq_split* vs, int H, int64_t T, size_t* bytes);
+
+/*
+ * One decode step of attention (as tq_attend_decode) over channel-split caches: K split `ks`
+ * (MSE or prod groups), V split `vs` (MSE groups), both over the same d channels (their
+ * outlier lists may differ). s_t = scale * (sum over the K groups of <q_group, k~_t,group>),
+ * p = softmax(s), out_h = sum_t p_t v~_t with each V group reconstructed in its own
+ * channels. Planes [H][T] per group; q [H][d]; out fp32 [H][d]; workspace of at least
+ * tq_split_attend_workspace() bytes, 256-byte aligned.
+ */
+int tq_split_attend_decode(const tq_split* ks, const tq_split* vs, const void* q, int qdtype, int H, int64_t T,
+                           const tq_planes* k_outer, const tq_planes* k_inner, const tq_planes* v_outer,
+                           const tq_planes* v_inner, float scale, float* out, void* workspace,
+                           size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

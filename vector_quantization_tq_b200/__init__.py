@@ -55,6 +55,12 @@ def _load():
     return ctypes.CDLL(LIB_PATH, mode=ctypes.RTLD_GLOBAL)
 
 
+class Planes(ctypes.Structure):
+    """Device planes of one channel group (tq_planes): codes, qjl, norms, rnorms."""
+    _fields_ = [("codes", ctypes.c_void_p), ("qjl", ctypes.c_void_p), ("norms", ctypes.c_void_p),
+                ("rnorms", ctypes.c_void_p)]
+
+
 _lib = _load()
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -89,6 +95,19 @@ _SIGS = {
     "tq_ip_stats": (_I, [_P, _P, _I64, _I, _P, _I64, _P, _P, _I]),
     "tq_search_workspace": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_SZ)]),
     "tq_search_topk": (_I, [_P, _P, _I, _I64, _P, _P, _P, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "tq_attend_decode_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float,
+                                      _P, _P, _SZ, _P]),
+    "tq_attend_append_decode": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _I, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                     ctypes.c_float, _P, _P, _SZ, _P]),
+    "tq_split_create": (_I, [_P, _P, _P, _I, ctypes.POINTER(_P)]),
+    "tq_split_destroy": (None, [_P]),
+    "tq_split_quantize": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _P]),
+    "tq_split_dequant": (_I, [_P, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _I64, _P, _P]),
+    "tq_split_score": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _I64, _P, _P]),
+    "tq_split_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
+    "tq_split_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes),
+                                    ctypes.POINTER(Planes), ctypes.POINTER(Planes), ctypes.c_float, _P, _P, _SZ,
+                                    _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -321,6 +340,29 @@ def attend_decode(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms, vcodes
                                  _ptr(workspace), ws_bytes, _stream(stream)), "tq_attend_decode")
 
 
+def attend_decode_grouped(ks: State, vs: State, q, G: int, T: int, Tcap: int, kcodes, kqjl, knorms, krnorms, vcodes,
+                          vnorms, scale: float, out, workspace, ws_bytes=None, stream=None):
+    """H = q.shape[0] query heads, G per KV head; planes [H/G][Tcap], the first T rows valid."""
+    H = q.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.tq_attend_decode_grouped(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, G, T, Tcap, _ptr(kcodes),
+                                         _ptr(kqjl), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
+                                         float(scale), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "tq_attend_decode_grouped")
+
+
+def attend_append_decode(ks: State, vs: State, q, G: int, k_new, v_new, T: int, Tcap: int, kcodes, kqjl, knorms,
+                         krnorms, vcodes, vnorms, scale: float, out, workspace, ws_bytes=None, stream=None):
+    """Encode k_new / v_new [H/G][d] into row T of each KV head's planes, then attend over T + 1 tokens."""
+    H = q.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.tq_attend_append_decode(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, G, _ptr(k_new),
+                                        _ptr(v_new), _dtype_code(k_new), T, Tcap, _ptr(kcodes), _ptr(kqjl),
+                                        _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale),
+                                        _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "tq_attend_append_decode")
+
+
 def attend_decode_noalloc(ks: State, vs: State, q, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale: float,
                           out, H=None, T=None, stream=None):
     """tq_attend_decode with the library's fixed device scratch instead of a workspace.
@@ -357,3 +399,87 @@ def search_topk(st: State, q, codes, qjl, norms, rnorms, k: int, idx, vals, work
     _check(_lib.tq_search_topk(st.handle, _ptr(q), _dtype_code(q), nq, _ptr(codes), _ptr(qjl), _ptr(norms),
                                _ptr(rnorms), n, k, _ptr(idx), _ptr(vals), _ptr(workspace), ws_bytes,
                                _stream(stream)), "tq_search_topk")
+
+
+# ---- outlier-channel split ----------------------------------------------------------------
+
+def _planes(pl):
+    codes, qjl, norms, rnorms = pl
+    return Planes(_ptr(codes), _ptr(qjl), _ptr(norms), _ptr(rnorms))
+
+
+class Split:
+    """The channels `channels` (ascending) quantized by `outer`, the rest by `inner`."""
+
+    def __init__(self, outer: State, inner: State, channels):
+        ch = np.ascontiguousarray(channels, dtype=np.int32)
+        self.outer, self.inner = outer, inner
+        self.channels = ch
+        self.d = outer.d + inner.d
+        self._h = _P()
+        _check(_lib.tq_split_create(outer.handle, inner.handle, ch.ctypes.data, len(ch), ctypes.byref(self._h)),
+               "tq_split_create")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def empty_planes(self, n: int, device=None):
+        """((codes, qjl, norms, rnorms) of the outer group, same of the inner group)."""
+        return self.outer.empty_planes(n, device), self.inner.empty_planes(n, device)
+
+    def close(self):
+        if self._h:
+            _lib.tq_split_destroy(self._h)
+            self._h = _P()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def split_quantize(sp: Split, x, outer_planes, inner_planes, stream=None, n=None, ld=None):
+    n = x.shape[0] if n is None else n
+    ld = x.stride(0) if ld is None else ld
+    po, pi = _planes(outer_planes), _planes(inner_planes)
+    _check(_lib.tq_split_quantize(sp.handle, _ptr(x), _dtype_code(x), n, ld, ctypes.byref(po), ctypes.byref(pi),
+                                  _stream(stream)), "tq_split_quantize")
+
+
+def split_dequant(sp: Split, outer_planes, inner_planes, out, stream=None, n=None):
+    n = out.shape[0] if n is None else n
+    po, pi = _planes(outer_planes), _planes(inner_planes)
+    _check(_lib.tq_split_dequant(sp.handle, ctypes.byref(po), ctypes.byref(pi), n, _ptr(out), _stream(stream)),
+           "tq_split_dequant")
+
+
+def split_score(sp: Split, q, outer_planes, inner_planes, scores, groups: int = 1, nq=None, n=None, stream=None):
+    nq = (q.shape[-2] if q.dim() == 3 else q.shape[0] // groups) if nq is None else nq
+    norms = outer_planes[2]
+    n = norms.shape[-1] if n is None else n
+    if norms.dim() == 1 and n == norms.shape[0] and groups > 1:
+        n = norms.shape[0] // groups
+    po, pi = _planes(outer_planes), _planes(inner_planes)
+    _check(_lib.tq_split_score(sp.handle, _ptr(q), _dtype_code(q), groups, nq, ctypes.byref(po), ctypes.byref(pi),
+                               n, _ptr(scores), _stream(stream)), "tq_split_score")
+
+
+def split_attend_workspace(ks: Split, vs: Split, H: int, T: int) -> int:
+    n = _SZ()
+    _check(_lib.tq_split_attend_workspace(ks.handle, vs.handle, H, T, ctypes.byref(n)), "tq_split_attend_workspace")
+    return n.value
+
+
+def split_attend_decode(ks: Split, vs: Split, q, k_planes, v_planes, scale: float, out, workspace, ws_bytes=None,
+                        H=None, T=None, stream=None):
+    """k_planes / v_planes: (outer planes, inner planes) as from Split.empty_planes."""
+    H = q.shape[0] if H is None else H
+    T = k_planes[0][2].numel() // H if T is None else T
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    ko, ki = _planes(k_planes[0]), _planes(k_planes[1])
+    vo, vi = _planes(v_planes[0]), _planes(v_planes[1])
+    _check(_lib.tq_split_attend_decode(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, ctypes.byref(ko),
+                                       ctypes.byref(ki), ctypes.byref(vo), ctypes.byref(vi), float(scale), _ptr(out),
+                                       _ptr(workspace), ws_bytes, _stream(stream)), "tq_split_attend_decode")

@@ -64,7 +64,8 @@ struct TileBuf {
 
 template <int BK, bool KPROD, int BV>
 __global__ void __launch_bounds__(kThreads)
-attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict__ luts, int64_t T, int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
+attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict__ luts, int64_t T, int G, int64_t Tcap,
+                  int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
                   const float* __restrict__ knorms, const float* __restrict__ krnorms,
                   const uint8_t* __restrict__ vcodes, const float* __restrict__ vnorms, float scale,
                   float* __restrict__ part) {
@@ -87,7 +88,7 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t_begin = (int64_t)split * chunk;
     const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
-    const int64_t hT = (int64_t)h * T;
+    const int64_t hT = (int64_t)(h / G) * Tcap;   // planes of this query head's KV head
 
     // Stage a tile (tokens t0 .. t0+255 of this head) into buffer `sb`; rows past the end of
     // this split are not copied and not read.
@@ -268,7 +269,7 @@ size_t smem_bytes() {
 }
 
 template <int BK, bool KPROD, int BV>
-int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
+int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     auto kern = attend_lut_kernel<BK, KPROD, BV>;
@@ -278,36 +279,36 @@ int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, i
         if (e != cudaSuccess) return (int)e;
     }
     dim3 grid((unsigned)nsplit, (unsigned)H);
-    kern<<<grid, kThreads, smem, s>>>(ks, vs, luts, T, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale,
+    kern<<<grid, kThreads, smem, s>>>(ks, vs, luts, T, G, Tcap, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale,
                                       part);
     return (int)cudaGetLastError();
 }
 
 template <int BK, bool KPROD>
-int launch_v(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
+int launch_v(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     switch (vs.b_mse) {
-        case 2: return launch_t<BK, KPROD, 2>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 2: return launch_t<BK, KPROD, 2>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
-        case 3: return launch_t<BK, KPROD, 3>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 3: return launch_t<BK, KPROD, 3>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
-        case 4: return launch_t<BK, KPROD, 4>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 4: return launch_t<BK, KPROD, 4>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                               vcodes, vnorms, scale, part, s);
         default: return (int)cudaErrorInvalidValue;
     }
 }
 
 template <bool KPROD>
-int launch_k(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int nsplit,
+int launch_k(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap, int nsplit,
              int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
              const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
     switch (ks.b_mse) {
-        case 2: return launch_v<2, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 2: return launch_v<2, KPROD>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
-        case 3: return launch_v<3, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 3: return launch_v<3, KPROD>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
-        case 4: return launch_v<4, KPROD>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+        case 4: return launch_v<4, KPROD>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
                                           vcodes, vnorms, scale, part, s);
         default: return (int)cudaErrorInvalidValue;
     }
@@ -321,14 +322,14 @@ bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kc
     return a16(kcodes) && a16(vcodes) && (kqjl == nullptr || a16(kqjl)) && ks.d == kD && vs.d == kD && ks.b_mse >= 2 && ks.b_mse <= 4 && vs.b_mse >= 2 && vs.b_mse <= 4;
 }
 
-int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T,
-                            int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G,
+                            int64_t Tcap, int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                             float scale, float* part, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    if (kqjl) return launch_k<true>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes,
+    if (kqjl) return launch_k<true>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes,
                                     vnorms, scale, part, s);
-    return launch_k<false>(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
+    return launch_k<false>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
                            scale, part, s);
 }
 

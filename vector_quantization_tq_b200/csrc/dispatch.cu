@@ -4,8 +4,8 @@
 
 namespace tq {
 
-int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
-                          uint8_t* qjl, float* norms, float* rnorms, void* stream);
+int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
+                          int64_t ostride, uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
 
 bool encode_tc_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
 int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl,
@@ -40,7 +40,20 @@ int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64
     }
     if (encode_tc_supported(st, dtype, n, ld))
         return launch_encode_tc(st, x, n, ld, codes, qjl, norms, rnorms, stream);
-    return launch_encode_generic(st, x, dtype, n, ld, codes, qjl, norms, rnorms, stream);
+    return launch_encode_generic(st, x, dtype, n, ld, nullptr, 1, codes, qjl, norms, rnorms, stream);
+}
+
+// Encode the channels chan[0..d) of each input row (a channel group of a split).
+int launch_encode_channels(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
+                           uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+    return launch_encode_generic(st, x, dtype, n, ld, chan, 1, codes, qjl, norms, rnorms, stream);
+}
+
+// Encode n rows into plane rows 0, ostride, 2 ostride, ... (one new token per head of a
+// cache whose heads are ostride rows apart).
+int launch_encode_strided(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, int64_t ostride,
+                          uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+    return launch_encode_generic(st, x, dtype, n, ld, nullptr, ostride, codes, qjl, norms, rnorms, stream);
 }
 
 }  // namespace tq

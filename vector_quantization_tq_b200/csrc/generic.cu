@@ -48,7 +48,7 @@ __device__ __forceinline__ void fwht(float (&v)[E], int tid, float* xch) {
     for (int h = 1; h < E; h <<= 1) {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            if ((e & h) == 0) {
+            if ((e & h) == 0 && e + h < E) {   // always true for the power-of-two E the RHT uses
                 const float a = v[e], b = v[e + h];
                 v[e] = a + b;
                 v[e + h] = a - b;
@@ -87,8 +87,8 @@ __device__ __forceinline__ int groups_per_block() { return NT == 32 ? 8 : 1; }
 template <int E, int NT>
 __global__ void __launch_bounds__(NT == 32 ? 256 : NT)
 encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t n, int64_t ld,
-              uint8_t* __restrict__ codes, uint8_t* __restrict__ qjl, float* __restrict__ norms,
-              float* __restrict__ rnorms) {
+              const int32_t* __restrict__ chan, int64_t ostride, uint8_t* __restrict__ codes,
+              uint8_t* __restrict__ qjl, float* __restrict__ norms, float* __restrict__ rnorms) {
     constexpr int D = NT * E;
     constexpr int GPB = (NT == 32) ? 8 : 1;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -112,7 +112,12 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
 
     for (int64_t vec = (int64_t)blockIdx.x * GPB + g; vec < n; vec += (int64_t)gridDim.x * GPB) {
         float xv[E];
-        load_elems<E>(x, dtype, vec * ld + (int64_t)tid * E, xv);
+        if (chan == nullptr) {
+            load_elems<E>(x, dtype, vec * ld + (int64_t)tid * E, xv);
+        } else {   // element j of this vector is channel chan[j] of the input row
+#pragma unroll
+            for (int e = 0; e < E; ++e) xv[e] = mat_elem(x, dtype, vec * ld + __ldg(chan + tid * E + e));
+        }
         float ss = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) ss = fmaf(xv[e], xv[e], ss);
@@ -156,18 +161,18 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
 #pragma unroll
             for (int e = 0; e < E; ++e) zbuf[tid * E + e] = (s[e] >= 0.f) ? 1 : 0;
             if (tid == 0) {
-                norms[vec] = nu;
-                rnorms[vec] = rho;
+                norms[vec * ostride] = nu;
+                rnorms[vec * ostride] = rho;
             }
         } else if (tid == 0) {
-            norms[vec] = nu;
+            norms[vec * ostride] = nu;
         }
         group_sync<NT>();
         // pack codes: stream bit p = 32w + lane -> code p / b, bit p % b
         if (st.b_mse > 0) {
             const int b = st.b_mse;
             const int W = b * D / 32;
-            uint32_t* out = reinterpret_cast<uint32_t*>(codes + vec * st.code_bytes);
+            uint32_t* out = reinterpret_cast<uint32_t*>(codes + vec * ostride * st.code_bytes);
             for (int w = warp_in_group; w < W; w += WPG) {
                 const int p = 32 * w + lane;
                 const int j = p / b;
@@ -177,7 +182,7 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
             }
         }
         if (prod) {
-            uint32_t* out = reinterpret_cast<uint32_t*>(qjl + vec * st.qjl_bytes);
+            uint32_t* out = reinterpret_cast<uint32_t*>(qjl + vec * ostride * st.qjl_bytes);
             for (int w = warp_in_group; w < D / 32; w += WPG) {
                 const uint32_t word = __ballot_sync(0xffffffffu, zbuf[32 * w + lane]);
                 if (lane == 0) out[w] = word;
@@ -194,7 +199,7 @@ template <int E, int NT>
 __global__ void __launch_bounds__(NT == 32 ? 256 : NT)
 dequant_kernel(const DevState st, const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
                const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
-               float* __restrict__ out) {
+               const int32_t* __restrict__ chan, int64_t ldo, float* __restrict__ out) {
     constexpr int D = NT * E;
     constexpr int GPB = (NT == 32) ? 8 : 1;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -240,9 +245,14 @@ dequant_kernel(const DevState st, const uint8_t* __restrict__ codes, const uint8
             group_sync<NT>();
         }
         const float nu = __ldg(norms + vec);
-        float* o = out + vec * D + tid * E;
+        if (chan == nullptr) {
+            float* o = out + vec * ldo + tid * E;
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = xo[e] * nu;
+            for (int e = 0; e < E; ++e) o[e] = xo[e] * nu;
+        } else {   // element j goes to channel chan[j] of the output row
+#pragma unroll
+            for (int e = 0; e < E; ++e) out[vec * ldo + __ldg(chan + tid * E + e)] = xo[e] * nu;
+        }
     }
 }
 
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t nq,
              const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
              const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
-             float* __restrict__ scores) {
+             int accumulate, float* __restrict__ scores) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int d = st.d;
     float* ctab = reinterpret_cast<float*>(smem_raw);
@@ -321,7 +331,11 @@ score_kernel(const DevState st, const void* __restrict__ q, int qdtype, int64_t 
         score_sums<kScoreQT>(st, ctab, qp, u, nqt, codes, qjl, gk, a1, a2);
         const float nu = __ldg(norms + gk);
         const float g2 = (qjl != nullptr) ? __ldg(rnorms + gk) * st.qjl_scale : 0.f;
-        for (int i = 0; i < nqt; ++i) scores[(grp * nq + q0 + i) * n + key] = nu * fmaf(g2, a2[i], a1[i]);
+        for (int i = 0; i < nqt; ++i) {
+            float* dst = scores + (grp * nq + q0 + i) * n + key;
+            const float v = nu * fmaf(g2, a2[i], a1[i]);
+            *dst = accumulate ? *dst + v : v;
+        }
     }
 }
 
@@ -339,7 +353,7 @@ size_t attend_smem_bytes(int d) {
 
 __global__ void __launch_bounds__(kAttThreads)
 attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict__ q, int qdtype,
-                    int64_t T, int64_t chunk, const uint8_t* __restrict__ kcodes,
+                    int64_t T, int G, int64_t Tcap, int64_t chunk, const uint8_t* __restrict__ kcodes,
                     const uint8_t* __restrict__ kqjl, const float* __restrict__ knorms,
                     const float* __restrict__ krnorms, const uint8_t* __restrict__ vcodes,
                     const float* __restrict__ vnorms, float scale, float* __restrict__ part) {
@@ -363,6 +377,7 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
     prep_queries_dev(ks, reinterpret_cast<const unsigned char*>(q) + (size_t)h * d * qelem, qdtype, 1, qs, qp, u,
                      stage);
 
+    const int64_t kvb = (int64_t)(h / G) * Tcap;   // planes of this query head's KV head
     const int64_t t_begin = (int64_t)split * chunk;
     const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
     // Value accumulation layout: d <= 256: `per` threads per coordinate split the tokens;
@@ -371,6 +386,7 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
     const int jpt = (d <= kAttThreads) ? 1 : d / kAttThreads;
     const int j0 = (d <= kAttThreads) ? (threadIdx.x % d) : threadIdx.x;
     const int half = (d <= kAttThreads) ? (threadIdx.x / d) : 0;
+    const bool vact = half < per;   // d not dividing 256: the last threads take no coordinate
     float acc[kAttMaxJ];
 #pragma unroll
     for (int m = 0; m < kAttMaxJ; ++m) acc[m] = 0.f;
@@ -380,12 +396,92 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
         const int cnt = (int)(t_end - t0 < kAttThreads ? t_end - t0 : kAttThreads);
         float s = -INFINITY;
         if (threadIdx.x < cnt) {
-            const int64_t gk = (int64_t)h * T + t0 + threadIdx.x;
+            const int64_t gk = kvb + t0 + threadIdx.x;
             float a1[1], a2[1];
             score_sums<1>(ks, kc, qp, u, 1, kcodes, kqjl, gk, a1, a2);
             const float g2 = (kqjl != nullptr) ? __ldg(krnorms + gk) * ks.qjl_scale : 0.f;
             s = scale * __ldg(knorms + gk) * fmaf(g2, a2[0], a1[0]);
         }
+        float mx = warp_max(s);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        float tmax = red[0];
+        for (int i = 1; i < kAttThreads / 32; ++i) tmax = fmaxf(tmax, red[i]);
+        __syncthreads();
+        const float m_new = fmaxf(m_run, tmax);
+        const float alpha = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
+        const float p = (threadIdx.x < cnt) ? __expf(s - m_new) : 0.f;
+        const float psum = warp_sum(p);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = psum;
+        if (threadIdx.x < cnt) wt[threadIdx.x] = p * __ldg(vnorms + kvb + t0 + threadIdx.x);
+        __syncthreads();
+        float tsum = 0.f;
+        for (int i = 0; i < kAttThreads / 32; ++i) tsum += red[i];
+        l_run = l_run * alpha + tsum;
+        m_run = m_new;
+#pragma unroll
+        for (int m = 0; m < kAttMaxJ; ++m) acc[m] *= alpha;
+        for (int t = half; vact && t < cnt; t += per) {
+            const uint32_t* row =
+                reinterpret_cast<const uint32_t*>(vcodes + (kvb + t0 + t) * vs.code_bytes);
+            const float w = wt[t];
+#pragma unroll
+            for (int m = 0; m < kAttMaxJ; ++m)
+                if (m < jpt) acc[m] = fmaf(w, vc[extract_code(row, vnw, j0 + m * kAttThreads, vs.b_mse)], acc[m]);
+        }
+        __syncthreads();
+    }
+    float* rec = part + ((int64_t)h * nsplit + split) * (d + 2);
+    if (d <= kAttThreads) {
+        if (vact) accs[half * d + j0] = acc[0];
+        __syncthreads();
+        for (int jj = threadIdx.x; jj < d; jj += blockDim.x) {
+            float a = 0.f;
+            for (int hh = 0; hh < per; ++hh) a += accs[hh * d + jj];
+            rec[2 + jj] = a;
+        }
+    } else {
+        for (int m = 0; m < jpt; ++m) rec[2 + j0 + m * kAttThreads] = acc[m];
+    }
+    if (threadIdx.x == 0) {
+        rec[0] = m_run;
+        rec[1] = l_run;
+    }
+}
+
+// Value sums of a decode step whose scores are given: per head h, s_t = scale * scores[h][t];
+// block (split, h) writes the record (m, l, acc[dv]) of its tokens, acc in the rotated domain
+// of the value state (the layout attend_combine_kernel merges). Used for channel-split caches,
+// where each channel group of V has its own state and gets its own records.
+__global__ void __launch_bounds__(kAttThreads)
+attend_values_kernel(const DevState vs, const float* __restrict__ scores, float scale, int64_t T, int64_t chunk,
+                     const uint8_t* __restrict__ vcodes, const float* __restrict__ vnorms, float* __restrict__ part) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int d = vs.d;
+    const int h = blockIdx.y;
+    const int split = blockIdx.x;
+    const int nsplit = gridDim.x;
+    float* vc = reinterpret_cast<float*>(smem_raw);       // V centroids
+    float* wt = vc + kMaxLevels;                          // kAttThreads weights p_t * ||v_t||
+    float* red = wt + kAttThreads;                        // 32
+    float* accs = red + 32;                               // max(d, kAttThreads)
+    for (int i = threadIdx.x; i < vs.L; i += blockDim.x) vc[i] = vs.c[i];
+    __syncthreads();
+    const int64_t t_begin = (int64_t)split * chunk;
+    const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
+    const int per = (d <= kAttThreads) ? kAttThreads / d : 1;
+    const int jpt = (d <= kAttThreads) ? 1 : d / kAttThreads;
+    const int j0 = (d <= kAttThreads) ? (threadIdx.x % d) : threadIdx.x;
+    const int half = (d <= kAttThreads) ? (threadIdx.x / d) : 0;
+    const bool vact = half < per;
+    float acc[kAttMaxJ];
+#pragma unroll
+    for (int m = 0; m < kAttMaxJ; ++m) acc[m] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const int vnw = vs.code_bytes / 4;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += kAttThreads) {
+        const int cnt = (int)(t_end - t0 < kAttThreads ? t_end - t0 : kAttThreads);
+        const float s = (threadIdx.x < cnt) ? scale * __ldg(scores + (int64_t)h * T + t0 + threadIdx.x) : -INFINITY;
         float mx = warp_max(s);
         if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
         __syncthreads();
@@ -405,7 +501,7 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
         m_run = m_new;
 #pragma unroll
         for (int m = 0; m < kAttMaxJ; ++m) acc[m] *= alpha;
-        for (int t = half; t < cnt; t += per) {
+        for (int t = half; vact && t < cnt; t += per) {
             const uint32_t* row =
                 reinterpret_cast<const uint32_t*>(vcodes + ((int64_t)h * T + t0 + t) * vs.code_bytes);
             const float w = wt[t];
@@ -417,7 +513,7 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
     }
     float* rec = part + ((int64_t)h * nsplit + split) * (d + 2);
     if (d <= kAttThreads) {
-        accs[half * d + j0] = acc[0];
+        if (vact) accs[half * d + j0] = acc[0];
         __syncthreads();
         for (int jj = threadIdx.x; jj < d; jj += blockDim.x) {
             float a = 0.f;
@@ -434,7 +530,8 @@ attend_split_kernel(const DevState ks, const DevState vs, const void* __restrict
 }
 
 __global__ void __launch_bounds__(256)
-attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ part, float* __restrict__ out) {
+attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ part, const int32_t* __restrict__ chan,
+                      int64_t ldo, float* __restrict__ out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int d = vs.d;
     const int h = blockIdx.x;
@@ -468,12 +565,12 @@ attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ p
             __syncthreads();
         }
         for (int k = threadIdx.x; k < d; k += blockDim.x)
-            out[(int64_t)h * d + k] = (rht_neg(vs, k) ? -o[k] : o[k]) * vs.rsqrt_d;
+            out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = (rht_neg(vs, k) ? -o[k] : o[k]) * vs.rsqrt_d;
     } else {
         for (int k = threadIdx.x; k < d; k += blockDim.x) {
             float a = 0.f;
             for (int j = 0; j < d; ++j) a = fmaf(mat_elem(vs.pi, vs.mat_dtype, (int64_t)j * d + k), o[j], a);
-            out[(int64_t)h * d + k] = a;
+            out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = a;
         }
     }
 }
@@ -637,8 +734,8 @@ int num_sms() {
 }
 
 template <int E, int NT>
-int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
-                    uint8_t* qjl, float* norms, float* rnorms, cudaStream_t s) {
+int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
+                    int64_t ostride, uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, cudaStream_t s) {
     constexpr int GPB = (NT == 32) ? 8 : 1;
     const int threads = NT * GPB;
     const size_t smem = (2 * kMaxLevels + 8) * sizeof(float) + GPB * (NT * E) * (sizeof(float) + 2);
@@ -646,13 +743,13 @@ int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int64_t blocks_needed = (n + GPB - 1) / GPB;
     const int blocks = (int)std::min<int64_t>(blocks_needed, (int64_t)num_sms() * 16);
-    kern<<<blocks, threads, smem, s>>>(st, x, dtype, n, ld, codes, qjl, norms, rnorms);
+    kern<<<blocks, threads, smem, s>>>(st, x, dtype, n, ld, chan, ostride, codes, qjl, norms, rnorms);
     return (int)cudaGetLastError();
 }
 
 template <int E, int NT>
 int launch_dequant_t(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
-                     const float* rnorms, int64_t n, float* out, cudaStream_t s) {
+                     const float* rnorms, int64_t n, const int32_t* chan, int64_t ldo, float* out, cudaStream_t s) {
     constexpr int GPB = (NT == 32) ? 8 : 1;
     const int threads = NT * GPB;
     const size_t smem = kMaxLevels * sizeof(float) + GPB * (NT * E) * sizeof(float);
@@ -660,54 +757,90 @@ int launch_dequant_t(const DevState& st, const uint8_t* codes, const uint8_t* qj
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int64_t blocks_needed = (n + GPB - 1) / GPB;
     const int blocks = (int)std::min<int64_t>(blocks_needed, (int64_t)num_sms() * 16);
-    kern<<<blocks, threads, smem, s>>>(st, codes, qjl, norms, rnorms, n, out);
+    kern<<<blocks, threads, smem, s>>>(st, codes, qjl, norms, rnorms, n, chan, ldo, out);
     return (int)cudaGetLastError();
+}
+
+// Calls f(E, NT) (as integral constants) for the thread layout of dimension d: a warp per
+// vector with E = d / 32 coordinates per lane up to d = 256, a block of NT = d / 8 above.
+template <typename F>
+int with_layout(int d, F&& f) {
+    using std::integral_constant;
+    switch (d) {
+        case 32: return f(integral_constant<int, 1>{}, integral_constant<int, 32>{});
+        case 64: return f(integral_constant<int, 2>{}, integral_constant<int, 32>{});
+        case 96: return f(integral_constant<int, 3>{}, integral_constant<int, 32>{});
+        case 128: return f(integral_constant<int, 4>{}, integral_constant<int, 32>{});
+        case 160: return f(integral_constant<int, 5>{}, integral_constant<int, 32>{});
+        case 192: return f(integral_constant<int, 6>{}, integral_constant<int, 32>{});
+        case 224: return f(integral_constant<int, 7>{}, integral_constant<int, 32>{});
+        case 256: return f(integral_constant<int, 8>{}, integral_constant<int, 32>{});
+        case 512: return f(integral_constant<int, 8>{}, integral_constant<int, 64>{});
+        case 1024: return f(integral_constant<int, 8>{}, integral_constant<int, 128>{});
+        case 1536: return f(integral_constant<int, 8>{}, integral_constant<int, 192>{});
+        case 2048: return f(integral_constant<int, 8>{}, integral_constant<int, 256>{});
+        default: return (int)cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
-int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
-                          uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
+                          int64_t ostride, uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    switch (st.d) {
-        case 32: return launch_encode_t<1, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 64: return launch_encode_t<2, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 128: return launch_encode_t<4, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 256: return launch_encode_t<8, 32>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 512: return launch_encode_t<8, 64>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 1024: return launch_encode_t<8, 128>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 1536: return launch_encode_t<8, 192>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        case 2048: return launch_encode_t<8, 256>(st, x, dtype, n, ld, codes, qjl, norms, rnorms, s);
-        default: return (int)cudaErrorInvalidValue;
-    }
+    return with_layout(st.d, [&](auto e, auto nt) {
+        return launch_encode_t<decltype(e)::value, decltype(nt)::value>(st, x, dtype, n, ld, chan, ostride, codes,
+                                                                         qjl, norms, rnorms, s);
+    });
 }
 
 int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
-                   const float* rnorms, int64_t n, float* out, void* stream) {
+                   const float* rnorms, int64_t n, const int32_t* chan, int64_t ldo, float* out, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    switch (st.d) {
-        case 32: return launch_dequant_t<1, 32>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 64: return launch_dequant_t<2, 32>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 128: return launch_dequant_t<4, 32>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 256: return launch_dequant_t<8, 32>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 512: return launch_dequant_t<8, 64>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 1024: return launch_dequant_t<8, 128>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 1536: return launch_dequant_t<8, 192>(st, codes, qjl, norms, rnorms, n, out, s);
-        case 2048: return launch_dequant_t<8, 256>(st, codes, qjl, norms, rnorms, n, out, s);
-        default: return (int)cudaErrorInvalidValue;
+    return with_layout(st.d, [&](auto e, auto nt) {
+        return launch_dequant_t<decltype(e)::value, decltype(nt)::value>(st, codes, qjl, norms, rnorms, n, chan,
+                                                                          ldo, out, s);
+    });
+}
+
+namespace {
+// out[r][j] = q[r][chan[j]] (elements of 2 or 4 bytes).
+template <typename T>
+__global__ void gather_rows_kernel(const T* __restrict__ q, int64_t count, int64_t ldq,
+                                   const int32_t* __restrict__ chan, int m, T* __restrict__ out) {
+    const int64_t total = count * m;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / m;
+        out[i] = q[r * ldq + __ldg(chan + (i - r * m))];
     }
+}
+}  // namespace
+
+int launch_gather_rows(const void* q, int dtype, int64_t count, int64_t ldq, const int32_t* chan, int m, void* out,
+                       void* stream) {
+    if (count <= 0 || m <= 0) return 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t total = count * m;
+    const int blocks = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 8);
+    if (dtype == TQ_F32)
+        gather_rows_kernel<float><<<blocks, 256, 0, s>>>(reinterpret_cast<const float*>(q), count, ldq, chan, m,
+                                                         reinterpret_cast<float*>(out));
+    else
+        gather_rows_kernel<uint16_t><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(q), count, ldq, chan,
+                                                            m, reinterpret_cast<uint16_t*>(out));
+    return (int)cudaGetLastError();
 }
 
 bool score_lut_supported(const DevState& st);
 int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
-                     void* stream);
+                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
+                     float* scores, void* stream);
 
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
-                 void* stream) {
+                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
+                 float* scores, void* stream) {
     if (score_lut_supported(st))
-        return launch_score_lut(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, stream);
+        return launch_score_lut(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, stream);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t smem = score_smem_bytes(st.d);
     if (smem > 48 * 1024) cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -718,7 +851,8 @@ int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, 
     kb = std::min<int64_t>(kb, std::max<int64_t>(want, 1));
     kb = std::min<int64_t>(kb, 1 << 20);
     dim3 grid((unsigned)kb, (unsigned)qtiles, (unsigned)groups);
-    score_kernel<<<grid, kScoreThreads, smem, s>>>(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, scores);
+    score_kernel<<<grid, kScoreThreads, smem, s>>>(st, q, qdtype, nq, codes, qjl, norms, rnorms, n, accumulate,
+                                                     scores);
     return (int)cudaGetLastError();
 }
 
@@ -733,8 +867,8 @@ int attend_splits(int H, int64_t T) {
 
 bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kcodes, const void* kqjl,
                           const void* vcodes);
-int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T,
-                            int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
+int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G,
+                            int64_t Tcap, int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl,
                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
                             float scale, float* part, void* stream);
 
@@ -751,8 +885,8 @@ size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T) {
     return b;
 }
 
-int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T,
-                  const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int G,
+                  int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
                   const uint8_t* vcodes, const float* vnorms, float scale, float* out, void* ws, size_t ws_bytes,
                   void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
@@ -765,19 +899,77 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
         float* luts = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ws) + attend_part_bytes(ks, H, T));
         e = (cudaError_t)launch_query_tables128(ks, q, qdtype, H, luts, stream);
         if (e == cudaSuccess)
-            e = (cudaError_t)launch_attend_lut_split(ks, vs, luts, H, T, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
-                                                     vcodes, vnorms, scale, part, stream);
+            e = (cudaError_t)launch_attend_lut_split(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms,
+                                                     krnorms, vcodes, vnorms, scale, part, stream);
     } else {
         const size_t smem = attend_smem_bytes(ks.d);
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(attend_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         dim3 grid((unsigned)nsplit, (unsigned)H);
-        attend_split_kernel<<<grid, kAttThreads, smem, s>>>(ks, vs, q, qdtype, T, chunk, kcodes, kqjl, knorms,
-                                                             krnorms, vcodes, vnorms, scale, part);
+        attend_split_kernel<<<grid, kAttThreads, smem, s>>>(ks, vs, q, qdtype, T, G, Tcap, chunk, kcodes, kqjl,
+                                                             knorms, krnorms, vcodes, vnorms, scale, part);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return (int)e;
-    attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, out);
+    attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, nullptr, vs.d, out);
+    return (int)cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------
+// Decode attention over channel-split K and V caches: scores summed over the two K groups
+// into the workspace, then per V group the value records and their combine (Pi_V^T of the
+// group, scattered to the group's channels of out).
+// ------------------------------------------------------------------------------------
+namespace {
+size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+}  // namespace
+
+size_t split_attend_ws_bytes(int dk, int dv_outer, int dv, int H, int64_t T) {
+    if (H <= 0 || T <= 0) return 0;
+    const int sp = attend_splits(H, T);
+    return al256((size_t)H * T * sizeof(float)) + al256((size_t)H * dk * sizeof(float)) +
+           al256((size_t)H * sp * (dv_outer + 2) * sizeof(float)) +
+           al256((size_t)H * sp * (dv - dv_outer + 2) * sizeof(float));
+}
+
+int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* kchan, const DevState& vo,
+                        const DevState& vi, const int32_t* vchan, const void* q, int qdtype, int H, int64_t T,
+                        const SplitPlanes& kp, const SplitPlanes& vp, float scale, float* out, void* ws,
+                        void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    const int dk = ko.d + ki.d, dv = vo.d + vi.d;
+    const size_t es = (qdtype == TQ_F32) ? 4 : 2;
+    unsigned char* w = reinterpret_cast<unsigned char*>(ws);
+    float* scores = reinterpret_cast<float*>(w);
+    w += al256((size_t)H * T * sizeof(float));
+    unsigned char* qo = w;
+    unsigned char* qi = w + (size_t)H * ko.d * es;   // ko.d * es is a multiple of 16
+    w += al256((size_t)H * dk * sizeof(float));
+    const int sp = attend_splits(H, T);
+    const int64_t chunk = (T + sp - 1) / sp;
+    const int nsplit = (int)((T + chunk - 1) / chunk);
+    float* part_o = reinterpret_cast<float*>(w);
+    float* part_i = reinterpret_cast<float*>(w + al256((size_t)H * sp * (vo.d + 2) * sizeof(float)));
+    int e = launch_gather_rows(q, qdtype, H, dk, kchan, ko.d, qo, stream);
+    if (e == 0) e = launch_gather_rows(q, qdtype, H, dk, kchan + ko.d, ki.d, qi, stream);
+    if (e == 0)
+        e = launch_score(ko, qo, qdtype, H, 1, kp.codes[0], kp.qjl[0], kp.norms[0], kp.rnorms[0], T, 0, scores,
+                         stream);
+    if (e == 0)
+        e = launch_score(ki, qi, qdtype, H, 1, kp.codes[1], kp.qjl[1], kp.norms[1], kp.rnorms[1], T, 1, scores,
+                         stream);
+    if (e != 0) return e;
+    for (int g = 0; g < 2; ++g) {
+        const DevState& v = g ? vi : vo;
+        float* part = g ? part_i : part_o;
+        const size_t smem = (size_t)(kMaxLevels + kAttThreads + 32 + (v.d > kAttThreads ? v.d : kAttThreads)) *
+                            sizeof(float);
+        dim3 grid((unsigned)nsplit, (unsigned)H);
+        attend_values_kernel<<<grid, kAttThreads, smem, s>>>(v, scores, scale, T, chunk, vp.codes[g], vp.norms[g],
+                                                             part);
+        attend_combine_kernel<<<H, 256, v.d * sizeof(float), s>>>(v, nsplit, part, g ? vchan + vo.d : vchan, dv,
+                                                                  out);
+    }
     return (int)cudaGetLastError();
 }
 

@@ -35,7 +35,8 @@ struct DeviceGuard {
 
 bool kernel_dim_supported(int d) {
     switch (d) {
-        case 32: case 64: case 128: case 256: case 512: case 1024: case 1536: case 2048:
+        case 32: case 64: case 96: case 128: case 160: case 192: case 224: case 256:
+        case 512: case 1024: case 1536: case 2048:
             return true;
         default:
             return false;
@@ -482,7 +483,7 @@ int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl, con
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
     return cuda_status((cudaError_t)launch_dequant(st->dev, codes, prod ? qjl : nullptr, norms,
-                                                   prod ? rnorms : nullptr, n, out, stream));
+                                                   prod ? rnorms : nullptr, n, nullptr, st->p.d, out, stream));
 }
 
 int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int64_t nq,
@@ -499,7 +500,169 @@ int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int6
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
     return cuda_status((cudaError_t)launch_score(st->dev, q, qdtype, groups, nq, codes, prod ? qjl : nullptr,
-                                                 norms, prod ? rnorms : nullptr, n, scores, stream));
+                                                 norms, prod ? rnorms : nullptr, n, 0, scores, stream));
+}
+
+// ---- outlier-channel split -----------------------------------------------------------
+
+namespace {
+bool planes_ok(const tq_state* st, const tq_planes* p) {
+    if (!p || !p->norms || !aligned16(p->norms)) return false;
+    if (st->b_mse > 0 && (!p->codes || !aligned16(p->codes))) return false;
+    if (st->p.mode == TQ_PROD && (!p->qjl || !p->rnorms || !aligned16(p->qjl) || !aligned16(p->rnorms)))
+        return false;
+    return true;
+}
+}  // namespace
+
+int tq_split_create(const tq_state* outer, const tq_state* inner, const int32_t* h_channels, int m,
+                    tq_split** out) {
+    if (!outer || !inner || !out || m < 1) return TQ_EINVAL;
+    *out = nullptr;
+    if (outer->p.d != m || outer->p.mode != inner->p.mode || outer->p.device != inner->p.device) return TQ_EINVAL;
+    if (!h_channels) return TQ_EINVAL;
+    const int d = m + inner->p.d;
+    std::vector<int32_t> maps(d);
+    for (int i = 0; i < m; ++i) {
+        if (h_channels[i] < 0 || h_channels[i] >= d || (i > 0 && h_channels[i] <= h_channels[i - 1])) return TQ_EINVAL;
+        maps[i] = h_channels[i];
+    }
+    for (int c = 0, j = 0, k = m; c < d; ++c) {   // the inner map: every channel not listed, ascending
+        if (j < m && h_channels[j] == c) ++j;
+        else maps[k++] = c;
+    }
+    DeviceGuard g(outer->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    auto* sp = new tq_split;
+    sp->outer = outer;
+    sp->inner = inner;
+    sp->d = d;
+    sp->channels.assign(h_channels, h_channels + m);
+    cudaError_t e = cudaMalloc(&sp->d_chan, (size_t)d * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemcpy(sp->d_chan, maps.data(), (size_t)d * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        if (sp->d_chan) cudaFree(sp->d_chan);
+        delete sp;
+        return cuda_status(e);
+    }
+    *out = sp;
+    return TQ_OK;
+}
+
+void tq_split_destroy(tq_split* sp) {
+    if (!sp) return;
+    if (sp->d_chan) {
+        DeviceGuard g(sp->outer->p.device);
+        cudaFree(sp->d_chan);
+    }
+    delete sp;
+}
+
+int tq_split_quantize(const tq_split* sp, const void* x, int dtype, int64_t n, int64_t ld,
+                      const tq_planes* outer, const tq_planes* inner, void* stream) {
+    if (!sp || n < 0) return TQ_EINVAL;
+    if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    const size_t es = (dtype == TQ_F32) ? 4 : 2;
+    if (!x || ld < sp->d || !aligned16(x) || ((size_t)ld * es) % 16) return TQ_EINVAL;
+    if (!planes_ok(sp->outer, outer) || !planes_ok(sp->inner, inner)) return TQ_EINVAL;
+    DeviceGuard g(sp->outer->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    const bool prod = sp->outer->p.mode == TQ_PROD;
+    const int m = sp->outer->p.d;
+    int e = launch_encode_channels(sp->outer->dev, x, dtype, n, ld, sp->d_chan, outer->codes,
+                                   prod ? outer->qjl : nullptr, outer->norms, prod ? outer->rnorms : nullptr, stream);
+    if (e == 0)
+        e = launch_encode_channels(sp->inner->dev, x, dtype, n, ld, sp->d_chan + m, inner->codes,
+                                   prod ? inner->qjl : nullptr, inner->norms, prod ? inner->rnorms : nullptr, stream);
+    return cuda_status((cudaError_t)e);
+}
+
+int tq_split_dequant(const tq_split* sp, const tq_planes* outer, const tq_planes* inner, int64_t n, float* out,
+                     void* stream) {
+    if (!sp || n < 0) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    if (!out || !aligned16(out) || !planes_ok(sp->outer, outer) || !planes_ok(sp->inner, inner)) return TQ_EINVAL;
+    DeviceGuard g(sp->outer->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    const bool prod = sp->outer->p.mode == TQ_PROD;
+    const int m = sp->outer->p.d;
+    int e = launch_dequant(sp->outer->dev, outer->codes, prod ? outer->qjl : nullptr, outer->norms,
+                           prod ? outer->rnorms : nullptr, n, sp->d_chan, sp->d, out, stream);
+    if (e == 0)
+        e = launch_dequant(sp->inner->dev, inner->codes, prod ? inner->qjl : nullptr, inner->norms,
+                           prod ? inner->rnorms : nullptr, n, sp->d_chan + m, sp->d, out, stream);
+    return cuda_status((cudaError_t)e);
+}
+
+int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups, int64_t nq,
+                   const tq_planes* outer, const tq_planes* inner, int64_t n, float* scores, void* stream) {
+    if (!sp || groups < 0 || nq < 0 || n < 0) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (groups == 0 || nq == 0 || n == 0) return TQ_OK;
+    if (groups > 65535) return TQ_EUNSUPPORTED;
+    if (!q || !scores || !aligned16(q) || !planes_ok(sp->outer, outer) || !planes_ok(sp->inner, inner))
+        return TQ_EINVAL;
+    DeviceGuard g(sp->outer->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool prod = sp->outer->p.mode == TQ_PROD;
+    const int m = sp->outer->p.d, r = sp->d - m;
+    const int64_t rows = groups * nq;
+    const size_t es = (qdtype == TQ_F32) ? 4 : 2;
+    // [rows][m] then [rows][d - m], each 256-byte aligned
+    const size_t b_out = ((size_t)rows * m * es + 255) & ~(size_t)255;
+    void* qg = nullptr;
+    cudaError_t ce = cudaMallocAsync(&qg, b_out + (size_t)rows * r * es, s);
+    if (ce != cudaSuccess) return cuda_status(ce);
+    void* q_in = reinterpret_cast<unsigned char*>(qg) + b_out;
+    int e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan, m, qg, stream);
+    if (e == 0) e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan + m, r, q_in, stream);
+    if (e == 0)
+        e = launch_score(sp->outer->dev, qg, qdtype, groups, nq, outer->codes, prod ? outer->qjl : nullptr,
+                         outer->norms, prod ? outer->rnorms : nullptr, n, 0, scores, stream);
+    if (e == 0)
+        e = launch_score(sp->inner->dev, q_in, qdtype, groups, nq, inner->codes, prod ? inner->qjl : nullptr,
+                         inner->norms, prod ? inner->rnorms : nullptr, n, 1, scores, stream);
+    const cudaError_t fe = cudaFreeAsync(qg, s);
+    return cuda_status(e ? (cudaError_t)e : fe);
+}
+
+int tq_split_attend_workspace(const tq_split* ks, const tq_split* vs, int H, int64_t T, size_t* bytes) {
+    if (!ks || !vs || !bytes || H < 0 || T < 0) return TQ_EINVAL;
+    *bytes = split_attend_ws_bytes(ks->d, vs->outer->p.d, vs->d, H, T);
+    return TQ_OK;
+}
+
+int tq_split_attend_decode(const tq_split* ks, const tq_split* vs, const void* q, int qdtype, int H, int64_t T,
+                           const tq_planes* k_outer, const tq_planes* k_inner, const tq_planes* v_outer,
+                           const tq_planes* v_inner, float scale, float* out, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    if (!ks || !vs || H < 0 || T < 0) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (vs->outer->p.mode != TQ_MSE || ks->d != vs->d || ks->outer->p.device != vs->outer->p.device)
+        return TQ_EINVAL;
+    if (!std::isfinite(scale)) return TQ_EINVAL;
+    if (H == 0) return TQ_OK;
+    if (T == 0 || H > 65535) return T == 0 ? TQ_EINVAL : TQ_EUNSUPPORTED;
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return TQ_EINVAL;
+    if (!planes_ok(ks->outer, k_outer) || !planes_ok(ks->inner, k_inner) || !planes_ok(vs->outer, v_outer) ||
+        !planes_ok(vs->inner, v_inner))
+        return TQ_EINVAL;
+    const size_t need = split_attend_ws_bytes(ks->d, vs->outer->p.d, vs->d, H, T);
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return TQ_EINVAL;
+    DeviceGuard g(ks->outer->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    const bool prod = ks->outer->p.mode == TQ_PROD;
+    SplitPlanes kp{{k_outer->codes, k_inner->codes},
+                   {prod ? k_outer->qjl : nullptr, prod ? k_inner->qjl : nullptr},
+                   {k_outer->norms, k_inner->norms},
+                   {prod ? k_outer->rnorms : nullptr, prod ? k_inner->rnorms : nullptr}};
+    SplitPlanes vp{{v_outer->codes, v_inner->codes}, {nullptr, nullptr}, {v_outer->norms, v_inner->norms},
+                   {nullptr, nullptr}};
+    return cuda_status((cudaError_t)launch_split_attend(ks->outer->dev, ks->inner->dev, ks->d_chan, vs->outer->dev,
+                                                         vs->inner->dev, vs->d_chan, q, qdtype, H, T, kp, vp, scale,
+                                                         out, workspace, stream));
 }
 
 int tq_attend_workspace(const tq_state* ks, const tq_state* vs, int H, int64_t T, size_t* bytes) {
@@ -528,9 +691,77 @@ int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int 
     if (ws_bytes < need) return TQ_ENOMEM;
     DeviceGuard g(ks->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
-    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, kcodes, prod ? kqjl : nullptr,
-                                                  knorms, prod ? krnorms : nullptr, vcodes, vnorms, scale, out,
-                                                  workspace, ws_bytes, stream));
+    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, 1, T, kcodes,
+                                                  prod ? kqjl : nullptr, knorms, prod ? krnorms : nullptr, vcodes,
+                                                  vnorms, scale, out, workspace, ws_bytes, stream));
+}
+
+namespace {
+// Checks shared by the grouped and appending decode steps.
+int check_grouped(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int G, int64_t T,
+                  int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                  const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale, const float* out) {
+    if (!ks || !vs || H < 1 || G < 1 || H % G != 0 || T < 1 || Tcap < T) return TQ_EINVAL;
+    if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
+    if (vs->p.mode != TQ_MSE || ks->p.d != vs->p.d || ks->p.device != vs->p.device) return TQ_EINVAL;
+    if (!std::isfinite(scale)) return TQ_EINVAL;
+    const bool prod = ks->p.mode == TQ_PROD;
+    if (!q || !out || !knorms || !vnorms || (ks->b_mse > 0 && !kcodes) || !vcodes ||
+        (prod && (!kqjl || !krnorms)))
+        return TQ_EINVAL;
+    if (!aligned16(q) || !aligned16(out)) return TQ_EINVAL;
+    return TQ_OK;
+}
+}  // namespace
+
+int tq_attend_decode_grouped(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int G,
+                             int64_t T, int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl,
+                             const float* knorms, const float* krnorms, const uint8_t* vcodes, const float* vnorms,
+                             float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_grouped(ks, vs, q, qdtype, H, G, T, Tcap, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale,
+                           out);
+    if (rc != TQ_OK) return rc;
+    const size_t need = attend_workspace_bytes(ks->dev, H, T);
+    if (need > 0 && (!workspace || ((uintptr_t)workspace & 255u))) return TQ_EINVAL;
+    if (ws_bytes < need) return TQ_ENOMEM;
+    DeviceGuard g(ks->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    const bool prod = ks->p.mode == TQ_PROD;
+    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, G, Tcap, kcodes,
+                                                  prod ? kqjl : nullptr, knorms, prod ? krnorms : nullptr, vcodes,
+                                                  vnorms, scale, out, workspace, ws_bytes, stream));
+}
+
+int tq_attend_append_decode(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int G,
+                            const void* k_new, const void* v_new, int kvdtype, int64_t T, int64_t Tcap,
+                            uint8_t* kcodes, uint8_t* kqjl, float* knorms, float* krnorms, uint8_t* vcodes,
+                            float* vnorms, float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+    if (T < 0 || T >= Tcap) return TQ_EINVAL;
+    int rc = check_grouped(ks, vs, q, qdtype, H, G, T + 1, Tcap, kcodes, kqjl, knorms, krnorms, vcodes, vnorms,
+                           scale, out);
+    if (rc != TQ_OK) return rc;
+    if (kvdtype != TQ_F32 && kvdtype != TQ_BF16) return TQ_EINVAL;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return TQ_EINVAL;
+    const size_t need = attend_workspace_bytes(ks->dev, H, T + 1);
+    if (need > 0 && (!workspace || ((uintptr_t)workspace & 255u))) return TQ_EINVAL;
+    if (ws_bytes < need) return TQ_ENOMEM;
+    DeviceGuard g(ks->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    const bool prod = ks->p.mode == TQ_PROD;
+    const int Hkv = H / G, d = ks->p.d;
+    // 1. the new token of every KV head into row T of that head's planes
+    int e = launch_encode_strided(ks->dev, k_new, kvdtype, Hkv, d, Tcap,
+                                  kcodes ? kcodes + T * ks->dev.code_bytes : nullptr,
+                                  prod ? kqjl + T * ks->dev.qjl_bytes : nullptr, knorms + T,
+                                  prod ? krnorms + T : nullptr, stream);
+    if (e == 0)
+        e = launch_encode_strided(vs->dev, v_new, kvdtype, Hkv, d, Tcap, vcodes + T * vs->dev.code_bytes, nullptr,
+                                  vnorms + T, nullptr, stream);
+    // 2. attention over the T + 1 tokens
+    if (e == 0)
+        e = launch_attend(ks->dev, vs->dev, q, qdtype, H, T + 1, G, Tcap, kcodes, prod ? kqjl : nullptr, knorms,
+                          prod ? krnorms : nullptr, vcodes, vnorms, scale, out, workspace, ws_bytes, stream);
+    return cuda_status((cudaError_t)e);
 }
 
 int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void* q, int qdtype, int H, int64_t T,
@@ -554,9 +785,9 @@ int tq_attend_decode_noalloc(const tq_state* ks, const tq_state* vs, const void*
     void* scratch = nullptr;
     int e = attend_static_scratch(&scratch);
     if (e != 0) return cuda_status((cudaError_t)e);
-    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, kcodes, prod ? kqjl : nullptr,
-                                                  knorms, prod ? krnorms : nullptr, vcodes, vnorms, scale, out,
-                                                  scratch, kAttendStaticScratchBytes, stream));
+    return cuda_status((cudaError_t)launch_attend(ks->dev, vs->dev, q, qdtype, H, T, 1, T, kcodes,
+                                                  prod ? kqjl : nullptr, knorms, prod ? krnorms : nullptr, vcodes,
+                                                  vnorms, scale, out, scratch, kAttendStaticScratchBytes, stream));
 }
 
 int tq_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,

@@ -53,6 +53,14 @@ struct tq_state {
     tq::DevState dev;                // kernel view
 };
 
+struct tq_split {
+    const tq_state* outer;           // channels `chan_outer`, dimension m
+    const tq_state* inner;           // the other channels, ascending, dimension d - m
+    int d;
+    std::vector<int32_t> channels;   // host copy of the outer channel list
+    int32_t* d_chan = nullptr;       // device: outer map [m], then inner map [d - m]
+};
+
 namespace tq {
 
 // ---- host helpers (host.cpp / codebook.cpp / linalg.cpp) ----
@@ -67,11 +75,33 @@ void set_cuda_error(int err);
 // ---- kernel launchers (kernels .cu files); all return a cudaError_t value ----
 int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld,
                   uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+int launch_encode_strided(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, int64_t ostride,
+                          uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+int launch_encode_channels(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
+                           uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+// out row stride ldo; chan (optional): element j of a vector goes to column chan[j]
 int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl,
-                   const float* norms, const float* rnorms, int64_t n, float* out, void* stream);
+                   const float* norms, const float* rnorms, int64_t n, const int32_t* chan, int64_t ldo,
+                   float* out, void* stream);
+// accumulate != 0: scores += estimates (else scores = estimates)
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq,
                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
-                 const float* rnorms, int64_t n, float* scores, void* stream);
+                 const float* rnorms, int64_t n, int accumulate, float* scores, void* stream);
+// rows of q [count][ldq] gathered at columns chan[0..m) into out [count][m] (same dtype)
+int launch_gather_rows(const void* q, int dtype, int64_t count, int64_t ldq, const int32_t* chan, int m, void* out,
+                       void* stream);
+// Planes of the two channel groups of a split (index 0: outer, 1: inner).
+struct SplitPlanes {
+    const uint8_t* codes[2];
+    const uint8_t* qjl[2];
+    const float* norms[2];
+    const float* rnorms[2];
+};
+size_t split_attend_ws_bytes(int dk, int dv_outer, int dv, int H, int64_t T);
+int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* kchan, const DevState& vo,
+                        const DevState& vi, const int32_t* vchan, const void* q, int qdtype, int H, int64_t T,
+                        const SplitPlanes& kp, const SplitPlanes& vp, float scale, float* out, void* ws,
+                        void* stream);
 int read_device_error(int* flag);
 int take_device_error_gemm(int* flag);
 int take_device_error_search(int* flag);
@@ -82,8 +112,9 @@ size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
 // QJL nibbles): floats per query, and a launch building them for `count` query rows.
 size_t query_table_floats(const DevState& st);
 int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, void* stream);
+// H query heads, G of them per KV head; the planes of KV head g start at row g * Tcap
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
-                  int64_t T, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+                  int64_t T, int G, int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
                   const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,
                   float* out, void* ws, size_t ws_bytes, void* stream);
 int attend_static_scratch(void** out);

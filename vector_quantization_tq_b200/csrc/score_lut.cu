@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kThreads)
 score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
                  const uint8_t* __restrict__ codes, const uint8_t* __restrict__ qjl,
                  const float* __restrict__ norms, const float* __restrict__ rnorms, int64_t n,
-                 int keys_per_block, float* __restrict__ scores) {
+                 int keys_per_block, int accumulate, float* __restrict__ scores) {
     using Gr = Groups<B>;
     using LS = LutShape<D, B, PROD>;
     constexpr int NG = LS::NG;
@@ -321,8 +321,13 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
             for (int wi = 0; wi < NQ / 8; ++wi) add_nibbles<QT, LS::SIZE>(z[wi], tab + LS::MSE + 8 * wi * 16, a2);
         }
 #pragma unroll
-        for (int qi = 0; qi < QT; ++qi)
-            if (qi < nqt) scores[(grp * nq + q0 + qi) * n + key] = nu * fmaf(g2, a2[qi], a1[qi]);
+        for (int qi = 0; qi < QT; ++qi) {
+            if (qi < nqt) {
+                float* dst = scores + (grp * nq + q0 + qi) * n + key;
+                const float v = nu * fmaf(g2, a2[qi], a1[qi]);
+                *dst = accumulate ? *dst + v : v;
+            }
+        }
     }
 }
 
@@ -340,8 +345,8 @@ int sm_count_lut() {
 
 template <int D, int B, bool PROD, int QT>
 int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-               const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
-               cudaStream_t s) {
+               const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
+               float* scores, cudaStream_t s) {
     using LS = LutShape<D, B, PROD>;
     const int64_t qtiles = (nq + QT - 1) / QT;
     if (qtiles > 65535 || groups > 65535 || groups * nq > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
@@ -364,7 +369,7 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
             ce = cudaErrorInvalidConfiguration;
         } else {
             dim3 grid((unsigned)kb, (unsigned)qtiles, (unsigned)groups);
-            kern<<<grid, kThreads, smem, s>>>(st, luts, nq, codes, qjl, norms, rnorms, n, (int)per, scores);
+            kern<<<grid, kThreads, smem, s>>>(st, luts, nq, codes, qjl, norms, rnorms, n, (int)per, accumulate, scores);
             ce = cudaGetLastError();
         }
     }
@@ -374,29 +379,29 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
 
 template <int D, int B, bool PROD>
 int launch_lut_q(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
                  cudaStream_t s) {
-    if (nq == 1) return launch_lut<D, B, PROD, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-    return launch_lut<D, B, PROD, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
+    if (nq == 1) return launch_lut<D, B, PROD, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+    return launch_lut<D, B, PROD, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
 }
 
 template <int D, int B>
 int launch_lut_m(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
                  cudaStream_t s) {
-    if (qjl) return launch_lut_q<D, B, true>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-    return launch_lut_q<D, B, false>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
+    if (qjl) return launch_lut_q<D, B, true>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+    return launch_lut_q<D, B, false>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
 }
 
 template <int D>
 int launch_lut_b(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                 const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
                  cudaStream_t s) {
     switch (st.b_mse) {
-        case 1: return launch_lut_m<D, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-        case 2: return launch_lut_m<D, 2>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-        case 3: return launch_lut_m<D, 3>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-        case 4: return launch_lut_m<D, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
+        case 1: return launch_lut_m<D, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 2: return launch_lut_m<D, 2>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 3: return launch_lut_m<D, 3>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 4: return launch_lut_m<D, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
         default: return (int)cudaErrorInvalidValue;
     }
 }
@@ -437,11 +442,11 @@ bool score_lut_supported(const DevState& st) {
 }
 
 int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
-                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, float* scores,
+                     const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
                      void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    if (st.d == 128) return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
-    return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, scores, s);
+    if (st.d == 128) return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+    return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
 }
 
 }  // namespace tq
