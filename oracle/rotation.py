@@ -16,7 +16,7 @@ from __future__ import annotations
 import numpy as np
 import scipy.linalg
 
-__all__ = ["haar_from_gaussian", "rht_matrix", "round_f32", "round_bf16"]
+__all__ = ["haar_from_gaussian", "paley_hadamard12", "hadamard", "rht_matrix", "round_f32", "round_bf16"]
 
 
 def haar_from_gaussian(g: np.ndarray) -> np.ndarray:
@@ -27,12 +27,33 @@ def haar_from_gaussian(g: np.ndarray) -> np.ndarray:
     return q * s[None, :]
 
 
+def paley_hadamard12() -> np.ndarray:
+    """Paley's Hadamard matrix of order 12 (from GF(11))."""
+    q = 11
+    residues = {(x * x) % q for x in range(1, q)}
+    chi = np.array([0.0] + [1.0 if a in residues else -1.0 for a in range(1, q)])
+    Q = np.array([[chi[(j - i) % q] for j in range(q)] for i in range(q)])
+    core = np.zeros((q + 1, q + 1))
+    core[0, 1:] = 1.0
+    core[1:, 0] = -1.0
+    core[1:, 1:] = Q
+    return np.eye(q + 1) + core
+
+
+def hadamard(d: int) -> np.ndarray:
+    """Hadamard matrix of order d: Sylvester's for d = 2^k, H_12 (x) Sylvester's for 12 * 2^k."""
+    if d & (d - 1) == 0:
+        return scipy.linalg.hadamard(d).astype(np.float64)
+    if d % 12 == 0 and (d // 12) & (d // 12 - 1) == 0:
+        return np.kron(paley_hadamard12(), scipy.linalg.hadamard(d // 12).astype(np.float64))
+    raise ValueError(f"no Hadamard matrix built for d = {d}")
+
+
 def rht_matrix(signs: np.ndarray) -> np.ndarray:
-    """Pi = H_d diag(eps) / sqrt(d) with H_d Sylvester's Hadamard matrix (d a power of two)."""
+    """Pi = H_d diag(eps) / sqrt(d) (see `hadamard` for the orders covered)."""
     eps = np.asarray(signs, dtype=np.float64)
     d = eps.shape[0]
-    h = scipy.linalg.hadamard(d).astype(np.float64)
-    return h * eps[None, :] / np.sqrt(d)
+    return hadamard(d) * eps[None, :] / np.sqrt(d)
 
 
 def round_f32(a: np.ndarray) -> np.ndarray:

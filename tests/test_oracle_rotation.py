@@ -9,6 +9,8 @@ vector over all 128 dimensions).
 import math
 
 import numpy as np
+import pytest
+import scipy.linalg
 from scipy import stats
 
 import synth
@@ -73,3 +75,27 @@ def test_uniform_inputs_fixed_rotation_follow_lemma1_and_gaussian_limit():
         if d == 1536:
             # Large d: the Beta law is close to N(0, 1/d).
             assert stats.kstest(v * math.sqrt(d), stats.norm.cdf).pvalue > 1e-3
+
+
+def test_paley_hadamard12_is_a_skew_hadamard_matrix():
+    # Paley I (q = 11): H H^T = 12 I, entries +-1, and H - I is skew-symmetric.
+    H = rot.paley_hadamard12()
+    assert H.shape == (12, 12) and set(np.unique(H)) == {-1.0, 1.0}
+    np.testing.assert_array_equal(H @ H.T, 12 * np.eye(12))
+    np.testing.assert_array_equal((H - np.eye(12)).T, -(H - np.eye(12)))
+    # the quadratic residues of GF(11) are 1, 3, 4, 5, 9: row 1 of Q, shifted by the border
+    np.testing.assert_array_equal(H[1, 2:], [1, -1, 1, 1, 1, -1, -1, -1, 1, -1])
+
+
+@pytest.mark.parametrize("d", [96, 192, 384, 1536])
+def test_kronecker_rht_is_orthogonal(d):
+    eps = synth.rht_signs(d, seed=2)
+    P = rot.rht_matrix(eps)
+    np.testing.assert_allclose(P @ P.T, np.eye(d), atol=1e-12)
+    # structure: entry (i, j) = H12[i / m][j / m] * H_m[i % m][j % m] * eps_j / sqrt(d), m = d / 12
+    m = d // 12
+    H12, Hm = rot.paley_hadamard12(), scipy.linalg.hadamard(m)
+    i, j = 5 * m + 3, 7 * m + 1
+    assert P[i, j] == H12[5, 7] * Hm[3, 1] * eps[j] / np.sqrt(d)
+    # a rotated one-hot vector spreads evenly: every |coordinate| = 1/sqrt(d)
+    np.testing.assert_allclose(np.abs(P[:, 17]), 1 / np.sqrt(d), rtol=1e-12)
