@@ -117,7 +117,7 @@ def test_state_create_validation_without_gpu():
     ]
     for p in bad:
         assert lib.tq_state_create(ctypes.byref(p), None, None, None, ctypes.byref(h)) == 1
-    unsup = [tq.Params(96, 3, 0, 1, 0, 0, 0, 1),  # RHT needs a power of two
+    unsup = [tq.Params(160, 3, 0, 1, 0, 0, 0, 1),  # RHT needs a Hadamard order: 2^k or 12 * 2^k
              tq.Params(100, 3, 0, 0, 0, 0, 0, 1)]  # no kernel for d = 100
     for p in unsup:
         assert lib.tq_state_create(ctypes.byref(p), None, None, None, ctypes.byref(h)) == 2

@@ -124,11 +124,14 @@ def test_c2_prod_rht_kv_keys(tokens):
 # --------------------------------------------------------------------------------------
 # Config 3 (reduced): fused decode attention, K prod b=4, V mse b=4, dense Pi.
 # --------------------------------------------------------------------------------------
-@pytest.mark.parametrize("H,T", [(3, 1000), (2, 300)])
-def test_c3_decode_attention(H, T):
-    d = 128
-    kp = Pair(tq, d, 4, tq.PROD, tq.ROT_DENSE, tq.F32)
-    vp = Pair(tq, d, 4, tq.MSE, tq.ROT_DENSE, tq.F32)
+@pytest.mark.parametrize("H,T,d,rot", [(3, 1000, 128, tq.ROT_DENSE), (2, 300, 128, tq.ROT_DENSE),
+                                       (2, 300, 96, tq.ROT_RHT), (2, 257, 192, tq.ROT_RHT),
+                                       (2, 300, 160, tq.ROT_DENSE)])
+def test_c3_decode_attention(H, T, d, rot):
+    # d = 128 runs the table kernel; the other shapes the general kernel (96 and 192 with the
+    # order-12 Kronecker Hadamard rotation, 160 a width that does not divide the block)
+    kp = Pair(tq, d, 4, tq.PROD, rot, tq.F32)
+    vp = Pair(tq, d, 4, tq.MSE, rot, tq.F32)
     K = synth.unit_vectors(H * T, d, seed=synth.SEED_DATA)
     V = synth.unit_vectors(H * T, d, seed=synth.SEED_DATA + 5)
     qb = synth.decode_queries(H, d)
@@ -175,6 +178,10 @@ CASES = [
     (128, 6, tq.MSE, tq.ROT_DENSE, tq.F32), (2048, 1, tq.PROD, tq.ROT_RHT, tq.BF16),
     (512, 2, tq.PROD, tq.ROT_DENSE, tq.BF16), (1536, 3, tq.MSE, tq.ROT_DENSE, tq.BF16),
     (1024, 4, tq.PROD, tq.ROT_DENSE, tq.BF16),
+    # Hadamard orders 12 * 2^k (Paley H_12 Kronecker Sylvester) and widths 32 k up to 256
+    (96, 3, tq.PROD, tq.ROT_RHT, tq.F32), (192, 2, tq.MSE, tq.ROT_RHT, tq.F32),
+    (1536, 2, tq.PROD, tq.ROT_RHT, tq.BF16), (160, 2, tq.PROD, tq.ROT_DENSE, tq.F32),
+    (224, 3, tq.MSE, tq.ROT_DENSE, tq.F32),
 ]
 
 

@@ -154,4 +154,42 @@ __device__ __forceinline__ void add_nibbles(uint32_t w, const float* t0, float (
     }
 }
 
+
+// In-place Hadamard transform of order d = 12 m (m a power of two) on buf[0..d), viewed as
+// 12 rows of m: Sylvester's transform along each row, then Paley's H_12 (rows of st.h12,
+// bit c of row a <=> H_12[a][c] = -1) across the rows; `transpose` applies H_12^T instead
+// (Sylvester's factor is symmetric), which inverts the transform up to 1/d. Threads
+// tid = 0..nt-1 of a group share buf; `sync` orders their shared-memory accesses.
+template <typename Sync>
+__device__ __forceinline__ void kron_hadamard(float* buf, int d, const uint32_t* __restrict__ h12, bool transpose,
+                                              int tid, int nt, Sync sync) {
+    const int m = d / 12;
+    for (int h = 1; h < m; h <<= 1) {
+        for (int p = tid; p < d / 2; p += nt) {
+            const int row = p / (m >> 1), pr = p - row * (m >> 1);
+            const int j = row * m + (pr / h) * 2 * h + (pr % h);
+            const float a = buf[j], b = buf[j + h];
+            buf[j] = a + b;
+            buf[j + h] = a - b;
+        }
+        sync();
+    }
+    for (int col = tid; col < m; col += nt) {
+        float t[12];
+#pragma unroll
+        for (int c = 0; c < 12; ++c) t[c] = buf[c * m + col];
+#pragma unroll
+        for (int a = 0; a < 12; ++a) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < 12; ++c) {
+                const bool neg = transpose ? ((h12[c] >> a) & 1u) : ((h12[a] >> c) & 1u);
+                acc += neg ? -t[c] : t[c];
+            }
+            buf[a * m + col] = acc;
+        }
+    }
+    sync();
+}
+
 }  // namespace tq

@@ -26,7 +26,7 @@ int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64
         cudaStream_t s = (cudaStream_t)stream;
         const int64_t chunk = n < kGemmChunk ? n : kGemmChunk;
         void* ws = nullptr;
-        cudaError_t e = cudaMallocAsync(&ws, encode_gemm_ws_bytes(st.d, chunk), s);
+        cudaError_t e = (cudaError_t)scratch_alloc(&ws, encode_gemm_ws_bytes(st.d, chunk), s);
         if (e != cudaSuccess) return (int)e;
         int rc = 0;
         for (int64_t c0 = 0; c0 < n && rc == 0; c0 += chunk) {
@@ -35,7 +35,7 @@ int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64
                                     codes + c0 * st.code_bytes, qjl ? qjl + c0 * st.qjl_bytes : nullptr,
                                     norms + c0, rnorms ? rnorms + c0 : nullptr, ws, stream);
         }
-        e = cudaFreeAsync(ws, s);
+        e = (cudaError_t)scratch_free(ws, s);
         return rc ? rc : (int)e;
     }
     if (encode_tc_supported(st, dtype, n, ld))

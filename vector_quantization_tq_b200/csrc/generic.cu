@@ -126,7 +126,17 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
         if (st.rot == TQ_ROT_RHT) {
 #pragma unroll
             for (int e = 0; e < E; ++e) y[e] = rht_neg(st, tid * E + e) ? -xv[e] : xv[e];
-            fwht<E, NT>(y, tid, vbuf);
+            if constexpr ((D & (D - 1)) == 0) {
+                fwht<E, NT>(y, tid, vbuf);
+            } else {   // d = 12 * 2^k
+#pragma unroll
+                for (int e = 0; e < E; ++e) vbuf[tid * E + e] = y[e];
+                group_sync<NT>();
+                kron_hadamard(vbuf, D, st.h12, false, tid, NT, [] { group_sync<NT>(); });
+#pragma unroll
+                for (int e = 0; e < E; ++e) y[e] = vbuf[tid * E + e];
+                group_sync<NT>();
+            }
             const float sc = (nu > 0.f) ? st.rsqrt_d / nu : 0.f;
 #pragma unroll
             for (int e = 0; e < E; ++e) y[e] *= sc;
@@ -234,7 +244,17 @@ dequant_kernel(const DevState st, const uint8_t* __restrict__ codes, const uint8
         }
         float xo[E];
         if (st.rot == TQ_ROT_RHT) {
-            fwht<E, NT>(yt, tid, vbuf);
+            if constexpr ((D & (D - 1)) == 0) {
+                fwht<E, NT>(yt, tid, vbuf);
+            } else {   // d = 12 * 2^k: the transposed transform
+#pragma unroll
+                for (int e = 0; e < E; ++e) vbuf[tid * E + e] = yt[e];
+                group_sync<NT>();
+                kron_hadamard(vbuf, D, st.h12, true, tid, NT, [] { group_sync<NT>(); });
+#pragma unroll
+                for (int e = 0; e < E; ++e) yt[e] = vbuf[tid * E + e];
+                group_sync<NT>();
+            }
 #pragma unroll
             for (int e = 0; e < E; ++e) xo[e] = (rht_neg(st, tid * E + e) ? -yt[e] : yt[e]) * st.rsqrt_d;
         } else {
@@ -555,14 +575,18 @@ attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ p
     __syncthreads();
     // out = Pi_V^T o
     if (vs.rot == TQ_ROT_RHT) {
-        for (int hh = 1; hh < d; hh <<= 1) {
-            for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
-                const int j = (p / hh) * 2 * hh + (p % hh);
-                const float a = o[j], b = o[j + hh];
-                o[j] = a + b;
-                o[j + hh] = a - b;
+        if ((d & (d - 1)) == 0) {
+            for (int hh = 1; hh < d; hh <<= 1) {
+                for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
+                    const int j = (p / hh) * 2 * hh + (p % hh);
+                    const float a = o[j], b = o[j + hh];
+                    o[j] = a + b;
+                    o[j + hh] = a - b;
+                }
+                __syncthreads();
             }
-            __syncthreads();
+        } else {   // d = 12 * 2^k: the transposed transform
+            kron_hadamard(o, d, vs.h12, true, threadIdx.x, blockDim.x, [] { __syncthreads(); });
         }
         for (int k = threadIdx.x; k < d; k += blockDim.x)
             out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = (rht_neg(vs, k) ? -o[k] : o[k]) * vs.rsqrt_d;

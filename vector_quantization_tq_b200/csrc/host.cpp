@@ -89,9 +89,11 @@ int finish_state(tq_state* st) {
     ds.rsqrt_d = (float)(1.0 / std::sqrt((double)d));
     for (int i = 0; i < ds.L; ++i) ds.c[i] = (float)st->centroids[i];
     for (int i = 0; i + 1 < ds.L; ++i) ds.t[i] = (float)st->bounds[i];
-    if (p.rot == TQ_ROT_RHT)
+    if (p.rot == TQ_ROT_RHT) {
         for (int j = 0; j < d; ++j)
             if (st->signs[j] < 0) ds.signs[j / 32] |= 1u << (j % 32);
+        if (!is_pow2(d)) paley_hadamard12_rows(ds.h12);   // d = 12 * 2^k: H_12 (x) Sylvester
+    }
 
     const size_t es = (p.mat_dtype == TQ_F32) ? 4 : 2;
     const size_t mat = (size_t)d * d * es;
@@ -162,7 +164,9 @@ int validate_params(const tq_params* p) {
     if (p->mode == TQ_MSE && (p->b < 1 || p->b > 8)) return TQ_EINVAL;
     if (p->mode == TQ_PROD && (p->b < 1 || p->b > 9)) return TQ_EINVAL;
     if (p->device < 0) return TQ_EINVAL;
-    if (p->rot == TQ_ROT_RHT && !is_pow2(p->d)) return TQ_EUNSUPPORTED;
+    // Hadamard orders: 2^k (Sylvester), or 12 * 2^k (Paley's order 12 Kronecker Sylvester)
+    if (p->rot == TQ_ROT_RHT && !is_pow2(p->d) && !(p->d % 12 == 0 && is_pow2(p->d / 12)))
+        return TQ_EUNSUPPORTED;
     if (!kernel_dim_supported(p->d)) return TQ_EUNSUPPORTED;
     return TQ_OK;
 }
@@ -613,7 +617,7 @@ int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups
     // [rows][m] then [rows][d - m], each 256-byte aligned
     const size_t b_out = ((size_t)rows * m * es + 255) & ~(size_t)255;
     void* qg = nullptr;
-    cudaError_t ce = cudaMallocAsync(&qg, b_out + (size_t)rows * r * es, s);
+    cudaError_t ce = (cudaError_t)scratch_alloc(&qg, b_out + (size_t)rows * r * es, s);
     if (ce != cudaSuccess) return cuda_status(ce);
     void* q_in = reinterpret_cast<unsigned char*>(qg) + b_out;
     int e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan, m, qg, stream);
@@ -624,7 +628,7 @@ int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups
     if (e == 0)
         e = launch_score(sp->inner->dev, q_in, qdtype, groups, nq, inner->codes, prod ? inner->qjl : nullptr,
                          inner->norms, prod ? inner->rnorms : nullptr, n, 1, scores, stream);
-    const cudaError_t fe = cudaFreeAsync(qg, s);
+    const cudaError_t fe = (cudaError_t)scratch_free(qg, s);
     return cuda_status(e ? (cudaError_t)e : fe);
 }
 

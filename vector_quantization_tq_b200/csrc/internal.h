@@ -34,6 +34,7 @@ struct DevState {
     const void* s;      // S, row-major [d][d] (prod)
     const void* sT;     // S^T, row-major [d][d] (prod)
     uint32_t signs[kMaxDim / 32];  // RHT: bit j set <=> eps_j = -1
+    uint32_t h12[12];              // RHT with d = 12 * 2^k: bit c of row a set <=> H_12[a][c] = -1
     float c[kMaxLevels];           // centroids (fp32 stored values)
     float t[kMaxLevels];           // boundaries t[0..L-2]
 };
@@ -70,6 +71,7 @@ void philox_gaussian(uint64_t seed, size_t count, double* out);
 void philox_signs(uint64_t seed, size_t count, int8_t* out);
 int haar_from_gaussian(int d, const double* g, double* pi_out);
 float bf16_round_host(float x);
+void paley_hadamard12_rows(uint32_t rows[12]);
 void set_cuda_error(int err);
 
 // ---- kernel launchers (kernels .cu files); all return a cudaError_t value ----
@@ -102,6 +104,9 @@ int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* k
                         const DevState& vi, const int32_t* vchan, const void* q, int qdtype, int H, int64_t T,
                         const SplitPlanes& kp, const SplitPlanes& vp, float scale, float* out, void* ws,
                         void* stream);
+// Stream-ordered scratch buffers from the library's per-device pool (cudaError_t values).
+int scratch_alloc(void** p, size_t bytes, void* stream);
+int scratch_free(void* p, void* stream);
 int read_device_error(int* flag);
 int take_device_error_gemm(int* flag);
 int take_device_error_search(int* flag);

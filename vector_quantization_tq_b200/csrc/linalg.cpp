@@ -143,4 +143,24 @@ float bf16_round_host(float x) {
     return r;
 }
 
+// Paley's Hadamard matrix of order 12 (q = 11, q = 3 mod 4): H = I + [[0, 1^T], [-1, Q]],
+// Q[i][j] = chi(j - i) with chi the quadratic character of GF(11). rows[a] has bit c set
+// where H[a][c] = -1.
+void paley_hadamard12_rows(uint32_t rows[12]) {
+    constexpr int q = 11;
+    int chi[q] = {0};
+    for (int a = 1; a < q; ++a) chi[a] = -1;
+    for (int x = 1; x < q; ++x) chi[(x * x) % q] = 1;
+    for (int a = 0; a < 12; ++a) {
+        rows[a] = 0;
+        for (int c = 0; c < 12; ++c) {
+            int v;
+            if (a == 0) v = (c == 0) ? 1 : 1;                       // I + border row of ones
+            else if (c == 0) v = -1;                                 // border column of -1
+            else v = chi[((c - 1) - (a - 1) + q) % q] + (a == c ? 1 : 0);
+            if (v < 0) rows[a] |= 1u << c;
+        }
+    }
+}
+
 }  // namespace tq

@@ -72,16 +72,21 @@ __device__ __forceinline__ void prep_queries_dev(const DevState& st, const void*
             qp[i] = rht_neg(st, j) ? -qs[i] : qs[i];
         }
         __syncthreads();
-        for (int h = 1; h < d; h <<= 1) {
-            for (int p = threadIdx.x; p < count * d / 2; p += blockDim.x) {
-                const int qi = p / (d / 2), pr = p % (d / 2);
-                const int j = (pr / h) * 2 * h + (pr % h);
-                float* v = qp + qi * d;
-                const float a = v[j], b = v[j + h];
-                v[j] = a + b;
-                v[j + h] = a - b;
+        if ((d & (d - 1)) == 0) {
+            for (int h = 1; h < d; h <<= 1) {
+                for (int p = threadIdx.x; p < count * d / 2; p += blockDim.x) {
+                    const int qi = p / (d / 2), pr = p % (d / 2);
+                    const int j = (pr / h) * 2 * h + (pr % h);
+                    float* v = qp + qi * d;
+                    const float a = v[j], b = v[j + h];
+                    v[j] = a + b;
+                    v[j + h] = a - b;
+                }
+                __syncthreads();
             }
-            __syncthreads();
+        } else {   // d = 12 * 2^k
+            for (int qi = 0; qi < count; ++qi)
+                kron_hadamard(qp + qi * d, d, st.h12, false, threadIdx.x, blockDim.x, [] { __syncthreads(); });
         }
         for (int i = threadIdx.x; i < count * d; i += blockDim.x) qp[i] *= st.rsqrt_d;
     } else {

@@ -271,19 +271,18 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
 
     const int64_t k_begin = (int64_t)blockIdx.x * keys_per_block;
     const int64_t k_end = (n < k_begin + keys_per_block) ? n : k_begin + keys_per_block;
-    for (int64_t key = k_begin + threadIdx.x; key < k_end; key += kThreads) {
+    // The next key's bytes are loaded before the current key's lookups (one key in flight
+    // per thread while the tables are read).
+    constexpr int ZW = PROD ? D / 32 : 1;
+    auto load_key = [&](int64_t key, uint32_t (&w)[CW], uint32_t (&z)[ZW], float& rn, float& nu) {
         const int64_t gk = grp * n + key;
-        uint32_t w[CW];
-        {
-            const uint4* src = reinterpret_cast<const uint4*>(codes + gk * (D * B / 8));
+        const uint4* src = reinterpret_cast<const uint4*>(codes + gk * (D * B / 8));
 #pragma unroll
-            for (int i = 0; i < CW / 4; ++i) {
-                const uint4 v = __ldg(src + i);
-                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-            }
+        for (int i = 0; i < CW / 4; ++i) {
+            const uint4 v = __ldg(src + i);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
         }
-        uint32_t z[PROD ? D / 32 : 1];
-        float g2 = 0.f;
+        rn = 0.f;
         if constexpr (PROD) {
             const uint4* zs = reinterpret_cast<const uint4*>(qjl + gk * (D / 8));
 #pragma unroll
@@ -291,9 +290,22 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
                 const uint4 v = __ldg(zs + i);
                 z[4 * i] = v.x; z[4 * i + 1] = v.y; z[4 * i + 2] = v.z; z[4 * i + 3] = v.w;
             }
-            g2 = __ldg(rnorms + gk) * st.qjl_scale;
+            rn = __ldg(rnorms + gk);
         }
-        const float nu = __ldg(norms + gk);
+        nu = __ldg(norms + gk);
+    };
+    uint32_t wn[CW] = {}, zn[ZW] = {};
+    float rnn = 0.f, nun = 0.f;
+    if (k_begin + threadIdx.x < k_end) load_key(k_begin + threadIdx.x, wn, zn, rnn, nun);
+    for (int64_t key = k_begin + threadIdx.x; key < k_end; key += kThreads) {
+        uint32_t w[CW], z[ZW];
+#pragma unroll
+        for (int i = 0; i < CW; ++i) w[i] = wn[i];
+#pragma unroll
+        for (int i = 0; i < ZW; ++i) z[i] = zn[i];
+        const float g2 = rnn * st.qjl_scale;
+        const float nu = nun;
+        if (key + kThreads < k_end) load_key(key + kThreads, wn, zn, rnn, nun);
         float a1[QT], a2[QT];
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) a1[qi] = a2[qi] = 0.f;
@@ -323,7 +335,7 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) {
             if (qi < nqt) {
-                float* dst = scores + (grp * nq + q0 + qi) * n + key;
+                float* dst = scores + (grp * nq + q0 + qi) * n + key;   // key of this group
                 const float v = nu * fmaf(g2, a2[qi], a1[qi]);
                 *dst = accumulate ? *dst + v : v;
             }
@@ -352,7 +364,8 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
     if (qtiles > 65535 || groups > 65535 || groups * nq > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
     // Per-query tables in a stream-ordered scratch buffer, built once per query.
     float* luts = nullptr;
-    cudaError_t ce = cudaMallocAsync(reinterpret_cast<void**>(&luts), (size_t)groups * nq * LS::SIZE * sizeof(float), s);
+    cudaError_t ce = (cudaError_t)scratch_alloc(reinterpret_cast<void**>(&luts),
+                                                (size_t)groups * nq * LS::SIZE * sizeof(float), s);
     if (ce != cudaSuccess) return (int)ce;
     ce = (cudaError_t)launch_tables<D, B, PROD>(st, q, qdtype, groups * nq, luts, s);
     if (ce == cudaSuccess) {
@@ -373,7 +386,7 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
             ce = cudaGetLastError();
         }
     }
-    cudaError_t fe = cudaFreeAsync(luts, s);
+    cudaError_t fe = (cudaError_t)scratch_free(luts, s);
     return (int)(ce != cudaSuccess ? ce : fe);
 }
 
