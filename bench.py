@@ -257,10 +257,9 @@ C5_N, C5_D, C5_NQ, C5_K = 1_000_000, 1536, 1000, 10
 
 
 def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: float):
-    """Time the dense tensor-core encode and the top-10 search on the embedding-search shape."""
+    """Time the tensor-core encode and the top-10 search on the embedding-search shape, with the
+    dense Haar Pi and with the randomized Hadamard Pi (order 1536 = 12 x 128; S stays Gaussian)."""
     d = C5_D
-    st = tq.State(d, 2, tq.PROD, tq.ROT_DENSE, tq.BF16, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0),
-                  s=synth.gaussian_matrix(d, synth.SEED_S))
     g = torch.Generator(device=dev)
     g.manual_seed(4242)
     mu = torch.randn(256, d, generator=g, device=dev)
@@ -271,39 +270,52 @@ def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: flo
     qlab = torch.randint(0, 256, (C5_NQ,), generator=g, device=dev)
     qv = mu[qlab] + 0.3 * torch.randn(C5_NQ, d, generator=g, device=dev) / d ** 0.5
     qv = (qv / qv.norm(dim=1, keepdim=True)).to(torch.bfloat16)
-    codes, qjl, norms, rnorms = st.empty_planes(C5_N, dev)
     idx = torch.empty((C5_NQ, C5_K), dtype=torch.int64, device=dev)
     vals = torch.empty((C5_NQ, C5_K), dtype=torch.float32, device=dev)
-    ws = torch.empty(tq.search_workspace(st, C5_NQ, C5_N, C5_K), dtype=torch.uint8, device=dev)
+    res = {}
+    for rot in (tq.ROT_DENSE, tq.ROT_RHT):
+        if rot == tq.ROT_DENSE:
+            st = tq.State(d, 2, tq.PROD, rot, tq.BF16, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0),
+                          s=synth.gaussian_matrix(d, synth.SEED_S))
+            enc_flops = 4.0 * d * d * C5_N          # Pi x and S r
+        else:
+            st = tq.State(d, 2, tq.PROD, rot, tq.BF16, device=dev.index, signs=synth.rht_signs(d),
+                          s=synth.gaussian_matrix(d, synth.SEED_S))
+            enc_flops = 2.0 * d * d * C5_N          # S r (the rotation is O(d log d) adds)
+        codes, qjl, norms, rnorms = st.empty_planes(C5_N, dev)
+        ws = torch.empty(tq.search_workspace(st, C5_NQ, C5_N, C5_K), dtype=torch.uint8, device=dev)
 
-    def enc():
-        tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
+        def enc():
+            tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
 
-    def srch():
-        tq.search_topk(st, qv, codes, qjl, norms, rnorms, C5_K, idx, vals, ws, stream=stream)
+        def srch():
+            tq.search_topk(st, qv, codes, qjl, norms, rnorms, C5_K, idx, vals, ws, stream=stream)
 
-    out = {}
-    for name, fn, flops in (("encode", enc, 4.0 * d * d * C5_N), ("search", srch, 4.0 * d * C5_NQ * C5_N)):
-        for _ in range(max(2, min(warmup, 3))):
-            fn()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = max(2, min(steps, 5))
-        e0.record(stream)
-        for _ in range(reps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / reps
-        tf = flops / (ms / 1e3) / 1e12
-        out[name] = {"ms": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": tflops_peak,
-                                            "unit": "TFLOP/s", "frac": tf / tflops_peak,
-                                            "algorithmic_flops_per_launch": flops}}
-    out["encode"]["mvec_s"] = C5_N / (out["encode"]["ms"] / 1e3) / 1e6
-    out["workload"] = ("embedding search: 1,000,000 x 1536 bf16 (Gaussian mixture, 256 centres), prod b=2, dense "
-                       "Pi and S bf16 (tensor cores), 1000 queries, top-10")
-    st.close()
-    return out
+        out = {}
+        for name, fn, flops in (("encode", enc, enc_flops), ("search", srch, 4.0 * d * C5_NQ * C5_N)):
+            for _ in range(max(2, min(warmup, 3))):
+                fn()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(2, min(steps, 5))
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / reps
+            tf = flops / (ms / 1e3) / 1e12
+            out[name] = {"ms": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": tflops_peak,
+                                                "unit": "TFLOP/s", "frac": tf / tflops_peak,
+                                                "algorithmic_flops_per_launch": flops}}
+        out["encode"]["mvec_s"] = C5_N / (out["encode"]["ms"] / 1e3) / 1e6
+        st.close()
+        res["dense" if rot == tq.ROT_DENSE else "rht"] = out
+    res["dense"]["workload"] = ("embedding search: 1,000,000 x 1536 bf16 (Gaussian mixture, 256 centres), prod b=2, "
+                                "dense Pi and S bf16 (tensor cores), 1000 queries, top-10")
+    res["rht"]["workload"] = ("the same with Pi = H_1536 diag(eps) / sqrt(1536), H_1536 = H_12 (x) H_128 (CUDA cores), "
+                              "S Gaussian bf16 (tensor cores)")
+    return res
 
 
 def oracle_sample(heads: int, seed: int):

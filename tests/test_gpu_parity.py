@@ -325,6 +325,25 @@ def test_tc_encoder_many_tiles(b, mode):
 # The dense tensor-core encoder (d >= 512, Pi and S bf16, bf16 input): several M tiles and
 # a ragged tail, more than one pass of its internal chunking.
 # --------------------------------------------------------------------------------------
+# Prod encode with the randomized Hadamard rotation at d >= 512 (bf16 in, bf16 S): residual
+# pass on the CUDA cores, S r and its signs on the tensor core; more than one internal chunk.
+@pytest.mark.parametrize("d,b,n", [(1536, 2, 5000), (512, 3, 70000), (2048, 2, 700)])
+def test_rht_encoder_with_tensor_core_signs(d, b, n):
+    pair = Pair(tq, d, b, tq.PROD, tq.ROT_RHT, tq.BF16)
+    bits, _ = synth.mixture_vectors(n, d, seed=63, centres=16)
+    bits[3] = 0                                             # a zero vector
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    gpu, gplanes = gpu_encode(pair, dev_bf16(bits), n)
+    tq.device_status(0)
+    bad = check_codes(pair, gpu, enc)
+    assert gpu["norms"][3] == 0.0 and gpu["rnorms"][3] == 0.0 and np.all(gpu["qjl"][3] == 255)
+    xt_o = pair.decode(enc)
+    xt_g = gpu_dequant(pair, gplanes, n)
+    ok = ~bad
+    ok[3] = False
+    assert np.max(rel_l2(xt_g[ok], xt_o[ok])) <= REL_L2
+
+
 @pytest.mark.parametrize("d,b,mode,n", [(1536, 2, 1, 5000), (512, 3, 1, 70000), (1536, 1, 0, 300)])
 def test_dense_gemm_encoder(d, b, mode, n):
     pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.BF16)
@@ -342,10 +361,13 @@ def test_dense_gemm_encoder(d, b, mode, n):
 # Tensor-core search (1-bit prod codes, dense Pi and S bf16): several query tiles and key
 # tiles with ragged tails; top-k against the oracle's estimates.
 # --------------------------------------------------------------------------------------
-@pytest.mark.parametrize("d,n,nq,k,qf32", [(512, 10000, 200, 10, False), (1536, 5000, 37, 16, True),
-                                            (512, 300, 5, 7, False)])
-def test_search_topk_tensor_core(d, n, nq, k, qf32):
-    pair = Pair(tq, d, 2, tq.PROD, tq.ROT_DENSE, tq.BF16)
+@pytest.mark.parametrize("d,n,nq,k,qf32,rot", [(512, 10000, 200, 10, False, tq.ROT_DENSE),
+                                                (1536, 5000, 37, 16, True, tq.ROT_DENSE),
+                                                (512, 300, 5, 7, False, tq.ROT_DENSE),
+                                                (1536, 5000, 37, 10, False, tq.ROT_RHT),
+                                                (1024, 3000, 9, 5, True, tq.ROT_RHT)])
+def test_search_topk_tensor_core(d, n, nq, k, qf32, rot):
+    pair = Pair(tq, d, 2, tq.PROD, rot, tq.BF16)
     bits, _ = synth.mixture_vectors(n, d, seed=61, centres=32)
     enc = pair.encode(synth.bf16_from_bits(bits))
     xt = pair.decode(enc)

@@ -12,6 +12,10 @@ int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, u
                      float* norms, float* rnorms, void* stream);
 
 bool encode_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
+bool encode_rht_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
+int launch_signs_gemm(const DevState& st, int64_t n, uint8_t* qjl, float* rnorms, void* ws, void* stream);
+int launch_encode_residual(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
+                           float* norms, uint16_t* r2out, float* rho_out, int rho_stride, void* stream);
 size_t encode_gemm_ws_bytes(int d, int64_t n);
 int launch_encode_gemm(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl,
                        float* norms, float* rnorms, void* ws, void* stream);
@@ -34,6 +38,24 @@ int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64
             rc = launch_encode_gemm(st, reinterpret_cast<const uint16_t*>(x) + c0 * ld, cn, ld,
                                     codes + c0 * st.code_bytes, qjl ? qjl + c0 * st.qjl_bytes : nullptr,
                                     norms + c0, rnorms ? rnorms + c0 : nullptr, ws, stream);
+        }
+        e = (cudaError_t)scratch_free(ws, s);
+        return rc ? rc : (int)e;
+    }
+    if (encode_rht_gemm_supported(st, dtype, n, ld)) {
+        cudaStream_t s = (cudaStream_t)stream;
+        const int64_t chunk = n < kGemmChunk ? n : kGemmChunk;
+        void* ws = nullptr;
+        cudaError_t e = (cudaError_t)scratch_alloc(&ws, encode_gemm_ws_bytes(st.d, chunk), s);
+        if (e != cudaSuccess) return (int)e;
+        int rc = 0;
+        for (int64_t c0 = 0; c0 < n && rc == 0; c0 += chunk) {
+            const int64_t cn = (n - c0 < chunk) ? n - c0 : chunk;
+            uint16_t* r2 = reinterpret_cast<uint16_t*>(ws);
+            float* rho = reinterpret_cast<float*>(r2 + (size_t)cn * 2 * st.d);
+            rc = launch_encode_residual(st, reinterpret_cast<const uint16_t*>(x) + c0 * ld, TQ_BF16, cn, ld,
+                                        codes + c0 * st.code_bytes, norms + c0, r2, rho, st.d / 256, stream);
+            if (rc == 0) rc = launch_signs_gemm(st, cn, qjl + c0 * st.qjl_bytes, rnorms + c0, ws, stream);
         }
         e = (cudaError_t)scratch_free(ws, s);
         return rc ? rc : (int)e;

@@ -319,6 +319,29 @@ bool encode_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld)
            st.d % 256 == 0 && st.b_mse >= 1 && st.b_mse <= 4 && n > 0 && n < ((int64_t)1 << 31) && ld >= st.d;
 }
 
+// Prod encode with the randomized Hadamard rotation at d >= 512 (bf16 S and input): the
+// rotation, codes and residual run on the CUDA cores (general encoder writing [r_hi | r_lo]
+// and ||r||^2), S r and its signs on the tensor core (the kSigns pass below).
+bool encode_rht_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld) {
+    return st.rot == TQ_ROT_RHT && st.mode == TQ_PROD && st.mat_dtype == TQ_BF16 && dtype == TQ_BF16 &&
+           st.d >= 512 && st.d % 256 == 0 && st.b_mse <= 4 && n > 0 && n < ((int64_t)1 << 31) && ld >= st.d;
+}
+
+// Signs of S r and ||r|| from the residual workspace (r2, rho_part) of n vectors.
+int launch_signs_gemm(const DevState& st, int64_t n, uint8_t* qjl, float* rnorms, void* ws, void* stream) {
+    const int d = st.d;
+    GemmParams p = {};
+    p.M = (int)n;
+    p.N = d;
+    p.K = 2 * d;
+    p.b_kwrap = d;
+    p.rho_part = reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(ws) + (size_t)n * 2 * d);
+    p.n_tiles = d / 256;
+    p.qjl = qjl;
+    p.rnorms = rnorms;
+    return run_gemm<256, kSigns>(ws, 2 * d, st.s, d, p, (cudaStream_t)stream);
+}
+
 // Dense tensor-core encode: ||x||, y = Pi x / ||x|| (codes + residual), then signs of S r.
 // Workspace: R = [r_hi | r_lo] bf16 [n][2d] and partial ||r||^2 [n][d/256].
 size_t encode_gemm_ws_bytes(int d, int64_t n) {

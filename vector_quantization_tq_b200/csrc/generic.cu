@@ -88,7 +88,8 @@ template <int E, int NT>
 __global__ void __launch_bounds__(NT == 32 ? 256 : NT)
 encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t n, int64_t ld,
               const int32_t* __restrict__ chan, int64_t ostride, uint8_t* __restrict__ codes,
-              uint8_t* __restrict__ qjl, float* __restrict__ norms, float* __restrict__ rnorms) {
+              uint8_t* __restrict__ qjl, float* __restrict__ norms, float* __restrict__ rnorms,
+              uint16_t* __restrict__ r2out, float* __restrict__ rho_out, int rho_stride) {
     constexpr int D = NT * E;
     constexpr int GPB = (NT == 32) ? 8 : 1;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -161,7 +162,24 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
             r[e] = (nu > 0.f) ? (y[e] - (st.b_mse > 0 ? ctab[c] : 0.f)) : 0.f;
             rr = fmaf(r[e], r[e], rr);
         }
-        if (prod) {
+        if (r2out != nullptr) {
+            // prod with S r on the tensor core: the residual as [r_hi | r_lo] bf16 rows
+            // (r_lo = bf16(r - r_hi)) and ||r||^2 for the signs pass
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = tid * E + e;
+                const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(r[e]));
+                const float lo = r[e] - __uint_as_float((uint32_t)hb << 16);
+                r2out[vec * 2 * D + j] = hb;
+                r2out[vec * 2 * D + D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+            }
+            const float rsum = group_sum<NT>(rr, red);
+            if (tid == 0) {
+                norms[vec * ostride] = nu;
+                rho_out[vec * rho_stride] = rsum;
+                for (int t = 1; t < rho_stride; ++t) rho_out[vec * rho_stride + t] = 0.f;
+            }
+        } else if (prod) {
             const float rho = sqrtf(group_sum<NT>(rr, red));
 #pragma unroll
             for (int e = 0; e < E; ++e) vbuf[tid * E + e] = r[e];
@@ -191,7 +209,7 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
                 if (lane == 0) out[w] = word;
             }
         }
-        if (prod) {
+        if (prod && r2out == nullptr) {
             uint32_t* out = reinterpret_cast<uint32_t*>(qjl + vec * ostride * st.qjl_bytes);
             for (int w = warp_in_group; w < D / 32; w += WPG) {
                 const uint32_t word = __ballot_sync(0xffffffffu, zbuf[32 * w + lane]);
@@ -759,7 +777,8 @@ int num_sms() {
 
 template <int E, int NT>
 int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
-                    int64_t ostride, uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, cudaStream_t s) {
+                    int64_t ostride, uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, uint16_t* r2out,
+                    float* rho_out, int rho_stride, cudaStream_t s) {
     constexpr int GPB = (NT == 32) ? 8 : 1;
     const int threads = NT * GPB;
     const size_t smem = (2 * kMaxLevels + 8) * sizeof(float) + GPB * (NT * E) * (sizeof(float) + 2);
@@ -767,7 +786,8 @@ int launch_encode_t(const DevState& st, const void* x, int dtype, int64_t n, int
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int64_t blocks_needed = (n + GPB - 1) / GPB;
     const int blocks = (int)std::min<int64_t>(blocks_needed, (int64_t)num_sms() * 16);
-    kern<<<blocks, threads, smem, s>>>(st, x, dtype, n, ld, chan, ostride, codes, qjl, norms, rnorms);
+    kern<<<blocks, threads, smem, s>>>(st, x, dtype, n, ld, chan, ostride, codes, qjl, norms, rnorms, r2out,
+                                       rho_out, rho_stride);
     return (int)cudaGetLastError();
 }
 
@@ -814,7 +834,19 @@ int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t 
     cudaStream_t s = (cudaStream_t)stream;
     return with_layout(st.d, [&](auto e, auto nt) {
         return launch_encode_t<decltype(e)::value, decltype(nt)::value>(st, x, dtype, n, ld, chan, ostride, codes,
-                                                                         qjl, norms, rnorms, s);
+                                                                         qjl, norms, rnorms, nullptr, nullptr, 0, s);
+    });
+}
+
+// Codes, norms, the residual operand [r_hi | r_lo] and ||r||^2 (first of rho_stride slots) of
+// a prod encode whose S r runs on the tensor core.
+int launch_encode_residual(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
+                           float* norms, uint16_t* r2out, float* rho_out, int rho_stride, void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    return with_layout(st.d, [&](auto e, auto nt) {
+        return launch_encode_t<decltype(e)::value, decltype(nt)::value>(st, x, dtype, n, ld, nullptr, 1, codes,
+                                                                         nullptr, norms, nullptr, r2out, rho_out,
+                                                                         rho_stride, s);
     });
 }
 

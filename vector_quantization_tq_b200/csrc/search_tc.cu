@@ -357,8 +357,40 @@ int launch_gemm_f32(const void* A, int64_t lda, const void* B, int64_t ldb, int 
 int launch_search_merge(int64_t nq, int64_t ncand, int k, const float* cand_v, const int64_t* cand_i, int64_t* idx,
                         float* vals, void* stream);
 
+namespace {
+// q' = Pi q for the randomized Hadamard rotation: one block per query (signs, the Sylvester
+// or Kronecker transform in shared memory, 1/sqrt(d)).
+__global__ void __launch_bounds__(256)
+rht_rows_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ qp) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float* v = reinterpret_cast<float*>(smem_raw);
+    const int d = st.d;
+    const int64_t r = blockIdx.x;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        const float x = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + r * d + j)
+                                           : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + r * d + j));
+        v[j] = rht_neg(st, j) ? -x : x;
+    }
+    __syncthreads();
+    if ((d & (d - 1)) == 0) {
+        for (int h = 1; h < d; h <<= 1) {
+            for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
+                const int j = (p / h) * 2 * h + (p % h);
+                const float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+            __syncthreads();
+        }
+    } else {
+        kron_hadamard(v, d, st.h12, false, threadIdx.x, blockDim.x, [] { __syncthreads(); });
+    }
+    for (int j = threadIdx.x; j < d; j += blockDim.x) qp[r * d + j] = v[j] * st.rsqrt_d;
+}
+}  // namespace
+
 bool search_tc_supported(const DevState& st, int qdtype, int k) {
-    return k <= kTopMax && st.mode == TQ_PROD && st.b_mse == 1 && st.rot == TQ_ROT_DENSE && st.mat_dtype == TQ_BF16 &&
+    return k <= kTopMax && st.mode == TQ_PROD && st.b_mse == 1 && st.mat_dtype == TQ_BF16 &&
            st.d >= 512 && st.d % 256 == 0 && k <= kTopMax && (qdtype == TQ_BF16 || qdtype == TQ_F32);
 }
 
@@ -408,7 +440,10 @@ int launch_search_tc(const DevState& st, const void* q, int qdtype, int64_t nq, 
     const unsigned blocks = (unsigned)((nq * d + threads - 1) / threads);
     int e;
     // q' = Pi q
-    if (qdtype == TQ_BF16) {
+    if (st.rot == TQ_ROT_RHT) {
+        rht_rows_kernel<<<(unsigned)nq, 256, d * sizeof(float), s>>>(st, q, qdtype, qp);
+        e = (int)cudaGetLastError();
+    } else if (qdtype == TQ_BF16) {
         e = launch_gemm_f32(q, d, st.pi, d, (int)nq, d, d, d, qp, d, stream);
     } else {
         split_rows_kernel<<<blocks, threads, 0, s>>>(reinterpret_cast<const float*>(q), nq, d, split, 1);
