@@ -251,6 +251,54 @@ def measure_split(tq, torch, x, q, heads, dev, stream, steps: int, warmup: int, 
     return res
 
 
+# Prefix coding of b = 4 MSE codes (the V cache's width in the decode shape): 1,048,576 unit
+# vectors, d = 128, RHT state; encode (lengths, scan, bit stream) and decode timed apart.
+ENT_N = 1 << 20
+
+
+def measure_entropy(tq, torch, dev, stream, steps: int, warmup: int):
+    st = tq.State(D, 4, tq.MSE, tq.ROT_RHT, tq.F32, device=dev.index, signs=synth.rht_signs(D))
+    g = torch.Generator(device=dev)
+    g.manual_seed(777)
+    x = torch.randn(ENT_N, D, generator=g, device=dev)
+    x /= x.norm(dim=1, keepdim=True)
+    codes, _, norms, _ = st.empty_planes(ENT_N, dev)
+    tq.quantize_mse(st, x, codes, norms, stream=stream)
+    offsets = torch.empty(ENT_N + 1, dtype=torch.int64, device=dev)
+    sbuf = torch.empty(tq.entropy_max_bytes(st, ENT_N), dtype=torch.uint8, device=dev)
+    ws = torch.empty(tq.entropy_workspace(st, ENT_N), dtype=torch.uint8, device=dev)
+    back = torch.empty_like(codes)
+
+    def enc():
+        tq.entropy_encode(st, codes, offsets, sbuf, ws, cuda_stream=stream)
+
+    def dec():
+        tq.entropy_decode(st, sbuf, offsets, back, cuda_stream=stream)
+
+    out = {}
+    for name, fn in (("encode", enc), ("decode", dec)):
+        for _ in range(max(2, min(warmup, 3))):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(2, min(steps, 10))
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        out[name] = e0.elapsed_time(e1) / reps
+    total_bits = int(offsets[-1].item())
+    _, _, mean = tq.entropy_table(st)
+    ok = bool(torch.equal(back, codes))
+    st.close()
+    return {"workload": "prefix code of b=4 MSE codes: 1,048,576 unit vectors x 128 (Huffman of the Lemma-1 index "
+                        "law, canonical)", "ms": out,
+            "encode_mvec_s": ENT_N / (out["encode"] / 1e3) / 1e6, "decode_mvec_s": ENT_N / (out["decode"] / 1e3) / 1e6,
+            "bits_per_coordinate": total_bits / (ENT_N * D), "law_mean_bits": mean,
+            "saving_vs_fixed": 1 - total_bits / (ENT_N * D * 4), "round_trip_exact": ok}
+
+
 # Embedding search (1,000,000 vectors, d = 1536, prod b = 2, dense Pi and S bf16, 1000 queries):
 # algorithmic flops: encode 4 d^2 per vector (Pi x and S r); search 4 d per (query, key).
 C5_N, C5_D, C5_NQ, C5_K = 1_000_000, 1536, 1000, 10
@@ -382,6 +430,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
     ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
     ap.add_argument("--no-split", action="store_true", help="skip the outlier-channel split measurement")
+    ap.add_argument("--no-entropy", action="store_true", help="skip the prefix-coding measurement")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -507,6 +556,9 @@ def main():
     split = None
     if not args.no_split:
         split = measure_split(tq, torch, x, q, heads, dev, stream, args.steps, args.warmup, peak)
+    ent = None
+    if not args.no_entropy:
+        ent = measure_entropy(tq, torch, dev, stream, args.steps, args.warmup)
     c5 = None
     if not args.no_c5:
         c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak())
@@ -543,6 +595,7 @@ def main():
         "decode_attention": decode,
         "embedding_search": c5,
         "outlier_split": split,
+        "prefix_code": ent,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -288,6 +288,41 @@ int tq_attend_append_decode(const tq_state* ks, const tq_state* vs, const void* 
                             uint8_t* kcodes, uint8_t* kqjl, float* knorms, float* krnorms, uint8_t* vcodes,
                             float* vnorms, float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- prefix coding of the indices -----------------------------------------------------
+ * TurboQuant review (Jump2Paper), limitations: an optimal prefix code on the b = 4 indices
+ * averages about 3.8 bits. The code is Huffman's code of the one-coordinate index law under
+ * Lemma 1 (cell probabilities of the state's Lloyd-Max boundaries), fixed per state: ties
+ * in the merges go to the lower node id (leaves 0..L-1, merged nodes L, L+1, ... in creation
+ * order); codewords are canonical. Stream layout: each vector's codes in coordinate order,
+ * each codeword first bit (most significant) first, vectors back to back, bit j of the
+ * stream = bit j % 8 of byte j / 8; offsets[k] = first bit of vector k, offsets[n] = total.
+ */
+
+/* Codeword lengths and canonical codewords (host arrays of 2^b_mse), and the mean length in
+   bits per coordinate under the index law. Any output may be NULL. */
+int tq_entropy_table(const tq_state* st, int* h_lengths, uint32_t* h_words, double* h_mean_bits);
+
+/* Stream capacity in bytes that tq_entropy_encode requires for n vectors (the longest
+   codeword for every coordinate, in whole 32-bit words, plus 16 bytes). */
+int tq_entropy_max_bytes(const tq_state* st, int64_t n, size_t* bytes);
+
+/* Workspace bytes that tq_entropy_encode needs for n vectors. */
+int tq_entropy_workspace(const tq_state* st, int64_t n, size_t* bytes);
+
+/*
+ * Encode the packed codes planes [n][code_bytes] (16-byte aligned) into `stream` (device,
+ * 4-byte aligned, `capacity` >= tq_entropy_max_bytes; zeroed here first) and offsets
+ * (device uint64 [n + 1], 8-byte aligned). workspace: >= tq_entropy_workspace bytes,
+ * 256-byte aligned. TQ_ENOMEM if capacity or workspace is too small.
+ */
+int tq_entropy_encode(const tq_state* st, const uint8_t* codes, int64_t n, uint64_t* offsets, uint8_t* stream,
+                      size_t capacity, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Decode n vectors of `stream` (offsets as written by tq_entropy_encode) back into packed
+   codes planes [n][code_bytes] (16-byte aligned). */
+int tq_entropy_decode(const tq_state* st, const uint8_t* stream, const uint64_t* offsets, int64_t n, uint8_t* codes,
+                      void* cuda_stream);
+
 /* ---- outlier-channel split ------------------------------------------------------------
  * TurboQuant review (Jump2Paper), experiment settings ("KV bit settings": 2.5 and 3.5 bits
  * with outlier and non-outlier channels separated; "outlier handling": 32 of 128 channels at

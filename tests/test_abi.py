@@ -138,3 +138,20 @@ def test_null_state_calls_are_rejected():
     buf = ctypes.create_string_buffer(b"XXXX" + bytes(200))
     h = ctypes.c_void_p()
     assert lib.tq_state_import(buf, 204, 0, ctypes.byref(h)) == 1
+
+
+def test_prefix_code_table_matches_oracle_without_gpu():
+    # the library's Huffman table (its own cell law, merges and canonical codewords) equals
+    # the oracle's for several (d, b); MSE states with the Hadamard rotation need no device
+    from oracle import codebook as CB
+    from oracle import entropy as EN
+    for d, b in ((128, 4), (128, 2), (256, 3), (32, 4)):
+        st = tq.State(d, b, tq.MSE, tq.ROT_RHT, tq.F32, signs=synth.rht_signs(d))
+        ln, w, mean = tq.entropy_table(st)
+        st.close()
+        _, t, _, _ = CB.lloyd_max(d, b)
+        p = EN.index_probabilities(d, t)
+        oln = EN.huffman_lengths(p)
+        np.testing.assert_array_equal(ln, oln)
+        np.testing.assert_array_equal(w, EN.canonical_codewords(oln))
+        assert abs(mean - float(np.sum(p * oln))) < 1e-9

@@ -99,6 +99,11 @@ _SIGS = {
                                       _P, _P, _SZ, _P]),
     "tq_attend_append_decode": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _I, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_float, _P, _P, _SZ, _P]),
+    "tq_entropy_table": (_I, [_P, _P, _P, _DP]),
+    "tq_entropy_max_bytes": (_I, [_P, _I64, ctypes.POINTER(_SZ)]),
+    "tq_entropy_workspace": (_I, [_P, _I64, ctypes.POINTER(_SZ)]),
+    "tq_entropy_encode": (_I, [_P, _P, _I64, _P, _P, _SZ, _P, _SZ, _P]),
+    "tq_entropy_decode": (_I, [_P, _P, _P, _I64, _P, _P]),
     "tq_split_create": (_I, [_P, _P, _P, _I, ctypes.POINTER(_P)]),
     "tq_split_destroy": (None, [_P]),
     "tq_split_quantize": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _P]),
@@ -483,3 +488,40 @@ def split_attend_decode(ks: Split, vs: Split, q, k_planes, v_planes, scale: floa
     _check(_lib.tq_split_attend_decode(ks.handle, vs.handle, _ptr(q), _dtype_code(q), H, T, ctypes.byref(ko),
                                        ctypes.byref(ki), ctypes.byref(vo), ctypes.byref(vi), float(scale), _ptr(out),
                                        _ptr(workspace), ws_bytes, _stream(stream)), "tq_split_attend_decode")
+
+
+# ---- prefix coding of the indices ---------------------------------------------------------
+
+def entropy_table(st: State):
+    """(lengths[2^b_mse], canonical codewords[2^b_mse], mean bits per coordinate)."""
+    L = 1 << st.b_mse
+    ln = np.zeros(L, dtype=np.int32)
+    w = np.zeros(L, dtype=np.uint32)
+    mean = ctypes.c_double()
+    _check(_lib.tq_entropy_table(st.handle, ln.ctypes.data, w.ctypes.data, ctypes.byref(mean)), "tq_entropy_table")
+    return ln, w, mean.value
+
+
+def entropy_max_bytes(st: State, n: int) -> int:
+    b = _SZ()
+    _check(_lib.tq_entropy_max_bytes(st.handle, n, ctypes.byref(b)), "tq_entropy_max_bytes")
+    return b.value
+
+
+def entropy_workspace(st: State, n: int) -> int:
+    b = _SZ()
+    _check(_lib.tq_entropy_workspace(st.handle, n, ctypes.byref(b)), "tq_entropy_workspace")
+    return b.value
+
+
+def entropy_encode(st: State, codes, offsets, stream, workspace, n=None, cuda_stream=None):
+    """codes [n][code_bytes] -> offsets [n + 1] (int64) and the prefix-coded stream (uint8)."""
+    n = codes.shape[0] if n is None else n
+    _check(_lib.tq_entropy_encode(st.handle, _ptr(codes), n, _ptr(offsets), _ptr(stream), stream.numel(),
+                                  _ptr(workspace), workspace.numel(), _stream(cuda_stream)), "tq_entropy_encode")
+
+
+def entropy_decode(st: State, stream, offsets, codes, n=None, cuda_stream=None):
+    n = codes.shape[0] if n is None else n
+    _check(_lib.tq_entropy_decode(st.handle, _ptr(stream), _ptr(offsets), n, _ptr(codes), _stream(cuda_stream)),
+           "tq_entropy_decode")

@@ -209,4 +209,19 @@ int build_codebook(int d, int b, double* c_out, double* t_out, double* dmse_out)
     return TQ_OK;
 }
 
+// Probabilities of the L cells of the boundaries t[0..L-2] under f_X (Lemma 1), computed for
+// the lower half and mirrored (the law is even).
+void index_law(int d, int L, const double* t, double* p) {
+    Law law(d);
+    for (int i = 0; i < L / 2; ++i) {
+        double a = (i == 0) ? -1.0 : t[i - 1];
+        double b = t[i];
+        double m0, m2;
+        law.moments02(a, b, &m0, &m2);
+        p[i] = m0;
+        p[L - 1 - i] = m0;
+    }
+    if (L == 1) p[0] = 1.0;
+}
+
 }  // namespace tq

@@ -507,6 +507,69 @@ int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int6
                                                  norms, prod ? rnorms : nullptr, n, 0, scores, stream));
 }
 
+// ---- prefix coding of the indices -------------------------------------------------------
+
+int tq_entropy_table(const tq_state* st, int* h_lengths, uint32_t* h_words, double* h_mean_bits) {
+    if (!st || st->b_mse < 1) return TQ_EINVAL;
+    EntropyTable tab;
+    int rc = build_prefix_code(st, &tab);
+    if (rc != TQ_OK) return rc;
+    for (int i = 0; i < tab.L; ++i) {
+        if (h_lengths) h_lengths[i] = tab.len[i];
+        if (h_words) h_words[i] = tab.word[i];
+    }
+    if (h_mean_bits) *h_mean_bits = tab.mean_bits;
+    return TQ_OK;
+}
+
+int tq_entropy_max_bytes(const tq_state* st, int64_t n, size_t* bytes) {
+    if (!st || st->b_mse < 1 || n < 0 || !bytes) return TQ_EINVAL;
+    EntropyTable tab;
+    int rc = build_prefix_code(st, &tab);
+    if (rc != TQ_OK) return rc;
+    const uint64_t bits = (uint64_t)n * st->p.d * tab.maxlen;
+    *bytes = (size_t)((bits + 31) / 32) * 4 + 16;
+    return TQ_OK;
+}
+
+int tq_entropy_workspace(const tq_state* st, int64_t n, size_t* bytes) {
+    if (!st || n < 0 || !bytes) return TQ_EINVAL;
+    *bytes = entropy_ws_bytes(n);
+    return TQ_OK;
+}
+
+int tq_entropy_encode(const tq_state* st, const uint8_t* codes, int64_t n, uint64_t* offsets, uint8_t* stream,
+                      size_t capacity, void* workspace, size_t ws_bytes, void* cuda_stream) {
+    if (!st || st->b_mse < 1 || n < 0) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    if (!codes || !offsets || !stream || !workspace || !aligned16(codes) || ((uintptr_t)offsets & 7u) ||
+        ((uintptr_t)stream & 3u) || ((uintptr_t)workspace & 255u))
+        return TQ_EINVAL;
+    EntropyTable tab;
+    int rc = build_prefix_code(st, &tab);
+    if (rc != TQ_OK) return rc;
+    const uint64_t bits = (uint64_t)n * st->p.d * tab.maxlen;
+    if (capacity < (size_t)((bits + 31) / 32) * 4 + 16 || ws_bytes < entropy_ws_bytes(n)) return TQ_ENOMEM;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_entropy_encode(st->dev, tab, codes, n, offsets, stream, capacity,
+                                                          workspace, cuda_stream));
+}
+
+int tq_entropy_decode(const tq_state* st, const uint8_t* stream, const uint64_t* offsets, int64_t n, uint8_t* codes,
+                      void* cuda_stream) {
+    if (!st || st->b_mse < 1 || n < 0) return TQ_EINVAL;
+    if (n == 0) return TQ_OK;
+    if (!codes || !offsets || !stream || !aligned16(codes) || ((uintptr_t)offsets & 7u) || ((uintptr_t)stream & 3u))
+        return TQ_EINVAL;
+    EntropyTable tab;
+    int rc = build_prefix_code(st, &tab);
+    if (rc != TQ_OK) return rc;
+    DeviceGuard g(st->p.device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_entropy_decode(st->dev, tab, stream, offsets, n, codes, cuda_stream));
+}
+
 // ---- outlier-channel split -----------------------------------------------------------
 
 namespace {

@@ -54,6 +54,29 @@ struct tq_state {
     tq::DevState dev;                // kernel view
 };
 
+// Canonical prefix code of the codebook indices (see entropy.cpp).
+namespace tq {
+constexpr int kMaxCodeLen = 32;
+struct EntropyTable {
+    int L;
+    int maxlen;
+    double mean_bits;
+    uint8_t len[kMaxLevels];           // codeword length of each index
+    uint32_t word[kMaxLevels];         // canonical codeword (first bit = most significant)
+    uint32_t rword[kMaxLevels];        // the codeword bit-reversed (first bit = bit 0)
+    uint16_t sym[kMaxLevels];          // indices in canonical (length, index) order
+    uint32_t first[kMaxCodeLen + 2];   // first codeword of each length
+    uint16_t count[kMaxCodeLen + 2];   // number of codewords of each length
+    uint16_t start[kMaxCodeLen + 2];   // position in sym of the first codeword of each length
+};
+int build_prefix_code(const tq_state* st, EntropyTable* tab);
+size_t entropy_ws_bytes(int64_t n);
+int launch_entropy_encode(const DevState& st, const EntropyTable& tab, const uint8_t* codes, int64_t n,
+                          uint64_t* offsets, uint8_t* stream, size_t capacity, void* ws, void* cuda_stream);
+int launch_entropy_decode(const DevState& st, const EntropyTable& tab, const uint8_t* stream, const uint64_t* offsets,
+                          int64_t n, uint8_t* codes, void* cuda_stream);
+}  // namespace tq
+
 struct tq_split {
     const tq_state* outer;           // channels `chan_outer`, dimension m
     const tq_state* inner;           // the other channels, ascending, dimension d - m
