@@ -109,6 +109,15 @@ int tq_last_cuda_error(void);
  */
 int tq_device_status(int device);
 
+/*
+ * Exercise the failure path of the bounded waits without a fault: on `device` (default
+ * stream) a kernel waits on an mbarrier phase that nothing completes, gives up after
+ * limit_us (1 .. 1e6 microseconds) and records the kernel error word. The next
+ * tq_device_status(device) then returns TQ_EDEVICE (and clears the word); the context stays
+ * usable. Returns the launch status.
+ */
+int tq_check_error_path(int device, uint32_t limit_us);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int tq_version(void);
 

@@ -73,6 +73,7 @@ _SIGS = {
     "tq_last_cuda_error": (_I, []),
     "tq_version": (_I, []),
     "tq_device_status": (_I, [_I]),
+    "tq_check_error_path": (_I, [_I, ctypes.c_uint32]),
     "tq_build_codebook": (_I, [_I, _I, _DP, _DP, _DP]),
     "tq_draw_gaussian": (_I, [ctypes.c_uint64, _SZ, _DP]),
     "tq_draw_signs": (_I, [ctypes.c_uint64, _SZ, _P]),

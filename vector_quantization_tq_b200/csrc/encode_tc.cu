@@ -1348,6 +1348,25 @@ int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, u
     }
 }
 
+namespace {
+// A wait that can only run out: one thread waits on the first phase of an mbarrier nothing
+// arrives on, gives up after limit_ns and records the error word, as every bounded wait of
+// the library does on a timeout.
+__global__ void expired_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+        if (!ptx::mbar_wait(&bar, 0u, limit_ns)) atomicExch(&g_tq_device_error, 1);
+    }
+}
+}  // namespace
+
+int launch_expired_wait(uint64_t limit_ns, void* stream) {
+    expired_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+    return (int)cudaGetLastError();
+}
+
 // Reads and clears the error words of all kernels with bounded waits (one word per
 // translation unit: the library is built without relocatable device code).
 int read_device_error(int* flag) {

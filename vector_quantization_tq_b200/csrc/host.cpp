@@ -206,6 +206,13 @@ int tq_device_status(int device) {
     return flag ? TQ_EDEVICE : TQ_OK;
 }
 
+int tq_check_error_path(int device, uint32_t limit_us) {
+    if (device < 0 || limit_us == 0 || limit_us > 1000000) return TQ_EINVAL;
+    DeviceGuard g(device);
+    if (!g.ok) return cuda_status(cudaGetLastError());
+    return cuda_status((cudaError_t)launch_expired_wait((uint64_t)limit_us * 1000ull, nullptr));
+}
+
 int tq_build_codebook(int d, int b, double* h_c, double* h_t, double* h_dmse) {
     if (d < 2 || b < 1 || b > 8) return TQ_EINVAL;
     return build_codebook(d, b, h_c, h_t, h_dmse);

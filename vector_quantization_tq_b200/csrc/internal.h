@@ -130,6 +130,7 @@ int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* k
 // Stream-ordered scratch buffers from the library's per-device pool (cudaError_t values).
 int scratch_alloc(void** p, size_t bytes, void* stream);
 int scratch_free(void* p, void* stream);
+int launch_expired_wait(uint64_t limit_ns, void* stream);
 int read_device_error(int* flag);
 int take_device_error_gemm(int* flag);
 int take_device_error_search(int* flag);
