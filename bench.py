@@ -200,7 +200,8 @@ def measure_decode(tq, torch, dev, stream, steps: int, warmup: int, peak: float)
 
 
 # Outlier-channel split of the same KV key batch: the 32 channels of largest mean square
-# (over the first 32,768 keys) at prod b=3, the other 96 at prod b=2 (dense Pi, fp32 state).
+# (over the first 32,768 keys) at prod b=3, the other 96 at prod b=2; each group rotated by
+# its randomized Hadamard transform (orders 32 and 96 = 12 x 8), S stored bf16.
 # Per vector: 256 B in; out 8 + 4 + 8 B (outer codes, QJL, norms) + 12 + 12 + 8 B (inner).
 SPLIT_M, SPLIT_BO, SPLIT_BR = 32, 3, 2
 SPLIT_BYTES_PER_VEC = 2 * D + (SPLIT_M * (SPLIT_BO - 1) // 8 + SPLIT_M // 8 + 8) + \
@@ -212,8 +213,8 @@ def measure_split(tq, torch, x, q, heads, dev, stream, steps: int, warmup: int, 
     nvec = x.shape[0]
     ms = torch.mean(x[:TOKENS].float() ** 2, dim=0)
     ch = np.sort(torch.argsort(ms, descending=True)[:SPLIT_M].cpu().numpy())
-    so = tq.State(SPLIT_M, SPLIT_BO, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, seed_pi=20, seed_s=21)
-    sr = tq.State(D - SPLIT_M, SPLIT_BR, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, seed_pi=22, seed_s=23)
+    so = tq.State(SPLIT_M, SPLIT_BO, tq.PROD, tq.ROT_RHT, tq.BF16, device=dev.index, seed_pi=20, seed_s=21)
+    sr = tq.State(D - SPLIT_M, SPLIT_BR, tq.PROD, tq.ROT_RHT, tq.BF16, device=dev.index, seed_pi=22, seed_s=23)
     sp = tq.Split(so, sr, ch)
     po, pr = sp.empty_planes(nvec, dev)
     scores = torch.empty((heads, 1, TOKENS), dtype=torch.float32, device=dev)
@@ -238,7 +239,7 @@ def measure_split(tq, torch, x, q, heads, dev, stream, steps: int, warmup: int, 
         out[name] = e0.elapsed_time(e1) / steps
     gbs = SPLIT_BYTES_PER_VEC * nvec / (out["encode"] / 1e3) / 1e9
     res = {"workload": f"outlier-channel split of the KV key batch: {SPLIT_M} channels at prod b={SPLIT_BO}, "
-                       f"{D - SPLIT_M} at prod b={SPLIT_BR} (dense Pi, fp32 state), "
+                       f"{D - SPLIT_M} at prod b={SPLIT_BR} (Hadamard Pi per group, S bf16), "
                        f"{SPLIT_M * SPLIT_BO + (D - SPLIT_M) * SPLIT_BR} bits per vector of codes",
            "effective_bits": (SPLIT_M * SPLIT_BO + (D - SPLIT_M) * SPLIT_BR) / D,
            "ms": out, "quantize_mvec_s": nvec / (out["encode"] / 1e3) / 1e6,

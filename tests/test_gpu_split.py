@@ -17,9 +17,11 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 tq = pytest.importorskip("vector_quantization_tq_b200")
 
-# (d, outlier channels m, outlier bits, other bits, mode): the stated 32@3 + 96@2 split,
+# (d, outlier channels m, outlier bits, other bits, mode, rotation, matrix dtype): the stated
+# 32@3 + 96@2 split (dense and with the groups' Hadamard transforms, orders 32 and 12 x 8),
 # a 2.5-bit split, an MSE split, and a wider head.
-CASES = [(128, 32, 3, 2, 1), (128, 32, 4, 2, 1), (128, 32, 3, 2, 0), (256, 64, 4, 3, 1)]
+CASES = [(128, 32, 3, 2, 1, 0, 0), (128, 32, 3, 2, 1, 1, 1), (128, 32, 4, 2, 1, 0, 0), (128, 32, 3, 2, 0, 0, 0),
+         (256, 64, 4, 3, 1, 0, 0)]
 
 
 def _host(planes):
@@ -30,14 +32,14 @@ def _host(planes):
     return out
 
 
-@pytest.mark.parametrize("d,m,bo,br,mode", CASES)
+@pytest.mark.parametrize("d,m,bo,br,mode,rot,md", CASES)
 @pytest.mark.parametrize("n", [3001])
-def test_split_encode_dequant_score(d, m, bo, br, mode, n):
+def test_split_encode_dequant_score(d, m, bo, br, mode, rot, md, n):
     bits = synth.kv_prefill_batch(1, n, d, seed=51)[0]
     x = synth.bf16_from_bits(bits).astype(np.float64)
     ch = OM.outlier_channels(x, m)
-    po = Pair(tq, m, bo, mode, tq.ROT_DENSE, tq.F32, seed_pi=20, seed_s=21)
-    pr = Pair(tq, d - m, br, mode, tq.ROT_DENSE, tq.F32, seed_pi=22, seed_s=23)
+    po = Pair(tq, m, bo, mode, rot, md, seed_pi=20, seed_s=21)
+    pr = Pair(tq, d - m, br, mode, rot, md, seed_pi=22, seed_s=23)
     sp = tq.Split(po.st, pr.st, ch)
     x_dev = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
     pl_o, pl_r = sp.empty_planes(n)
