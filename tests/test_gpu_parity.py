@@ -305,8 +305,8 @@ def test_tc_encoder(b, mode, n, pad):
     assert np.max(rel_l2(xt_g[~bad], xt_o[~bad]), initial=0) <= REL_L2
 
 
-# The pipelined encoder (b_mse 1 and 2) with several tiles per CTA: more tiles than the TMA
-# ring has stages on every SM, both residual buffers in use, and a ragged last tile.
+# The two-team encoder (b_mse 1 and 2) with several tiles per CTA: each team refills its two
+# TMA stages and reuses its TMEM columns across tiles, and the last tile is ragged.
 @pytest.mark.parametrize("b,mode", [(2, 1), (3, 1), (1, 0), (2, 0)])
 def test_tc_encoder_many_tiles(b, mode):
     d, n = 128, 148 * 128 * 5 + 77
