@@ -22,6 +22,11 @@ tq = pytest.importorskip("vector_quantization_tq_b200")
 # a 2.5-bit split, an MSE split, and a wider head.
 CASES = [(128, 32, 3, 2, 1, 0, 0), (128, 32, 3, 2, 1, 1, 1), (128, 32, 4, 2, 1, 0, 0), (128, 32, 3, 2, 0, 0, 0),
          (256, 64, 4, 3, 1, 0, 0)]
+# Splits of 128 bf16 channels whose groups are Hadamard-rotated at 1 or 2 code bits run on the
+# tensor-core encoder: the 32@3 + 96@2 split over several tiles per SM, a 64 + 64 MSE split,
+# and a 96-channel outer group.
+TC_CASES = [(128, 32, 3, 2, 1, 1, 1, 148 * 128 * 3 + 5), (128, 64, 2, 1, 0, 1, 1, 20000),
+            (128, 96, 2, 3, 1, 1, 1, 9001)]
 
 
 def _host(planes):
@@ -35,6 +40,15 @@ def _host(planes):
 @pytest.mark.parametrize("d,m,bo,br,mode,rot,md", CASES)
 @pytest.mark.parametrize("n", [3001])
 def test_split_encode_dequant_score(d, m, bo, br, mode, rot, md, n):
+    _split_case(d, m, bo, br, mode, rot, md, n)
+
+
+@pytest.mark.parametrize("d,m,bo,br,mode,rot,md,n", TC_CASES)
+def test_split_tensor_core_encoder(d, m, bo, br, mode, rot, md, n):
+    _split_case(d, m, bo, br, mode, rot, md, n)
+
+
+def _split_case(d, m, bo, br, mode, rot, md, n):
     bits = synth.kv_prefill_batch(1, n, d, seed=51)[0]
     x = synth.bf16_from_bits(bits).astype(np.float64)
     ch = OM.outlier_channels(x, m)

@@ -404,10 +404,91 @@ __device__ __forceinline__ uint32_t sign_word(const uint32_t (&d)[32]) {
     return ~(z0 | (z1 << 16));
 }
 
-template <int B, bool PROD>
+// The coordinates of a tile in one or two groups (an outlier-channel split): group 0 holds
+// the first m32 chunks of 32 output coordinates, group 1 the rest. Without a split, group 0
+// is everything and the rotation operand is H diag(eps) built from TcParams::sgn.
+struct DuoGroups {
+    const uint16_t* pmat;   // split: rotation operand [128 outputs][128 channels] bf16, else null
+    int m32;                // chunks in group 0
+    uint8_t* codes[2];
+    uint8_t* qjl[2];
+    float* norms[2];
+    float* rnorms[2];
+    int code_bytes[2];      // row strides of the planes
+    int qjl_bytes[2];
+    float t2[2];            // b = 2: boundary between the inner and outer level
+    float cs[2];            // inner level (b = 2) / the level (b = 1)
+    float cb[2];            // outer level
+    float rsqrt_d[2];       // 1 / sqrt(group dimension): ||x_g|| = ||y_g|| / sqrt(d_g)
+};
+
+// Quantizes 32 coordinates y (fp32 bits) of one vector at BC bits: code words w0 (and w1 for
+// BC = 2), and for prod the residual r = ys - sign(y) c split into bf16 hi + lo and its squares
+// added to e0 / e1. Level bits go into one chain per 16 coordinates with funnel shifts: BC = 2
+// puts (y < 0, inner) of coordinate j at bits 2j+1, 2j; BC = 1 the bit y < 0 at bit j. Pairs of
+// coordinates go through f32x2 arithmetic: ys = y sc; inner iff ys^2 < t2^2.
+template <int BC, bool PROD>
+__device__ __forceinline__ void duo_quant_chunk(const uint32_t (&y)[32], float2 sc2, float2 nt2, float2 dcb2,
+                                                float2 cb2, uint32_t& w0, uint32_t& w1, float2& e0, float2& e1,
+                                                uint32_t (&hi)[16], uint32_t (&lo)[16]) {
+    uint32_t wd[2] = {0u, 0u};
+    float2 r2[16];
+#pragma unroll
+    for (int ii = 7; ii >= 0; --ii) {
+#pragma unroll
+        for (int g = 1; g >= 0; --g) {
+            const int pi = 8 * g + ii;   // coordinates 2 pi, 2 pi + 1 of the chunk
+            const uint32_t yb0 = y[2 * pi], yb1 = y[2 * pi + 1];
+            const float2 ys = __fmul2_rn(f2(__uint_as_float(yb0), __uint_as_float(yb1)), sc2);
+            float2 mag = cb2;
+            if constexpr (BC == 2) {
+                const float2 dd = __ffma2_rn(ys, ys, nt2);   // < 0: inner level
+                wd[g] = __funnelshift_l(yb1, wd[g], 1);
+                wd[g] = __funnelshift_l(__float_as_uint(dd.y), wd[g], 1);
+                wd[g] = __funnelshift_l(yb0, wd[g], 1);
+                wd[g] = __funnelshift_l(__float_as_uint(dd.x), wd[g], 1);
+                // exactly 1 (inner) or 0: a nonzero dd is far above the subnormal range
+                const float2 stp = f2(__saturatef(dd.x * -0x1p126f), __saturatef(dd.y * -0x1p126f));
+                mag = __ffma2_rn(stp, dcb2, cb2);
+            } else {
+                wd[g] = __funnelshift_l(yb1, wd[g], 1);
+                wd[g] = __funnelshift_l(yb0, wd[g], 1);
+            }
+            // -sign(y) c
+            const float2 nsm = f2(__uint_as_float(__float_as_uint(mag.x) | (~yb0 & 0x80000000u)),
+                                  __uint_as_float(__float_as_uint(mag.y) | (~yb1 & 0x80000000u)));
+            r2[pi] = __fadd2_rn(ys, nsm);
+        }
+    }
+    if constexpr (BC == 2) {
+        // code = 2 [y >= 0] + [y >= 0] xnor [inner]: index of the level, LSB first
+        w0 = (~wd[0] & 0xAAAAAAAAu) | (~(wd[0] ^ (wd[0] >> 1)) & 0x55555555u);
+        w1 = (~wd[1] & 0xAAAAAAAAu) | (~(wd[1] ^ (wd[1] >> 1)) & 0x55555555u);
+    } else {
+        w0 = ~(wd[0] | (wd[1] << 16));
+    }
+    if constexpr (PROD) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float2 rp = r2[k];
+            if (k & 1) e1 = __ffma2_rn(rp, rp, e1);
+            else e0 = __ffma2_rn(rp, rp, e0);
+            const __nv_bfloat162 h = __float22bfloat162_rn(rp);
+            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+            const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
+            const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), rp);
+            const __nv_bfloat162 lb = __float22bfloat162_rn(l);
+            hi[k] = hb;
+            lo[k] = *reinterpret_cast<const uint32_t*>(&lb);
+        }
+    }
+}
+
+template <int B0, int B1, bool PROD, bool SPLIT>
 __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (three warps per sub-partition)
-encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
-    static_assert(B == 1 || B == 2, "the two-team encoder covers 1- and 2-bit codes");
+encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, const DuoGroups gp) {
+    static_assert((B0 == 1 || B0 == 2) && (B1 == 1 || B1 == 2), "the two-team encoder covers 1- and 2-bit codes");
+    static_assert(SPLIT || B0 == B1, "one code width without a split");
     extern __shared__ uint8_t smem_raw[];
     TcSmemDuo& sm = *reinterpret_cast<TcSmemDuo*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int* abort_flag = &sm.abort;
@@ -436,12 +517,21 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         ptx::tmem_alloc(&sm.tmem_base, kDuoCols);
         ptx::tmem_relinquish();
     }
-    // H diag(eps): entry (n, k) = (-1)^popcount(n & k) * eps_k, at chunk k/8 of row n.
-    for (int i = tid; i < kD * kD; i += kDuoThreads) {
-        const int n = i >> 7, k = i & 127;
-        const uint32_t neg = (__popc(n & k) & 1) ^ ((p.sgn[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u);
-        *reinterpret_cast<uint16_t*>(sm.hd + (k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) =
-            neg ? 0xBF80u : 0x3F80u;
+    if constexpr (SPLIT) {
+        // the groups' rotations as one operand (row n = output coordinate, K = input channel)
+        for (int i = tid; i < kD * 16; i += kDuoThreads) {
+            const int row = i >> 4, c = i & 15;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(gp.pmat + row * kD + c * 8));
+            *reinterpret_cast<uint4*>(sm.hd + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
+        }
+    } else {
+        // H diag(eps): entry (n, k) = (-1)^popcount(n & k) * eps_k, at chunk k/8 of row n.
+        for (int i = tid; i < kD * kD; i += kDuoThreads) {
+            const int n = i >> 7, k = i & 127;
+            const uint32_t neg = (__popc(n & k) & 1) ^ ((p.sgn[k >> 1] >> ((k & 1) ? 31 : 15)) & 1u);
+            *reinterpret_cast<uint16_t*>(sm.hd + (k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) =
+                neg ? 0xBF80u : 0x3F80u;
+        }
     }
     if constexpr (PROD) {
         for (int i = tid; i < kD * 16; i += kDuoThreads) {
@@ -548,7 +638,7 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         const int vrow = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t ycol = t_lane + 256u * (uint32_t)t, hlc = ycol + 128u;
-        const float t2 = p.t[2];
+        const int m32 = SPLIT ? gp.m32 : 4;   // chunks of group 0
         bool fail = false;
         // MMA results (read through tcgen05.ld after a tcgen05 fence): one lane waits, and the
         // warp barrier orders the other lanes after it.
@@ -566,16 +656,19 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                 break;
             }
             ptx::tc_fence_after();
-            // ||H D x||^2 = d ||x||^2; the normalised rotated coordinate is y / ||H D x||
-            constexpr bool kSignsOnly = (B == 1 && !PROD);   // the code is the sign of y: one pass
+            // ||y_g||^2 per group (||H D x||^2 = d ||x||^2); the normalised rotated coordinate
+            // is y / ||y_g||. qc: sums per chunk of 32 coordinates.
+            constexpr bool kSignsOnly = (!SPLIT && B0 == 1 && !PROD);   // the code is the sign of y: one pass
+            float qc[4];
+            uint32_t cw[8];   // code words in chunk order: chunk c at cw[2c] (and cw[2c + 1] at 2 bits)
             float2 q0 = f2(0.f, 0.f), q1 = f2(0.f, 0.f);
-            uint32_t cw[4 * B];   // the vector's code words
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t a0[32], a1[32];
                 ptx::tmem_ld32(ycol + h * 64, a0);
                 ptx::tmem_ld32(ycol + h * 64 + 32, a1);
                 ptx::tmem_wait_ld();
+                if constexpr (SPLIT) q0 = q1 = f2(0.f, 0.f);   // per chunk
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const float2 u0 = f2(__uint_as_float(a0[2 * k]), __uint_as_float(a0[2 * k + 1]));
@@ -583,95 +676,73 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                     q0 = __ffma2_rn(u0, u0, q0);
                     q1 = __ffma2_rn(u1, u1, q1);
                 }
+                qc[2 * h] = q0.x + q0.y;
+                qc[2 * h + 1] = q1.x + q1.y;
                 if constexpr (kSignsOnly) {
-                    cw[2 * h] = sign_word(a0);   // bit j = [y_j >= 0] = the 1-bit code
-                    cw[2 * h + 1] = sign_word(a1);
+                    cw[4 * h] = sign_word(a0);   // bit j = [y_j >= 0] = the 1-bit code
+                    cw[4 * h + 2] = sign_word(a1);
                 }
             }
-            const float ssq = (q0.x + q0.y) + (q1.x + q1.y);
+            float ssq[2] = {0.f, 0.f};
+            if constexpr (SPLIT) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    ssq[0] += (c < m32) ? qc[c] : 0.f;
+                    ssq[1] += (c < m32) ? 0.f : qc[c];
+                }
+            } else {
+                ssq[0] = (q0.x + q0.y) + (q1.x + q1.y);
+            }
             if constexpr (kSignsOnly) {   // y is read to the end: the next rotation may go
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&sm.bar_free[t]);
             }
-            const bool nz = ssq > 0.f;
-            const float sc = nz ? rsqrtf(ssq) : 0.f;
-            const float cs = nz ? p.c[B == 2 ? 2 : 1] : 0.f;   // inner level (b = 2) / the level (b = 1)
-            const float cb = nz ? p.c[B == 2 ? 3 : 1] : 0.f;   // outer level
-            const float2 sc2 = f2(sc, sc);
-            const float2 nt2 = f2(-t2 * t2, -t2 * t2);
-            const float2 dcb2 = f2(cs - cb, cs - cb), cb2 = f2(cb, cb);
-            float2 e0 = f2(0.f, 0.f), e1 = f2(0.f, 0.f);
-            // 32 coordinates at a time. Level bits go into one chain per 16 coordinates with
-            // funnel shifts: b = 2 puts (y < 0, inner) of coordinate j at bits 2j+1, 2j; b = 1
-            // the bit y < 0 at bit j. Pairs of coordinates go through f32x2 arithmetic:
-            // ys = y sc; inner iff ys^2 < t2^2; the residual is r = ys - sign(y) c, c the
-            // inner or outer level.
+            bool nz[2];
+            float sc[2], cs[2], cb[2], t2[2];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                nz[g] = ssq[g] > 0.f;
+                sc[g] = nz[g] ? rsqrtf(ssq[g]) : 0.f;
+                cs[g] = nz[g] ? gp.cs[g] : 0.f;
+                cb[g] = nz[g] ? gp.cb[g] : 0.f;
+                t2[g] = gp.t2[g];
+            }
+            float rs[2] = {0.f, 0.f};   // ||r_g||^2
+            float2 e0 = f2(0.f, 0.f), e1 = f2(0.f, 0.f);   // ||r||^2 in pairs (per chunk for a split)
+            // 32 coordinates at a time, each at its group's width, scale and levels.
 #pragma unroll
             for (int c = 0; c < (kSignsOnly ? 0 : 4); ++c) {
                 uint32_t y[32];
                 ptx::tmem_ld32(ycol + 32 * c, y);
                 ptx::tmem_wait_ld();
-                uint32_t wd[2] = {0u, 0u};
-                float2 r2[16];
-#pragma unroll
-                for (int ii = 7; ii >= 0; --ii) {
-#pragma unroll
-                    for (int g = 1; g >= 0; --g) {
-                        const int pi = 8 * g + ii;   // coordinates 2 pi, 2 pi + 1 of the chunk
-                        const uint32_t yb0 = y[2 * pi], yb1 = y[2 * pi + 1];
-                        const float2 ys = __fmul2_rn(f2(__uint_as_float(yb0), __uint_as_float(yb1)), sc2);
-                        float2 mag = cb2;
-                        if constexpr (B == 2) {
-                            const float2 dd = __ffma2_rn(ys, ys, nt2);   // < 0: inner level
-                            wd[g] = __funnelshift_l(yb1, wd[g], 1);
-                            wd[g] = __funnelshift_l(__float_as_uint(dd.y), wd[g], 1);
-                            wd[g] = __funnelshift_l(yb0, wd[g], 1);
-                            wd[g] = __funnelshift_l(__float_as_uint(dd.x), wd[g], 1);
-                            // exactly 1 (inner) or 0: a nonzero dd is far above the subnormal range
-                            const float2 stp = f2(__saturatef(dd.x * -0x1p126f), __saturatef(dd.y * -0x1p126f));
-                            mag = __ffma2_rn(stp, dcb2, cb2);
-                        } else {
-                            wd[g] = __funnelshift_l(yb1, wd[g], 1);
-                            wd[g] = __funnelshift_l(yb0, wd[g], 1);
-                        }
-                        // -sign(y) c
-                        const float2 nsm = f2(__uint_as_float(__float_as_uint(mag.x) | (~yb0 & 0x80000000u)),
-                                              __uint_as_float(__float_as_uint(mag.y) | (~yb1 & 0x80000000u)));
-                        r2[pi] = __fadd2_rn(ys, nsm);
-                    }
+                const bool g1 = SPLIT && c >= m32;   // the chunk's group (selects, no indexing)
+                const float scg = g1 ? sc[1] : sc[0], csg = g1 ? cs[1] : cs[0], cbg = g1 ? cb[1] : cb[0];
+                const float t2g = g1 ? t2[1] : t2[0];
+                const float2 sc2 = f2(scg, scg);
+                const float2 nt2 = f2(-t2g * t2g, -t2g * t2g);
+                const float2 dcb2 = f2(csg - cbg, csg - cbg), cb2 = f2(cbg, cbg);
+                uint32_t hi[16], lo[16];
+                if constexpr (SPLIT) e0 = e1 = f2(0.f, 0.f);
+                if (PROD && c == 1) {   // half way: the other team's next rotation may go
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&sm.bar_mid[t]);
                 }
-                if constexpr (B == 2) {
-                    // code = 2 [y >= 0] + [y >= 0] xnor [inner]: index of the level, LSB first
-#pragma unroll
-                    for (int g = 0; g < 2; ++g)
-                        cw[2 * c + g] = (~wd[g] & 0xAAAAAAAAu) | (~(wd[g] ^ (wd[g] >> 1)) & 0x55555555u);
-                } else {
-                    cw[c] = ~(wd[0] | (wd[1] << 16));
-                }
+                if (!g1)
+                    duo_quant_chunk<B0, PROD>(y, sc2, nt2, dcb2, cb2, cw[2 * c], cw[2 * c + 1], e0, e1, hi, lo);
+                else
+                    duo_quant_chunk<B1, PROD>(y, sc2, nt2, dcb2, cb2, cw[2 * c], cw[2 * c + 1], e0, e1, hi, lo);
                 if constexpr (PROD) {
-                    if (c == 1) {
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&sm.bar_mid[t]);
-                    }
-                    uint32_t hi[16], lo[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float2 rp = r2[k];
-                        if (k & 1) e1 = __ffma2_rn(rp, rp, e1);
-                        else e0 = __ffma2_rn(rp, rp, e0);
-                        const __nv_bfloat162 h = __float22bfloat162_rn(rp);
-                        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
-                        const float2 hf = f2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u));
-                        const float2 l = __ffma2_rn(hf, f2(-1.f, -1.f), rp);
-                        const __nv_bfloat162 lb = __float22bfloat162_rn(l);
-                        hi[k] = hb;
-                        lo[k] = *reinterpret_cast<const uint32_t*>(&lb);
+                    if constexpr (SPLIT) {
+                        const float ec = (e0.x + e0.y) + (e1.x + e1.y);
+                        rs[0] += g1 ? 0.f : ec;
+                        rs[1] += g1 ? ec : 0.f;
                     }
                     ptx::tmem_st16(hlc + 16 * c, hi);
                     ptx::tmem_st16(hlc + 64 + 16 * c, lo);
                 }
             }
+            if constexpr (PROD && !SPLIT) rs[0] = (e0.x + e0.y) + (e1.x + e1.y);
             if constexpr (PROD) ptx::tmem_wait_st();
             if constexpr (!kSignsOnly) {
                 ptx::tc_fence_before();
@@ -679,18 +750,45 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                 if (lane == 0) ptx::mbar_arrive(PROD ? &sm.bar_hl[t] : &sm.bar_free[t]);
             }
             if (row < p.n) {
-                if constexpr (B == 2) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.codes + row * 32);
-                    dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                    dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                if constexpr (!SPLIT) {
+                    if constexpr (B0 == 2) {
+                        uint4* dst = reinterpret_cast<uint4*>(gp.codes[0] + row * 32);
+                        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                    } else {
+                        *reinterpret_cast<uint4*>(gp.codes[0] + row * 16) = make_uint4(cw[0], cw[2], cw[4], cw[6]);
+                    }
                 } else {
-                    *reinterpret_cast<uint4*>(p.codes + row * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    uint32_t* dst0 = reinterpret_cast<uint32_t*>(gp.codes[0] + row * gp.code_bytes[0]);
+                    uint32_t* dst1 = reinterpret_cast<uint32_t*>(gp.codes[1] + row * gp.code_bytes[1]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (c < m32) {
+                            if constexpr (B0 == 2) {
+                                dst0[2 * c] = cw[2 * c];
+                                dst0[2 * c + 1] = cw[2 * c + 1];
+                            } else {
+                                dst0[c] = cw[2 * c];
+                            }
+                        } else {
+                            if constexpr (B1 == 2) {
+                                dst1[2 * (c - m32)] = cw[2 * c];
+                                dst1[2 * (c - m32) + 1] = cw[2 * c + 1];
+                            } else {
+                                dst1[c - m32] = cw[2 * c];
+                            }
+                        }
+                    }
+                    gp.norms[1][row] = sqrtf(ssq[1]) * gp.rsqrt_d[1];
                 }
-                p.norms[row] = sqrtf(ssq) * p.rsqrt_d;
+                gp.norms[0][row] = sqrtf(ssq[0]) * gp.rsqrt_d[0];
             }
             if constexpr (PROD) {
-                if (row < p.n) p.rnorms[row] = sqrtf((e0.x + e0.y) + (e1.x + e1.y));
-                // signs of S r, all ones for a zero vector
+                if (row < p.n) {
+                    gp.rnorms[0][row] = sqrtf(rs[0]);
+                    if constexpr (SPLIT) gp.rnorms[1][row] = sqrtf(rs[1]);
+                }
+                // signs of S r, all ones for a zero vector (group)
                 if (!wait_bar(&sm.bar_d[t], (uint32_t)(i & 1))) {
                     fail = true;
                     break;
@@ -709,9 +807,20 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&sm.bar_free[t]);
-                if (row < p.n)
-                    *reinterpret_cast<uint4*>(p.qjl + row * 16) =
-                        nz ? make_uint4(zw[0], zw[1], zw[2], zw[3]) : make_uint4(~0u, ~0u, ~0u, ~0u);
+                if (row < p.n) {
+                    if constexpr (!SPLIT) {
+                        *reinterpret_cast<uint4*>(gp.qjl[0] + row * 16) =
+                            nz[0] ? make_uint4(zw[0], zw[1], zw[2], zw[3]) : make_uint4(~0u, ~0u, ~0u, ~0u);
+                    } else {
+                        uint32_t* q0 = reinterpret_cast<uint32_t*>(gp.qjl[0] + row * gp.qjl_bytes[0]);
+                        uint32_t* q1 = reinterpret_cast<uint32_t*>(gp.qjl[1] + row * gp.qjl_bytes[1]);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            if (c < m32) q0[c] = nz[0] ? zw[c] : ~0u;
+                            else q1[c - m32] = nz[1] ? zw[c] : ~0u;
+                        }
+                    }
+                }
             }
         }
         if (fail) {
@@ -754,20 +863,50 @@ int sm_count() {
     return sms;
 }
 
-template <int B, bool PROD>
-int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl, float* norms,
-              float* rnorms, cudaStream_t stream) {
+// Levels of group g of the two-team encoder from a state with b_mse 1 or 2.
+void duo_levels(const DevState& st, DuoGroups& gp, int g) {
+    gp.t2[g] = (st.b_mse == 2) ? st.t[2] : 0.f;
+    gp.cs[g] = st.c[st.b_mse == 2 ? 2 : 1];
+    gp.cb[g] = st.c[st.b_mse == 2 ? 3 : 1];
+    gp.rsqrt_d[g] = st.rsqrt_d;
+}
+
+bool make_tmap(CUtensorMap* tmap, const void* x, int64_t n, int64_t ld) {
     EncodeTiledFn enc = encode_tiled_fn();
-    if (!enc) return (int)cudaErrorNotSupported;
-    CUtensorMap tmap;
+    if (!enc) return false;
     const cuuint64_t gdim[2] = {(cuuint64_t)kD, (cuuint64_t)n};
     const cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
     const cuuint32_t box[2] = {64, kTile};
     const cuuint32_t estride[2] = {1, 1};
-    CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
+    return enc(tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int B0, int B1, bool PROD, bool SPLIT>
+int launch_duo(const CUtensorMap& tmap, const TcParams& p, const DuoGroups& gp, cudaStream_t stream) {
+    auto kern = encode_duo_kernel<B0, B1, PROD, SPLIT>;
+    const size_t smem = sizeof(TcSmemDuo) + 1024;
+    static int attr_set_for_device = -1;   // per instantiation
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_set_for_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_set_for_device = dev;
+    }
+    const int64_t ntiles = (p.n + kTile - 1) / kTile;
+    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count());
+    kern<<<grid, kDuoThreads, smem, stream>>>(tmap, p, gp);
+    return (int)cudaGetLastError();
+}
+
+template <int B, bool PROD>
+int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, uint8_t* qjl, float* norms,
+              float* rnorms, cudaStream_t stream) {
+    CUtensorMap tmap;
+    if (!encode_tiled_fn()) return (int)cudaErrorNotSupported;
+    if (!make_tmap(&tmap, x, n, ld)) return (int)cudaErrorInvalidValue;
     TcParams p;
     p.codes = codes;
     p.qjl = qjl;
@@ -785,21 +924,42 @@ int launch_tc(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t*
         const bool n1 = (st.signs[(2 * i + 1) >> 5] >> ((2 * i + 1) & 31)) & 1u;
         p.sgn[i] = (n0 ? 0x8000u : 0u) | (n1 ? 0x80000000u : 0u);
     }
-    constexpr bool kTwo = (B == 1 || B == 2);
-    const size_t smem = (kTwo ? sizeof(TcSmemDuo) : sizeof(TcSmem)) + 1024;
-    auto kern = kTwo ? encode_duo_kernel<(B <= 2 ? B : 2), PROD> : encode_tc_kernel<B, PROD>;
-    static int attr_set_for_device = -1;   // per instantiation
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (attr_set_for_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return (int)e;
-        attr_set_for_device = dev;
+    if constexpr (B == 1 || B == 2) {
+        DuoGroups gp = {};
+        gp.pmat = nullptr;
+        gp.m32 = 4;
+        for (int g = 0; g < 2; ++g) {   // group 1 is empty without a split
+            gp.codes[g] = codes;
+            gp.qjl[g] = qjl;
+            gp.norms[g] = norms;
+            gp.rnorms[g] = rnorms;
+            gp.code_bytes[g] = st.code_bytes;
+            gp.qjl_bytes[g] = st.qjl_bytes;
+            duo_levels(st, gp, g);
+        }
+        return launch_duo<B, B, PROD, false>(tmap, p, gp, stream);
+    } else {
+        auto kern = encode_tc_kernel<B, PROD>;
+        const size_t smem = sizeof(TcSmem) + 1024;
+        static int attr_set_for_device = -1;   // per instantiation
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (attr_set_for_device != dev) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return (int)e;
+            attr_set_for_device = dev;
+        }
+        const int64_t ntiles = (n + kTile - 1) / kTile;
+        const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * 2);
+        kern<<<grid, kTile, smem, stream>>>(tmap, p);
+        return (int)cudaGetLastError();
     }
-    const int64_t ntiles = (n + kTile - 1) / kTile;
-    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)sm_count() * (kTwo ? 1 : 2));
-    kern<<<grid, kTwo ? kDuoThreads : kTile, smem, stream>>>(tmap, p);
-    return (int)cudaGetLastError();
+}
+
+template <int B0, bool PROD>
+int launch_split_b1(int b1, const CUtensorMap& tmap, const TcParams& p, const DuoGroups& gp, cudaStream_t s) {
+    if (b1 == 1) return launch_duo<B0, 1, PROD, true>(tmap, p, gp, s);
+    return launch_duo<B0, 2, PROD, true>(tmap, p, gp, s);
 }
 
 }  // namespace
@@ -830,6 +990,47 @@ int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, u
         case 4: return launch_tc<4, false>(st, x, n, ld, codes, qjl, norms, rnorms, s);
         default: return (int)cudaErrorInvalidValue;
     }
+}
+
+// The outlier-channel split of a 128-channel bf16 input on the two-team encoder: group 0
+// (state so, the first m output coordinates) and group 1 (si, the other 128 - m). pmat is the
+// two groups' rotations as one [128][128] bf16 operand (each row a Hadamard row times the
+// group's signs, placed at the group's channels), sbd the block-diagonal [128][128] S.
+bool split_tc_supported(const DevState& so, const DevState& si, int m) {
+    const bool prod = so.mode == TQ_PROD;
+    if (so.rot != TQ_ROT_RHT || si.rot != TQ_ROT_RHT || so.mode != si.mode) return false;
+    if (m % 32 != 0 || m < 32 || m > 96 || so.d != m || si.d != kD - m) return false;
+    if (so.b_mse < 1 || so.b_mse > 2 || si.b_mse < 1 || si.b_mse > 2) return false;
+    return !prod || (so.mat_dtype == TQ_BF16 && si.mat_dtype == TQ_BF16);
+}
+
+int launch_encode_split_tc(const DevState& so, const DevState& si, const uint16_t* pmat, const uint16_t* sbd,
+                           const void* x, int64_t n, int64_t ld, uint8_t* const codes[2], uint8_t* const qjl[2],
+                           float* const norms[2], float* const rnorms[2], void* stream) {
+    cudaStream_t s = (cudaStream_t)stream;
+    CUtensorMap tmap;
+    if (!encode_tiled_fn()) return (int)cudaErrorNotSupported;
+    if (!make_tmap(&tmap, x, n, ld)) return (int)cudaErrorInvalidValue;
+    TcParams p = {};
+    p.s = sbd;
+    p.n = n;
+    DuoGroups gp = {};
+    gp.pmat = pmat;
+    gp.m32 = so.d / 32;
+    const DevState* st[2] = {&so, &si};
+    for (int g = 0; g < 2; ++g) {
+        gp.codes[g] = codes[g];
+        gp.qjl[g] = qjl[g];
+        gp.norms[g] = norms[g];
+        gp.rnorms[g] = rnorms[g];
+        gp.code_bytes[g] = st[g]->code_bytes;
+        gp.qjl_bytes[g] = st[g]->qjl_bytes;
+        duo_levels(*st[g], gp, g);
+    }
+    const bool prod = so.mode == TQ_PROD;
+    if (so.b_mse == 1)
+        return prod ? launch_split_b1<1, true>(si.b_mse, tmap, p, gp, s) : launch_split_b1<1, false>(si.b_mse, tmap, p, gp, s);
+    return prod ? launch_split_b1<2, true>(si.b_mse, tmap, p, gp, s) : launch_split_b1<2, false>(si.b_mse, tmap, p, gp, s);
 }
 
 namespace {

@@ -589,6 +589,49 @@ bool planes_ok(const tq_state* st, const tq_planes* p) {
 }
 }  // namespace
 
+namespace {
+// Entry (n, k) of the Hadamard matrix of a state's order d: Sylvester's (-1)^popcount(n & k) for
+// d a power of two, else H_12 (x) H_{d/12} (Paley's H_12 from the state).
+bool hadamard_negative(const tq_state* st, int n, int k) {
+    const int d = st->p.d;
+    if ((d & (d - 1)) == 0) return __builtin_popcount((unsigned)(n & k)) & 1;
+    const int q = d / 12;
+    const bool neg12 = (st->dev.h12[n / q] >> (k / q)) & 1u;
+    return neg12 ^ (bool)(__builtin_popcount((unsigned)((n % q) & (k % q))) & 1);
+}
+
+uint16_t bf16_bits_exact(double v) {   // v is a stored bf16 value
+    const float f = (float)v;
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+// Operands of the split on the tensor-core encoder: row r < m of the rotation holds row r of
+// the outer group's H diag(eps) at the outer channels, row m + r the inner group's at the
+// inner channels (+-1: the 1/sqrt(d_g) of each group cancels in y / ||y_g||); then S of the
+// two groups on the diagonal blocks.
+void split_tc_operands(const tq_state* outer, const tq_state* inner, const std::vector<int32_t>& maps,
+                       std::vector<uint16_t>& ops) {
+    ops.assign(2 * 128 * 128, 0);
+    const tq_state* st[2] = {outer, inner};
+    int off = 0;
+    for (int g = 0; g < 2; ++g) {
+        const tq_state* s = st[g];
+        const int dg = s->p.d;
+        for (int n = 0; n < dg; ++n) {
+            for (int k = 0; k < dg; ++k) {
+                const bool eps_neg = (s->dev.signs[k >> 5] >> (k & 31)) & 1u;
+                ops[(size_t)(off + n) * 128 + maps[off + k]] = (hadamard_negative(s, n, k) ^ eps_neg) ? 0xBF80u : 0x3F80u;
+                if (s->p.mode == TQ_PROD)
+                    ops[128 * 128 + (size_t)(off + n) * 128 + off + k] = bf16_bits_exact(s->s[(size_t)n * dg + k]);
+            }
+        }
+        off += dg;
+    }
+}
+}  // namespace
+
 int tq_split_create(const tq_state* outer, const tq_state* inner, const int32_t* h_channels, int m,
                     tq_split** out) {
     if (!outer || !inner || !out || m < 1) return TQ_EINVAL;
@@ -614,8 +657,15 @@ int tq_split_create(const tq_state* outer, const tq_state* inner, const int32_t*
     sp->channels.assign(h_channels, h_channels + m);
     cudaError_t e = cudaMalloc(&sp->d_chan, (size_t)d * sizeof(int32_t));
     if (e == cudaSuccess) e = cudaMemcpy(sp->d_chan, maps.data(), (size_t)d * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && d == 128 && tq::split_tc_supported(outer->dev, inner->dev, m)) {
+        std::vector<uint16_t> ops;
+        split_tc_operands(outer, inner, maps, ops);
+        e = cudaMalloc(&sp->d_tc, ops.size() * sizeof(uint16_t));
+        if (e == cudaSuccess) e = cudaMemcpy(sp->d_tc, ops.data(), ops.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    }
     if (e != cudaSuccess) {
         if (sp->d_chan) cudaFree(sp->d_chan);
+        if (sp->d_tc) cudaFree(sp->d_tc);
         delete sp;
         return cuda_status(e);
     }
@@ -625,9 +675,10 @@ int tq_split_create(const tq_state* outer, const tq_state* inner, const int32_t*
 
 void tq_split_destroy(tq_split* sp) {
     if (!sp) return;
-    if (sp->d_chan) {
+    if (sp->d_chan || sp->d_tc) {
         DeviceGuard g(sp->outer->p.device);
-        cudaFree(sp->d_chan);
+        if (sp->d_chan) cudaFree(sp->d_chan);
+        if (sp->d_tc) cudaFree(sp->d_tc);
     }
     delete sp;
 }
@@ -644,6 +695,15 @@ int tq_split_quantize(const tq_split* sp, const void* x, int dtype, int64_t n, i
     if (!g.ok) return cuda_status(cudaGetLastError());
     const bool prod = sp->outer->p.mode == TQ_PROD;
     const int m = sp->outer->p.d;
+    if (sp->d_tc && dtype == TQ_BF16 && n < ((int64_t)1 << 31)) {
+        uint8_t* const codes[2] = {outer->codes, inner->codes};
+        uint8_t* const qjl[2] = {prod ? outer->qjl : nullptr, prod ? inner->qjl : nullptr};
+        float* const norms[2] = {outer->norms, inner->norms};
+        float* const rnorms[2] = {prod ? outer->rnorms : nullptr, prod ? inner->rnorms : nullptr};
+        return cuda_status((cudaError_t)tq::launch_encode_split_tc(sp->outer->dev, sp->inner->dev, sp->d_tc,
+                                                                   sp->d_tc + 128 * 128, x, n, ld, codes, qjl, norms,
+                                                                   rnorms, stream));
+    }
     int e = launch_encode_channels(sp->outer->dev, x, dtype, n, ld, sp->d_chan, outer->codes,
                                    prod ? outer->qjl : nullptr, outer->norms, prod ? outer->rnorms : nullptr, stream);
     if (e == 0)

@@ -83,6 +83,7 @@ struct tq_split {
     int d;
     std::vector<int32_t> channels;   // host copy of the outer channel list
     int32_t* d_chan = nullptr;       // device: outer map [m], then inner map [d - m]
+    uint16_t* d_tc = nullptr;        // tensor-core encoder operands (or null): rotation [128][128], then S [128][128], bf16
 };
 
 namespace tq {
@@ -115,6 +116,13 @@ int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, 
 // rows of q [count][ldq] gathered at columns chan[0..m) into out [count][m] (same dtype)
 int launch_gather_rows(const void* q, int dtype, int64_t count, int64_t ldq, const int32_t* chan, int m, void* out,
                        void* stream);
+// Outlier-channel split on the two-team tensor-core encoder (d = 128, bf16 input, both groups
+// RHT at 1 or 2 bits, m a multiple of 32): pmat / sbd are the [128][128] bf16 rotation and
+// block-diagonal S operands built by the host; planes index 0 = outer group, 1 = inner.
+bool split_tc_supported(const DevState& so, const DevState& si, int m);
+int launch_encode_split_tc(const DevState& so, const DevState& si, const uint16_t* pmat, const uint16_t* sbd,
+                           const void* x, int64_t n, int64_t ld, uint8_t* const codes[2], uint8_t* const qjl[2],
+                           float* const norms[2], float* const rnorms[2], void* stream);
 // Planes of the two channel groups of a split (index 0: outer, 1: inner).
 struct SplitPlanes {
     const uint8_t* codes[2];
