@@ -243,6 +243,27 @@ int launch_tables(const DevState& st, const void* q, int qdtype, int64_t count, 
     return (int)cudaGetLastError();
 }
 
+// N consecutive 32-bit words from a row whose stride is 4 N bytes (16-, 8- or 4-byte loads).
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t* __restrict__ src, uint32_t (&w)[N]) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else if constexpr (N % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
+            w[2 * i] = v.x; w[2 * i + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) w[i] = __ldg(src + i);
+    }
+}
+
 template <int D, int B, bool PROD, int QT>
 __global__ void __launch_bounds__(kThreads)
 score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
@@ -276,20 +297,10 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
     constexpr int ZW = PROD ? D / 32 : 1;
     auto load_key = [&](int64_t key, uint32_t (&w)[CW], uint32_t (&z)[ZW], float& rn, float& nu) {
         const int64_t gk = grp * n + key;
-        const uint4* src = reinterpret_cast<const uint4*>(codes + gk * (D * B / 8));
-#pragma unroll
-        for (int i = 0; i < CW / 4; ++i) {
-            const uint4 v = __ldg(src + i);
-            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
+        load_words<CW>(reinterpret_cast<const uint32_t*>(codes + gk * (D * B / 8)), w);
         rn = 0.f;
         if constexpr (PROD) {
-            const uint4* zs = reinterpret_cast<const uint4*>(qjl + gk * (D / 8));
-#pragma unroll
-            for (int i = 0; i < D / 128; ++i) {
-                const uint4 v = __ldg(zs + i);
-                z[4 * i] = v.x; z[4 * i + 1] = v.y; z[4 * i + 2] = v.z; z[4 * i + 3] = v.w;
-            }
+            load_words<ZW>(reinterpret_cast<const uint32_t*>(qjl + gk * (D / 8)), z);
             rn = __ldg(rnorms + gk);
         }
         nu = __ldg(norms + gk);
@@ -451,15 +462,21 @@ int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_
 }
 
 bool score_lut_supported(const DevState& st) {
-    return (st.d == 128 || st.d == 256) && st.b_mse >= 1 && st.b_mse <= 4;
+    const bool dim = st.d == 32 || st.d == 64 || st.d == 96 || st.d == 128 || st.d == 256;
+    return dim && st.b_mse >= 1 && st.b_mse <= 4;
 }
 
 int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                      const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
                      void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
-    if (st.d == 128) return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-    return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+    switch (st.d) {
+        case 32: return launch_lut_b<32>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 64: return launch_lut_b<64>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 96: return launch_lut_b<96>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 128: return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        default: return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+    }
 }
 
 }  // namespace tq
