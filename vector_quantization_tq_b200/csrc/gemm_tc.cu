@@ -4,7 +4,7 @@
 //
 // C[M x N] = A[M x K] * B[N x K]^T, A and B bf16 K-major in global memory, fp32 accumulate.
 // Warp-specialised CTA of 6 warps per 128 x BN output tile:
-//   warp 0  TMA producer: K-steps of 64 through a 4-stage shared-memory ring;
+//   warp 0  TMA producer: K-steps of 64 through a 2-stage shared-memory ring (two CTAs per SM);
 //   warp 1  MMA issuer: 4 x tcgen05.mma (M128 N=BN K16) per stage, commit frees the stage;
 //   warps 2-5 epilogue: one TMEM lane (= output row) per thread, 32 columns at a time.
 // Epilogues:
@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 2;   // 2 x 48 KB: two CTAs per SM, so one's epilogue overlaps the other's MMAs
 constexpr int kGemmThreads = 192;
 
 enum EpiKind { kStoreF32 = 0, kRotate = 1, kSigns = 2 };
@@ -65,7 +65,7 @@ struct __align__(1024) GemmSmem {
 };
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
