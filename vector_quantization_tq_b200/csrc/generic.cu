@@ -165,13 +165,31 @@ encode_kernel(const DevState st, const void* __restrict__ x, int dtype, int64_t 
         if (r2out != nullptr) {
             // prod with S r on the tensor core: the residual as [r_hi | r_lo] bf16 rows
             // (r_lo = bf16(r - r_hi)) and ||r||^2 for the signs pass
+            if constexpr (E == 8) {   // 16-byte stores of the thread's 8 hi and 8 lo halves
+                uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const int j = tid * E + e;
-                const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(r[e]));
-                const float lo = r[e] - __uint_as_float((uint32_t)hb << 16);
-                r2out[vec * 2 * D + j] = hb;
-                r2out[vec * 2 * D + D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+                for (int e = 0; e < E; e += 2) {
+                    uint32_t hb[2], lb[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        hb[k] = __bfloat16_as_ushort(__float2bfloat16_rn(r[e + k]));
+                        const float lo = r[e + k] - __uint_as_float(hb[k] << 16);
+                        lb[k] = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+                    }
+                    hw[e / 2] = hb[0] | (hb[1] << 16);
+                    lw[e / 2] = lb[0] | (lb[1] << 16);
+                }
+                *reinterpret_cast<uint4*>(r2out + vec * 2 * D + tid * E) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(r2out + vec * 2 * D + D + tid * E) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int j = tid * E + e;
+                    const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(r[e]));
+                    const float lo = r[e] - __uint_as_float((uint32_t)hb << 16);
+                    r2out[vec * 2 * D + j] = hb;
+                    r2out[vec * 2 * D + D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+                }
             }
             const float rsum = group_sum<NT>(rr, red);
             if (tid == 0) {
