@@ -858,8 +858,14 @@ int launch_encode_generic(const DevState& st, const void* x, int dtype, int64_t 
 
 // Codes, norms, the residual operand [r_hi | r_lo] and ||r||^2 (first of rho_stride slots) of
 // a prod encode whose S r runs on the tensor core.
+bool residual_rht_supported(const DevState& st);
+int launch_residual_rht(const DevState& st, const void* x, int64_t n, int64_t ld, uint8_t* codes, float* norms,
+                        uint16_t* r2out, float* rho_out, int rho_stride, void* stream);
+
 int launch_encode_residual(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
                            float* norms, uint16_t* r2out, float* rho_out, int rho_stride, void* stream) {
+    if (dtype == TQ_BF16 && residual_rht_supported(st))   // warp per vector, Hadamard in registers
+        return launch_residual_rht(st, x, n, ld, codes, norms, r2out, rho_out, rho_stride, stream);
     cudaStream_t s = (cudaStream_t)stream;
     return with_layout(st.d, [&](auto e, auto nt) {
         return launch_encode_t<decltype(e)::value, decltype(nt)::value>(st, x, dtype, n, ld, nullptr, 1, codes,
