@@ -139,11 +139,13 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                 const uint4 v = src[i];
                 w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
             }
-            float a1[1] = {0.f};
+            // table lookups into paired accumulators (two independent chains, f32x2 adds)
+            float2 p1[1] = {make_float2(0.f, 0.f)};
             if constexpr (KG::G == 4) {
 #pragma unroll
-                for (int wi = 0; wi < CW; ++wi) add_nibbles<1, 0>(w[wi], tm + 8 * wi * 16, a1);
+                for (int wi = 0; wi < CW; ++wi) add_nibbles<1, 0>(w[wi], tm + 8 * wi * 16, p1);
             } else {
+                static_assert(KG::NG % 2 == 0, "groups in pairs");
 #pragma unroll
                 for (int k = 0; k < KG::NG; ++k) {
                     const int bit = k * KG::G;
@@ -151,18 +153,20 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                     uint32_t e;
                     if (sh + KG::G <= 32) e = (w[wi] >> sh) & (KG::E - 1);
                     else e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (KG::E - 1);
-                    a1[0] += tm[k * KG::E + e];
+                    if (k & 1) p1[0].y += tm[k * KG::E + e];
+                    else p1[0].x += tm[k * KG::E + e];
                 }
             }
-            float a2[1] = {0.f}, g2 = 0.f;
+            float2 p2[1] = {make_float2(0.f, 0.f)};
+            float g2 = 0.f;
             if constexpr (KPROD) {
                 const uint4 zv = *reinterpret_cast<const uint4*>(B.kz + threadIdx.x * 16);
                 const uint32_t z[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-                for (int wi = 0; wi < 4; ++wi) add_nibbles<1, 0>(z[wi], tz + 8 * wi * 16, a2);
+                for (int wi = 0; wi < 4; ++wi) add_nibbles<1, 0>(z[wi], tz + 8 * wi * 16, p2);
                 g2 = B.kr[threadIdx.x] * ks.qjl_scale;
             }
-            s = scale * B.kn[threadIdx.x] * fmaf(g2, a2[0], a1[0]);
+            s = scale * B.kn[threadIdx.x] * fmaf(g2, p2[0].x + p2[0].y, p1[0].x + p1[0].y);
         }
         // ---- B: online softmax bookkeeping ----
         const float wm = warp_max(s);

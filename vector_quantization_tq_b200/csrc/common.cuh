@@ -133,12 +133,13 @@ __device__ __forceinline__ uint32_t extract_code(const uint32_t* __restrict__ ro
 }
 
 
-// Table lookups over the 8 nibbles of a packed word: acc[qi] += sum_m T_m[e_m], e_m the
-// m-th nibble of w and T_m the 16-entry float table at t0 + 16 m (query qi's tables
-// `stride` floats further on). Two masks put the nibbles, times 4, into bytes; a lookup is
-// then one byte permute and one shared-memory load.
+// Table lookups over the 8 nibbles of a packed word: acc[qi].x + acc[qi].y grows by
+// sum_m T_m[e_m], e_m the m-th nibble of w and T_m the 16-entry float table at t0 + 16 m
+// (query qi's tables STRIDE floats further on). Two masks put the nibbles, times 4, into
+// bytes; a lookup is then one byte permute and one shared-memory load, and the two values of
+// each permute go into .x and .y with one f32x2 add (two independent chains per query).
 template <int QT, int STRIDE>
-__device__ __forceinline__ void add_nibbles(uint32_t w, const float* t0, float (&acc)[QT]) {
+__device__ __forceinline__ void add_nibbles(uint32_t w, const float* t0, float2 (&acc)[QT]) {
     const uint32_t lo4 = (w << 2) & 0x3C3C3C3Cu;   // nibbles 0, 2, 4, 6
     const uint32_t hi4 = (w >> 2) & 0x3C3C3C3Cu;   // nibbles 1, 3, 5, 7
 #pragma unroll
@@ -148,12 +149,12 @@ __device__ __forceinline__ void add_nibbles(uint32_t w, const float* t0, float (
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) {
             const char* t = reinterpret_cast<const char*>(t0 + qi * STRIDE + 2 * m * 16);
-            acc[qi] += *reinterpret_cast<const float*>(t + o0);
-            acc[qi] += *reinterpret_cast<const float*>(t + 64 + o1);
+            const float2 v = make_float2(*reinterpret_cast<const float*>(t + o0),
+                                         *reinterpret_cast<const float*>(t + 64 + o1));
+            acc[qi] = __fadd2_rn(acc[qi], v);
         }
     }
 }
-
 
 // In-place Hadamard transform of order d = 12 m (m a power of two) on buf[0..d), viewed as
 // 12 rows of m: Sylvester's transform along each row, then Paley's H_12 (rows of st.h12,

@@ -318,12 +318,16 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
         const float nu = nun;
         if (key + kThreads < k_end) load_key(key + kThreads, wn, zn, rnn, nun);
         float a1[QT], a2[QT];
+        float2 p1[QT], p2[QT];   // paired accumulators of the nibble lookups
 #pragma unroll
-        for (int qi = 0; qi < QT; ++qi) a1[qi] = a2[qi] = 0.f;
+        for (int qi = 0; qi < QT; ++qi) {
+            a1[qi] = a2[qi] = 0.f;
+            p1[qi] = p2[qi] = make_float2(0.f, 0.f);
+        }
         if constexpr (Gr::G == 4) {
             // 16-entry tables: the 8 nibbles of a word, pre-scaled to byte offsets 4 e
 #pragma unroll
-            for (int wi = 0; wi < CW; ++wi) add_nibbles<QT, LS::SIZE>(w[wi], tab + 8 * wi * 16, a1);
+            for (int wi = 0; wi < CW; ++wi) add_nibbles<QT, LS::SIZE>(w[wi], tab + 8 * wi * 16, p1);
         } else {
 #pragma unroll
             for (int k = 0; k < NG; ++k) {
@@ -341,10 +345,12 @@ score_lut_kernel(const DevState st, const float* __restrict__ luts, int64_t nq,
         }
         if constexpr (PROD) {
 #pragma unroll
-            for (int wi = 0; wi < NQ / 8; ++wi) add_nibbles<QT, LS::SIZE>(z[wi], tab + LS::MSE + 8 * wi * 16, a2);
+            for (int wi = 0; wi < NQ / 8; ++wi) add_nibbles<QT, LS::SIZE>(z[wi], tab + LS::MSE + 8 * wi * 16, p2);
         }
 #pragma unroll
         for (int qi = 0; qi < QT; ++qi) {
+            a1[qi] += p1[qi].x + p1[qi].y;
+            a2[qi] += p2[qi].x + p2[qi].y;
             if (qi < nqt) {
                 float* dst = scores + (grp * nq + q0 + qi) * n + key;   // key of this group
                 const float v = nu * fmaf(g2, a2[qi], a1[qi]);
