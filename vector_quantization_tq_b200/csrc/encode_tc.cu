@@ -365,15 +365,18 @@ encode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 //   team t: warps 4t .. 4t+3 quantize (warp 4t+q owns TMEM lanes 32q .. 32q+31: one thread
 //   per vector, all 128 coordinates); lane 0 of warp 8+t streams the team's tiles with TMA
 //   (two stages) and issues its MMAs.
-//   TMEM columns of team t: Y_t = [256t, 256t+128) holds y = (H D) x and then S r of the same
-//   tile; HL_t = [256t+128, 256t+256) the residual operand (hi in 64 columns, lo in 64).
-// Per tile: rotation MMA into Y_t; the warps read y twice (||y||^2, then 32 coordinates at a
-// time: level bits, codes, and the residual split r = hi + lo, both bf16, written to HL_t); the
-// S r MMA (16 MMAs: K = 128 for hi, then for lo; A from TMEM) accumulates into Y_t in fp32;
-// the warps read the signs; only then may the team's next rotation overwrite Y_t. The split
-// keeps the error of S r at about 2^-16 |S| |r|, so a sign is decided as fp32 arithmetic on r
-// would decide it. The two producers are coupled so that the teams' quantize passes
-// alternate (one team computes while the other waits for the tensor core).
+//   TMEM columns of team t: two regions of 128, [256t, 256t+128) and [256t+128, 256t+256).
+//   For tile i the region i % 2 (Y) holds y = (H D) x and then S r, the other (HL) the
+//   residual operand (hi in 64 columns, lo in 64); the roles swap every tile (mse keeps y in
+//   the first region).
+// Per tile: rotation MMA into Y; the warps read y twice (||y||^2, then 32 coordinates at a
+// time: level bits, codes, and the residual split r = hi + lo, both bf16, written to HL); the
+// S r MMA (16 MMAs: K = 128 for hi, then for lo; A from TMEM) accumulates into Y in fp32; the
+// warps read the signs. The next tile's rotation goes to this tile's HL region as soon as S r
+// has read it, so it runs while the warps read the signs. The split keeps the error of S r
+// at about 2^-16 |S| |r|, so a sign is decided as fp32 arithmetic on r would decide it. The
+// two producers are coupled so that the teams' quantize passes alternate (one team computes
+// while the other waits for the tensor core).
 // ------------------------------------------------------------------------------------
 constexpr int kDuoThreads = 10 * 32;   // 8 quantizing warps + 2 producer warps
 constexpr uint32_t kDuoCols = 512;
@@ -387,7 +390,7 @@ struct __align__(1024) TcSmemDuo {
     uint64_t bar_y[2];                 // y of the team's current tile is in Y_t
     uint64_t bar_hl[2];                // residual written and y read (one arrival per warp)
     uint64_t bar_d[2];                 // S r is in Y_t
-    uint64_t bar_free[2];              // Y_t read to the end (one arrival per warp)
+    uint64_t bar_free[2];              // mse: Y_t read to the end (one arrival per warp)
     uint64_t bar_mid[2];               // half of the quantize pass done (one arrival per warp)
     uint32_t tmem_base;
     int abort;
@@ -554,7 +557,7 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, co
             const uint32_t idesc = ptx::idesc_bf16_f32(128, 128);
             const uint32_t s_addr = ptx::smem_addr(sm.s);
             const uint32_t hd_addr = ptx::smem_addr(sm.hd);
-            const uint32_t ycol = tmem + 256u * (uint32_t)t, hl = ycol + 128u;
+            const uint32_t tbase = tmem + 256u * (uint32_t)t;
             uint32_t tma_pend = 0u, tma_par = 0u;   // per stage: load in flight / its phase parity
             bool y_issued = false, d_issued = false;
             uint32_t y_par = 0u, d_par = 0u;
@@ -575,8 +578,15 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, co
                 ok = ptx::mbar_wait(&sm.bar_x[t][st], xpar);
                 if (!ok) break;
                 tma_pend &= ~(1u << st);
-                if (i > 0) {   // the warps have read Y_t of the previous tile to the end
-                    ok = ptx::mbar_wait(&sm.bar_free[t], (uint32_t)((i - 1) & 1)) && !*abort_flag;
+                // prod: the team's two regions swap roles every tile (y / S r of tile i in region
+                // i % 2, its residual in the other); the rotation may overwrite region i % 2 as
+                // soon as S r of tile i - 1 (which read it) is done. mse: one region, free once
+                // the warps have read it.
+                const uint32_t ycol = tbase + (PROD ? 128u * (uint32_t)(i & 1) : 0u);
+                const uint32_t hl = tbase + (PROD ? 128u * (uint32_t)((i + 1) & 1) : 128u);
+                if (i > 0) {
+                    ok = ptx::mbar_wait(PROD ? &sm.bar_d[t] : &sm.bar_free[t], (uint32_t)((i - 1) & 1)) &&
+                         !*abort_flag;
                     if (!ok) break;
                 }
                 if constexpr (PROD) {
@@ -637,7 +647,7 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, co
         const int64_t nt = (mytiles > t) ? (mytiles - t + 1) / 2 : 0;
         const int vrow = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t ycol = t_lane + 256u * (uint32_t)t, hlc = ycol + 128u;
+        const uint32_t tbase = t_lane + 256u * (uint32_t)t;
         const int m32 = SPLIT ? gp.m32 : 4;   // chunks of group 0
         bool fail = false;
         // MMA results (read through tcgen05.ld after a tcgen05 fence): one lane waits, and the
@@ -651,6 +661,9 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, co
         };
         for (int64_t i = 0; i < nt; ++i) {
             const int64_t row = (blockIdx.x + (t + 2 * i) * gridDim.x) * kTile + vrow;
+            // y (then S r) and the residual: regions i % 2 and (i + 1) % 2 for prod
+            const uint32_t ycol = tbase + (PROD ? 128u * (uint32_t)(i & 1) : 0u);
+            const uint32_t hlc = tbase + (PROD ? 128u * (uint32_t)((i + 1) & 1) : 128u);
             if (!wait_bar(&sm.bar_y[t], (uint32_t)(i & 1))) {
                 fail = true;
                 break;
@@ -804,9 +817,6 @@ encode_duo_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p, co
                     zw[2 * h] = sign_word(d0);
                     zw[2 * h + 1] = sign_word(d1);
                 }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sm.bar_free[t]);
                 if (row < p.n) {
                     if constexpr (!SPLIT) {
                         *reinterpret_cast<uint4*>(gp.qjl[0] + row * 16) =
