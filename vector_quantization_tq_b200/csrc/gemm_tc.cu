@@ -64,7 +64,8 @@ struct __align__(1024) GemmSmem {
     int abort;
 };
 
-template <int BN, int EPI>
+// BQ: code width of the kRotate epilogue (compile-time, so the code words stay in registers).
+template <int BN, int EPI, int BQ>
 __global__ void __launch_bounds__(kGemmThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                const GemmParams p) {
@@ -166,7 +167,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         dst[j] = make_float4(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1]),
                                              __uint_as_float(acc[4 * j + 2]), __uint_as_float(acc[4 * j + 3]));
                 } else if constexpr (EPI == kRotate) {
-                    const int b = p.b_mse;
+                    constexpr int b = BQ;
                     uint32_t cw[4] = {0u, 0u, 0u, 0u};   // 32 codes of b <= 4 bits
                     uint32_t hi[16], lo[16];
 #pragma unroll
@@ -267,7 +268,7 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64
     return r == CUDA_SUCCESS ? 0 : (int)cudaErrorInvalidValue;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int BQ = 0>
 int run_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, const GemmParams& p, cudaStream_t s) {
     if (p.K % kBK != 0 || p.N % BN != 0) return (int)cudaErrorInvalidValue;
     CUtensorMap ta, tb;
@@ -275,7 +276,7 @@ int run_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, const GemmP
     if (e) return e;
     e = make_map(&tb, B, p.N, p.K, ldb, BN);
     if (e) return e;
-    auto kern = gemm_tc_kernel<BN, EPI>;
+    auto kern = gemm_tc_kernel<BN, EPI, BQ>;
     const size_t smem = sizeof(GemmSmem<BN>) + 1024;
     static int attr_dev = -1;
     int dev = 0;
@@ -377,7 +378,12 @@ int launch_encode_gemm(const DevState& st, const void* x, int64_t n, int64_t ld,
         p.c_cent[i] = (i < st.L) ? st.c[i] : 0.f;
     }
     // y = X Pi^T: B = Pi, row-major [out][in], i.e. K-major in `in`.
-    e = run_gemm<256, kRotate>(x, ld, st.pi, d, p, s);
+    switch (st.b_mse) {
+        case 1: e = run_gemm<256, kRotate, 1>(x, ld, st.pi, d, p, s); break;
+        case 2: e = run_gemm<256, kRotate, 2>(x, ld, st.pi, d, p, s); break;
+        case 3: e = run_gemm<256, kRotate, 3>(x, ld, st.pi, d, p, s); break;
+        default: e = run_gemm<256, kRotate, 4>(x, ld, st.pi, d, p, s); break;
+    }
     if (e || st.mode != TQ_PROD) return e;
     // S r over K = 2d: A = [r_hi | r_lo], B = S reused for both halves of K.
     p.K = 2 * d;
