@@ -114,11 +114,10 @@ def test_c2_prod_rht_kv_keys(tokens):
     qv = synth.bf16_from_bits(qb)
     est = np.stack([qv[h] @ xt_o[h * tokens:(h + 1) * tokens].T for h in range(H)])
     sg = gpu_score(pair, dev_bf16(qb), oplanes, groups=H)[:, 0, :]
-    scale = np.maximum(1.0, np.abs(est))
-    assert np.max(np.abs(sg - est) / scale) <= ABS_SCORE
+    assert np.max(np.abs(sg - est)) <= ABS_SCORE
     sgg = gpu_score(pair, dev_bf16(qb), gplanes, groups=H)[:, 0, :]
     okk = ~bad.reshape(H, tokens)
-    assert np.max((np.abs(sgg - est) / scale)[okk]) <= ABS_SCORE
+    assert np.max(np.abs(sgg - est)[okk]) <= ABS_SCORE
 
 
 # --------------------------------------------------------------------------------------
@@ -219,7 +218,7 @@ def test_general_paths(d, b, mode, rot, md, bf16_in):
     q = synth.gaussian_vectors(11, d, seed=77)
     sg = gpu_score(pair, dev_f32(q), oplanes)[0]
     est = OQ.estimate(q, xt_o)
-    assert np.max(np.abs(sg - est) / np.maximum(1, np.abs(est))) <= ABS_SCORE
+    assert np.max(np.abs(sg - est)) <= ABS_SCORE
 
 
 def test_empty_inputs_are_noops():
