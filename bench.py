@@ -78,22 +78,37 @@ def tensor_peak():
 
 
 def stored_traffic(kernel_key: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if it matches the current source."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
+    """Per-launch DRAM bytes of one kernel from the committed ncu figures (profiles/traffic.json),
+    used only while the kernel's source file hashes to the captured source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         import hashlib
-        for line in open(p):
-            cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) == 5 and cells[0] == kernel_key:
-                src = os.path.join(ROOT, cells[2])
-                if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != cells[3]:
-                    return None
-                return float(cells[4])
+        with open(p) as f:
+            entry = json.load(f).get(kernel_key)
+        if not entry:
+            return None
+        src = os.path.join(ROOT, entry["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != entry["source_sha"]:
+            return None
+        return float(entry["dram_bytes_per_launch"])
     except Exception:
         return None
-    return None
+
+
+def time_on_stream(torch, fn, stream, dev, reps: int, warmup: int) -> float:
+    """Mean milliseconds of fn() over `reps` back-to-back calls, CUDA events on `stream`."""
+    for _ in range(max(3, warmup)):
+        fn()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / reps
 
 
 class ClockSampler:
@@ -218,12 +233,13 @@ def measure_split(tq, torch, x, q, heads, dev, stream, steps: int, warmup: int, 
     sp = tq.Split(so, sr, ch)
     po, pr = sp.empty_planes(nvec, dev)
     scores = torch.empty((heads, 1, TOKENS), dtype=torch.float32, device=dev)
+    sws = torch.empty(max(1, tq.split_score_workspace(sp, tq.BF16, heads, 1)), dtype=torch.uint8, device=dev)
 
     def enc():
         tq.split_quantize(sp, x, po, pr, stream=stream)
 
     def sc():
-        tq.split_score(sp, q, po, pr, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+        tq.split_score(sp, q, po, pr, scores, groups=heads, nq=1, n=TOKENS, stream=stream, workspace=sws)
 
     out = {}
     for name, fn in (("encode", enc), ("score", sc)):
@@ -333,9 +349,10 @@ def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: flo
             enc_flops = 2.0 * d * d * C5_N          # S r (the rotation is O(d log d) adds)
         codes, qjl, norms, rnorms = st.empty_planes(C5_N, dev)
         ws = torch.empty(tq.search_workspace(st, C5_NQ, C5_N, C5_K), dtype=torch.uint8, device=dev)
+        ews = torch.empty(max(1, tq.quantize_workspace(st, C5_N, tq.BF16)), dtype=torch.uint8, device=dev)
 
         def enc():
-            tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
+            tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream, workspace=ews)
 
         def srch():
             tq.search_topk(st, qv, codes, qjl, norms, rnorms, C5_K, idx, vals, ws, stream=stream)
@@ -367,8 +384,19 @@ def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: flo
     return res
 
 
-def oracle_sample(heads: int, seed: int):
-    """The oracle (fp64 numpy) on `heads` heads of the workload; returns (vectors, seconds, threads)."""
+def host_threads():
+    """(cores this process may run on, BLAS threads numpy uses)."""
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        blas = cores
+    return cores, blas
+
+
+def oracle_sample(heads: int, seed: int, single_thread: bool = False):
+    """The oracle (fp64 numpy) on `heads` heads of the workload; returns (vectors, seconds)."""
     from oracle import quantizer as OQ
     from oracle import rotation as OR
     eps = synth.rht_signs(D)
@@ -378,20 +406,128 @@ def oracle_sample(heads: int, seed: int):
     qv = synth.bf16_from_bits(synth.decode_queries(HEADS, D))
     data = [synth.bf16_from_bits(synth.kv_prefill_batch(HEADS, TOKENS, D, seed=seed, head_range=(h, h + 1))[0])
             for h in range(heads)]
+
+    def work():
+        t0 = time.perf_counter()
+        for h in range(heads):
+            codes, z, nu, rho, _, _ = OQ.encode_prod(data[h], Pi, S, cb)
+            OQ.pack_bits(codes, BITS - 1)
+            OQ.pack_bits(z, 1)
+            xt = OQ.decode_prod(codes, z, nu, rho, Pi, S, cb)
+            OQ.estimate(qv[h:h + 1], xt)
+        return time.perf_counter() - t0
+
+    if single_thread:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            return heads * TOKENS, work()
+    return heads * TOKENS, work()
+
+
+def oracle_c5_slice(nvec: int = 65536):
+    """The oracle on a seeded slice of the embedding-search shape (d = 1536, prod b = 2, dense Pi
+    and S bf16): encode + pack of `nvec` vectors, then the estimates of all 1000 queries against
+    them and a top-10; the times extrapolate linearly to 10^6 vectors."""
+    from oracle import attention as OA
+    from oracle import quantizer as OQ
+    from oracle import rotation as OR
+    d = C5_D
+    bits, _ = synth.mixture_vectors(nvec, d)
+    qbits, _ = synth.mixture_vectors(C5_NQ, d, seed=synth.SEED_DATA + 9, centre_seed=synth.SEED_DATA)
+    x, qv = synth.bf16_from_bits(bits), synth.bf16_from_bits(qbits)
+    Pi = OR.round_bf16(OR.haar_from_gaussian(synth.gaussian_matrix(d, 0)))
+    S = OR.round_bf16(synth.gaussian_matrix(d, synth.SEED_S))
+    cb = OQ.make_codebook(d, 1)
     t0 = time.perf_counter()
-    for h in range(heads):
-        codes, z, nu, rho, _, _ = OQ.encode_prod(data[h], Pi, S, cb)
-        OQ.pack_bits(codes, BITS - 1)
-        OQ.pack_bits(z, 1)
-        xt = OQ.decode_prod(codes, z, nu, rho, Pi, S, cb)
-        OQ.estimate(qv[h:h + 1], xt)
-    dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = len(os.sched_getaffinity(0))
-    return heads * TOKENS, dt, threads
+    codes, z, nu, rho, _, _ = OQ.encode_prod(x, Pi, S, cb)
+    OQ.pack_bits(codes, 1)
+    OQ.pack_bits(z, 1)
+    t1 = time.perf_counter()
+    OA.topk(OQ.estimate(qv, OQ.decode_prod(codes, z, nu, rho, Pi, S, cb)), C5_K)
+    t2 = time.perf_counter()
+    scale = C5_N / nvec
+    return {"sample": f"{nvec} of {C5_N} vectors x {d} (same recipe), all {C5_NQ} queries; times x {scale:.2f} "
+                      f"to the full database (linear in the vectors)",
+            "encode_s": t1 - t0, "search_s": t2 - t1, "encode_mvec_s": nvec / (t1 - t0) / 1e6,
+            "search_s_extrapolated": (t2 - t1) * scale, "encode_s_extrapolated": (t1 - t0) * scale}
+
+
+# Parity-size configuration: TurboQuant_mse b = 3, d = 128, 4096 unit vectors (fp32), dense
+# Haar Pi; encode, decode, and 64 unit queries x 4096 estimates. It fits in L2, so only rates
+# are reported.
+C1_N, C1_NQ = 4096, 64
+
+
+def measure_c1(tq, torch, dev, stream, steps: int, warmup: int):
+    d = D
+    st = tq.State(d, 3, tq.MSE, tq.ROT_DENSE, tq.F32, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0))
+    x = torch.from_numpy(synth.unit_vectors(C1_N, d, seed=synth.SEED_DATA)).to(dev)
+    q = torch.from_numpy(synth.unit_vectors(C1_NQ, d, seed=synth.SEED_DATA + 1)).to(dev)
+    codes, _, norms, _ = st.empty_planes(C1_N, dev)
+    xt = torch.empty_like(x)
+    scores = torch.empty((1, C1_NQ, C1_N), dtype=torch.float32, device=dev)
+    sws = torch.empty(max(1, tq.score_workspace(st, 1, C1_NQ)), dtype=torch.uint8, device=dev)
+    reps = max(10, steps)
+    ms = {
+        "encode": time_on_stream(torch, lambda: tq.quantize_mse(st, x, codes, norms, stream=stream), stream, dev,
+                                 reps, warmup),
+        "decode": time_on_stream(torch, lambda: tq.dequant(st, codes, None, norms, None, xt, stream=stream), stream,
+                                 dev, reps, warmup),
+        "score": time_on_stream(torch, lambda: tq.score(st, q, codes, None, norms, None, scores, stream=stream,
+                                                        workspace=sws), stream, dev, reps, warmup),
+    }
+    st.close()
+    return {"workload": "turboquant_mse b=3, d=128, 4096 unit vectors fp32, dense Haar Pi: encode, decode, "
+                        "64 queries x 4096 estimates (fits in L2: rates only, no roofline claim)",
+            "ms": ms, "encode_mvec_s": C1_N / (ms["encode"] / 1e3) / 1e6,
+            "decode_mvec_s": C1_N / (ms["decode"] / 1e3) / 1e6,
+            "score_gpairs_s": C1_N * C1_NQ / (ms["score"] / 1e3) / 1e9}
+
+
+# Distortion / bias sweep: 2^20 uniform unit vectors at d = 128 and 256, b = 1..4, MSE and
+# prod (dense Haar Pi fp32, S fp32), 1024 unit queries; statistics reduced on the device.
+C4_N, C4_NQ = 1 << 20, 1024
+
+
+def measure_c4(tq, torch, dev, stream):
+    import math
+    rows = []
+    for d in (128, 256):
+        g = torch.Generator(device=dev)
+        g.manual_seed(9000 + d)
+        x = torch.randn(C4_N, d, generator=g, device=dev)
+        x /= x.norm(dim=1, keepdim=True)
+        q = torch.randn(C4_NQ, d, generator=g, device=dev)
+        q /= q.norm(dim=1, keepdim=True)
+        xt = torch.empty_like(x)
+        sums = torch.zeros(6, dtype=torch.float64, device=dev)
+        for mode in (tq.MSE, tq.PROD):
+            for b in (1, 2, 3, 4):
+                st = tq.State(d, b, mode, tq.ROT_DENSE, tq.F32, device=dev.index,
+                              gauss_pi=synth.gaussian_matrix(d, 0), s=synth.gaussian_matrix(d, synth.SEED_S))
+                codes, qjl, norms, rnorms = st.empty_planes(C4_N, dev)
+                if mode == tq.MSE:
+                    enc = lambda: tq.quantize_mse(st, x, codes, norms, stream=stream)  # noqa: E731
+                else:
+                    enc = lambda: tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)  # noqa: E731
+                enc_ms = time_on_stream(torch, enc, stream, dev, 3, 1)
+                tq.dequant(st, codes, qjl, norms, rnorms, xt, stream=stream)
+                tq.ip_stats(x, xt, q, sums, device=dev.index, stream=stream)
+                torch.cuda.synchronize(dev)
+                s = sums.cpu().numpy()
+                n_pairs = C4_N * C4_NQ
+                mean_e = s[2] / n_pairs
+                rows.append({"d": d, "b": b, "mode": "mse" if mode == tq.MSE else "prod",
+                             "D_mse": s[0] / C4_N if mode == tq.MSE else None,
+                             "D_mse_theory": st.dmse if mode == tq.MSE else None,
+                             "lower_4^-b": 4.0 ** -b, "upper_sqrt3pi/2_4^-b": math.sqrt(3) * math.pi / 2 * 4.0 ** -b,
+                             "D_prod": s[3] / n_pairs if mode == tq.PROD else None,
+                             "slope": s[4] / s[5], "mean_ip_err": mean_e,
+                             "sd_ip_err": math.sqrt(max(0.0, s[3] / n_pairs - mean_e ** 2)),
+                             "encode_ms": enc_ms, "encode_mvec_s": C4_N / (enc_ms / 1e3) / 1e6})
+                st.close()
+    return {"workload": "distortion / bias sweep: 2^20 uniform unit vectors, d=128 and 256, b=1..4, mse and prod, "
+                        "dense Haar Pi, 1024 unit queries (statistics on the device)", "rows": rows}
 
 
 def run_reference(args, rank, world):
@@ -400,10 +536,11 @@ def run_reference(args, rank, world):
     heads = 4
     for _ in range(args.warmup):
         oracle_sample(heads, synth.SEED_DATA)
-    times, threads = [], 1
+    times = []
     for _ in range(args.steps):
-        n, dt, threads = oracle_sample(heads, synth.SEED_DATA)
+        _, dt = oracle_sample(heads, synth.SEED_DATA)
         times.append(dt)
+    cores, blas = host_threads()
     tot = sum(times)
     value = heads * TOKENS * args.steps / tot / 1e6
     line = {
@@ -411,7 +548,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "sample": f"{heads} of {HEADS} heads per step ({heads * TOKENS} vectors)"},
-        "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": cores, "blas_threads": blas, "kind": "oracle",
                          "sample": f"{heads} heads x {TOKENS} tokens per step, fp64 numpy oracle"},
         "e2e": {"value": value, "unit": "Mvec/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -432,6 +569,8 @@ def main():
     ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
     ap.add_argument("--no-split", action="store_true", help="skip the outlier-channel split measurement")
     ap.add_argument("--no-entropy", action="store_true", help="skip the prefix-coding measurement")
+    ap.add_argument("--no-c1", action="store_true", help="skip the parity-size configuration's rates")
+    ap.add_argument("--no-c4", action="store_true", help="skip the distortion / bias sweep")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -464,10 +603,13 @@ def main():
     codes, qjl, norms, rnorms = st.empty_planes(nvec, dev)
     scores = torch.empty((heads, 1, TOKENS), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    sws = torch.empty(max(1, tq.score_workspace(st, heads, 1)), dtype=torch.uint8, device=dev)
+    assert tq.quantize_workspace(st, nvec, tq.BF16) == 0   # the d = 128 encoder is one pass
 
     def step():
         tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
-        tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+        tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream,
+                 workspace=sws)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -486,7 +628,8 @@ def main():
             ev[i][0].record(stream)
             tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)
             ev[i][1].record(stream)
-            tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+            tq.score(st, q, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream,
+                     workspace=sws)
             ev[i][2].record(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
@@ -516,7 +659,8 @@ def main():
             dx.copy_(hx, non_blocking=True)
             dq.copy_(hq, non_blocking=True)
             tq.quantize_prod(st, dx, codes, qjl, norms, rnorms, stream=stream)
-            tq.score(st, dq, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream)
+            tq.score(st, dq, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream,
+                     workspace=sws)
             hc.copy_(codes, non_blocking=True)
             hz.copy_(qjl, non_blocking=True)
             hn.copy_(norms, non_blocking=True)
@@ -545,10 +689,16 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_s, dt, threads = oracle_sample(8, seed)
-        cpu = {"value": n_s / dt / 1e6, "unit": "Mvec/s", "cores": threads, "kind": "oracle",
+        cores, blas = host_threads()
+        n_s, dt = oracle_sample(8, seed)
+        n1, dt1 = oracle_sample(1, seed, single_thread=True)
+        cpu = {"value": n_s / dt / 1e6, "unit": "Mvec/s", "cores": cores, "blas_threads": blas, "kind": "oracle",
                "sample": f"8 of 32 heads ({n_s} vectors) of the same batch: fp64 numpy encode + pack + decode + "
-                         f"estimate, {dt:.2f} s wall"}
+                         f"estimate, {dt:.2f} s wall, numpy/BLAS on {blas} threads",
+               "single_thread": {"value": n1 / dt1 / 1e6, "unit": "Mvec/s", "cores": 1,
+                                 "sample": f"1 head ({n1} vectors), BLAS limited to 1 thread, {dt1:.2f} s wall"}}
+        if not args.no_c5:
+            cpu["embedding_search_slice"] = oracle_c5_slice()
 
     peak, peak_kind = measured_peaks()
     decode = None
@@ -563,6 +713,8 @@ def main():
     c5 = None
     if not args.no_c5:
         c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak())
+    c1 = None if args.no_c1 else measure_c1(tq, torch, dev, stream, args.steps, args.warmup)
+    c4 = None if args.no_c4 else measure_c4(tq, torch, dev, stream)
     enc_gbs = ENC_BYTES_PER_VEC * nvec / (enc_ms / 1e3) / 1e9
     sc_gbs = SCORE_BYTES_PER_KEY * nvec / (sc_ms / 1e3) / 1e9
     traffic = stored_traffic("encode_prod_d128")
@@ -597,6 +749,8 @@ def main():
         "embedding_search": c5,
         "outlier_split": split,
         "prefix_code": ent,
+        "parity_config": c1,
+        "distortion_sweep": c4,
         "cpu_baseline": cpu,
     }
     if rank == 0:

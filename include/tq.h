@@ -18,8 +18,11 @@
  *     Arguments are validated before any launch; on an error nothing is launched and
  *     no output is touched. tq_status_string() gives the text.
  *   - Pointers named h_* are host pointers; every other buffer pointer is a device
- *     pointer on the state's device. The caller owns all data buffers; the library owns
- *     tq_state objects (free with tq_state_destroy).
+ *     pointer on the state's device. The caller owns all data buffers and workspaces; the
+ *     library owns tq_state and tq_split objects (free with tq_state_destroy /
+ *     tq_split_destroy). Device memory is allocated only when a state or split is created;
+ *     every other call works in the caller's buffers (calls that need scratch space take a
+ *     workspace argument sized by a matching *_workspace query).
  *   - Device work is asynchronous on the given cudaStream_t (passed as void*; NULL is
  *     the legacy default stream). Buffers must stay valid until the stream reaches it.
  *   - A CUDA error seen at launch is returned as TQ_ECUDA; tq_last_cuda_error() gives
@@ -170,21 +173,36 @@ int tq_state_import(const void* h_buf, size_t bytes, int device, tq_state** out)
 int tq_code_layout(const tq_state* st, size_t* code_bytes, size_t* qjl_bytes);
 
 /*
+ * Workspace bytes that tq_quantize_mse / tq_quantize_prod need for n vectors of dtype with
+ * row stride ld (0 when the configuration needs none). Only the d >= 512 tensor-core encoders
+ * (bf16 input with dense bf16 Pi, or with the randomized Hadamard rotation, prod) need one:
+ * between their two passes each vector keeps a bf16 pair per coordinate of its residual and
+ * one partial norm per 256 coordinates, (4 d + 4 d / 256) bytes, for up to 65536 vectors at a
+ * time. A smaller workspace (at least the size for min(n, 128) vectors) is accepted and makes
+ * the encoder take more passes; this call returns the size that gives the fewest.
+ */
+int tq_quantize_workspace(const tq_state* st, int dtype, int64_t n, int64_t ld, size_t* bytes);
+
+/*
  * TurboQuant_mse encode of n vectors x (dtype TQ_F32 / TQ_BF16, row stride ld elements):
  * norms[i] = ||x_i||, y = Pi x_i / ||x_i||, codes = b-bit Lloyd-Max cell of each y_j
  * (the upper cell on a tie), packed as in the layout above. The state must be TQ_MSE.
- * n = 0 is a no-op. Errors: TQ_EINVAL, TQ_ECUDA.
+ * workspace: device memory of ws_bytes (see tq_quantize_workspace; 256-byte aligned; may be
+ * NULL when that size is 0). The library allocates nothing.
+ * n = 0 is a no-op. Errors: TQ_EINVAL, TQ_ENOMEM (workspace below the minimum), TQ_ECUDA.
  */
 int tq_quantize_mse(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
-                    uint8_t* codes, float* norms, void* stream);
+                    uint8_t* codes, float* norms, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * TurboQuant_prod encode (Jump2Paper, Theorem 2): (b-1)-bit MSE codes of y = Pi x/||x||,
  * residual r = y - c[idx] (rotated domain), rnorms[i] = ||r||, qjl bits of sign(S r).
  * The state must be TQ_PROD. A zero vector stores norm 0, the codes of y = 0, r = 0.
+ * workspace as for tq_quantize_mse.
  */
 int tq_quantize_prod(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
-                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* workspace,
+                     size_t ws_bytes, void* stream);
 
 /*
  * Reconstruction Q^{-1}: out[i] = ||x|| Pi^T (c[idx] + ||r|| sqrt(pi/2)/d S^T (2z - 1))
@@ -195,6 +213,13 @@ int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl,
                const float* norms, const float* rnorms, int64_t n, float* out, void* stream);
 
 /*
+ * Workspace bytes that tq_score needs for groups * nq queries: the per-query lookup tables of
+ * the table scorer (d = 32, 64, 96, 128, 256 with 1 to 4 code bits), built once per query;
+ * 0 for the other configurations, whose kernel prepares each query in shared memory.
+ */
+int tq_score_workspace(const tq_state* st, int64_t groups, int64_t nq, size_t* bytes);
+
+/*
  * Inner-product estimates <q, x~> straight from the packed codes, grouped:
  *   queries q [groups][nq][d] (dtype TQ_F32/TQ_BF16, contiguous rows),
  *   keys (codes/qjl/norms/rnorms) [groups][n],
@@ -203,10 +228,12 @@ int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl,
  *   <q, x~> = ||x|| ( sum_j q'_j c[idx_j] + ||r|| sqrt(pi/2)/d sum_j u_j (2 z_j - 1) ).
  * groups = 1 is plain all-pairs scoring; groups = heads with nq = 1 is one decode query
  * per head against that head's keys.
+ * workspace: at least tq_score_workspace() bytes of device memory, 256-byte aligned (NULL
+ * allowed when that size is 0). Errors: TQ_ENOMEM if ws_bytes is too small.
  */
 int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int64_t nq,
              const uint8_t* codes, const uint8_t* qjl, const float* norms, const float* rnorms,
-             int64_t n, float* scores, void* stream);
+             int64_t n, float* scores, void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes that tq_attend_decode needs for H heads and T tokens. */
 int tq_attend_workspace(const tq_state* ks, const tq_state* vs, int H, int64_t T, size_t* bytes);
@@ -231,10 +258,14 @@ int tq_attend_decode(const tq_state* ks, const tq_state* vs, const void* q, int 
  * other allocations, and latency-critical decode loops where an allocation's cost or
  * possible failure is not acceptable. (No counterpart on the reference pages: this is an
  * interface convenience around the decode step above, with the same arguments and result.)
- * The split partials go to a fixed device array of 4 MiB inside the library, which every
- * GPU that loads the library holds until the process exits; the entry point itself
- * allocates nothing. Calls that would need more than 4 MiB of partials
- * (H * splits * (d + 2) * 4 bytes, see tq_attend_workspace) return TQ_EUNSUPPORTED.
+ * The scratch that tq_attend_decode takes from its workspace (the split partials and, for
+ * d = 128 keys at 2 to 4 bits, the per-head query tables) goes to a fixed device array of
+ * 4 MiB inside the library, which every GPU that loads the library holds until the process
+ * exits; the entry point itself allocates nothing. A call is accepted when
+ * tq_attend_workspace(ks, vs, H, T) <= 4 MiB and returns TQ_EUNSUPPORTED otherwise (nothing
+ * is launched). That size grows with H and d, and the number of token splits grows with
+ * the device's SM count, so the largest accepted H differs between GPUs; query
+ * tq_attend_workspace on the device in use.
  * All calls on a device share the array and it keeps the last call's contents, so calls
  * whose work overlaps on the GPU (concurrent streams or threads) race and must be
  * serialised by the caller. The first call on each device looks up the array's device
@@ -375,14 +406,18 @@ int tq_split_quantize(const tq_split* sp, const void* x, int dtype, int64_t n, i
 int tq_split_dequant(const tq_split* sp, const tq_planes* outer, const tq_planes* inner, int64_t n,
                      float* out, void* stream);
 
+/* Workspace bytes that tq_split_score needs: the queries' two channel groups, gathered, and
+   the groups' score tables. */
+int tq_split_score_workspace(const tq_split* sp, int qdtype, int64_t groups, int64_t nq, size_t* bytes);
+
 /*
  * Estimates as tq_score (queries [groups][nq][d], planes [groups][n], scores fp32
- * [groups][nq][n]), summed over the two groups. The queries' channel groups are gathered
- * into a stream-ordered scratch buffer.
+ * [groups][nq][n]), summed over the two groups. workspace: at least tq_split_score_workspace()
+ * bytes, 256-byte aligned. Errors: TQ_ENOMEM if ws_bytes is too small.
  */
 int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups, int64_t nq,
                    const tq_planes* outer, const tq_planes* inner, int64_t n, float* scores,
-                   void* stream);
+                   void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes that tq_split_attend_decode needs for H heads and T tokens. */
 int tq_split_attend_workspace(const tq_split* ks, const tq_split* vs, int H, int64_t T, size_t* bytes);

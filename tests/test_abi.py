@@ -127,11 +127,14 @@ def test_state_create_validation_without_gpu():
 
 def test_null_state_calls_are_rejected():
     lib = tq.lib()
-    assert lib.tq_quantize_mse(None, None, 0, 1, 128, None, None, None) == 1
-    assert lib.tq_quantize_prod(None, None, 0, 1, 128, None, None, None, None, None) == 1
+    assert lib.tq_quantize_mse(None, None, 0, 1, 128, None, None, None, 0, None) == 1
+    assert lib.tq_quantize_prod(None, None, 0, 1, 128, None, None, None, None, None, 0, None) == 1
     assert lib.tq_dequant(None, None, None, None, None, 1, None, None) == 1
-    assert lib.tq_score(None, None, 0, 1, 1, None, None, None, None, 1, None, None) == 1
+    assert lib.tq_score(None, None, 0, 1, 1, None, None, None, None, 1, None, None, 0, None) == 1
     n = ctypes.c_size_t()
+    assert lib.tq_quantize_workspace(None, 0, 1, 128, ctypes.byref(n)) == 1
+    assert lib.tq_score_workspace(None, 1, 1, ctypes.byref(n)) == 1
+    assert lib.tq_split_score_workspace(None, 0, 1, 1, ctypes.byref(n)) == 1
     assert lib.tq_attend_workspace(None, None, 1, 1, ctypes.byref(n)) == 1
     assert lib.tq_search_workspace(None, 1, 1, 1, ctypes.byref(n)) == 1
     assert lib.tq_state_import(None, 0, 0, None) == 1
@@ -155,3 +158,13 @@ def test_prefix_code_table_matches_oracle_without_gpu():
         np.testing.assert_array_equal(ln, oln)
         np.testing.assert_array_equal(w, EN.canonical_codewords(oln))
         assert abs(mean - float(np.sum(p * oln))) < 1e-9
+
+
+def test_workspace_queries_without_gpu():
+    # host-side sizing only: an RHT MSE state holds no device matrices
+    st = tq.State(128, 3, tq.MSE, tq.ROT_RHT, tq.F32, signs=synth.rht_signs(128))
+    assert tq.quantize_workspace(st, 4096, tq.BF16) == 0          # one-pass encoder
+    # 3-bit codes: 64 tables of 6-bit groups (64 entries) per query, fp32
+    assert tq.score_workspace(st, 2, 3) == 2 * 3 * 64 * 64 * 4
+    assert tq.score_workspace(st, 0, 3) == 0
+    st.close()

@@ -21,7 +21,7 @@ __all__ = [
     "TQError", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
     "MSE", "PROD", "ROT_DENSE", "ROT_RHT", "F32", "BF16",
     "build_codebook", "draw_gaussian", "draw_signs", "haar_rotation",
-    "State", "quantize_mse", "quantize_prod", "dequant", "score",
+    "State", "quantize_workspace", "quantize_mse", "quantize_prod", "dequant", "score_workspace", "score",
     "attend_workspace", "attend_decode", "attend_decode_noalloc", "ip_stats", "search_workspace", "search_topk",
 ]
 
@@ -86,10 +86,12 @@ _SIGS = {
     "tq_state_export": (_I, [_P, _P, ctypes.POINTER(_SZ)]),
     "tq_state_import": (_I, [_P, _SZ, _I, ctypes.POINTER(_P)]),
     "tq_code_layout": (_I, [_P, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
-    "tq_quantize_mse": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P]),
-    "tq_quantize_prod": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _P]),
+    "tq_quantize_workspace": (_I, [_P, _I, _I64, _I64, ctypes.POINTER(_SZ)]),
+    "tq_quantize_mse": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "tq_quantize_prod": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
     "tq_dequant": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P]),
-    "tq_score": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
+    "tq_score_workspace": (_I, [_P, _I64, _I64, ctypes.POINTER(_SZ)]),
+    "tq_score": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "tq_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
     "tq_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _SZ, _P]),
     "tq_attend_decode_noalloc": (_I, [_P, _P, _P, _I, _I, _I64, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P]),
@@ -109,7 +111,9 @@ _SIGS = {
     "tq_split_destroy": (None, [_P]),
     "tq_split_quantize": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _P]),
     "tq_split_dequant": (_I, [_P, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _I64, _P, _P]),
-    "tq_split_score": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _I64, _P, _P]),
+    "tq_split_score_workspace": (_I, [_P, _I, _I64, _I64, ctypes.POINTER(_SZ)]),
+    "tq_split_score": (_I, [_P, _P, _I, _I64, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes), _I64, _P, _P,
+                            _SZ, _P]),
     "tq_split_attend_workspace": (_I, [_P, _P, _I, _I64, ctypes.POINTER(_SZ)]),
     "tq_split_attend_decode": (_I, [_P, _P, _P, _I, _I, _I64, ctypes.POINTER(Planes), ctypes.POINTER(Planes),
                                     ctypes.POINTER(Planes), ctypes.POINTER(Planes), ctypes.c_float, _P, _P, _SZ,
@@ -297,20 +301,43 @@ class State:
 
 # ---- device calls ----------------------------------------------------------------------
 
-def quantize_mse(st: State, x, codes, norms, stream=None, n=None, ld=None, dtype=None):
+def _ws(workspace, nbytes, device):
+    """(pointer, size) of a caller workspace; a torch buffer of `nbytes` is made when none is given.
+
+    The library itself never allocates device memory: this is the binding's plumbing, the
+    same as allocating the output planes."""
+    if workspace is not None:
+        return workspace, workspace.numel() * workspace.element_size()
+    if nbytes == 0:
+        return None, 0
+    import torch
+    return torch.empty(nbytes, dtype=torch.uint8, device=torch.device("cuda", device)), nbytes
+
+
+def quantize_workspace(st: State, n: int, dtype: int, ld=None) -> int:
+    out = _SZ()
+    _check(_lib.tq_quantize_workspace(st.handle, dtype, n, st.d if ld is None else ld, ctypes.byref(out)),
+           "tq_quantize_workspace")
+    return out.value
+
+
+def quantize_mse(st: State, x, codes, norms, stream=None, n=None, ld=None, dtype=None, workspace=None):
     n = x.shape[0] if n is None else n
     ld = x.stride(0) if ld is None else ld
     dt = _dtype_code(x) if dtype is None else dtype
-    _check(_lib.tq_quantize_mse(st.handle, _ptr(x), dt, n, ld, _ptr(codes), _ptr(norms), _stream(stream)),
-           "tq_quantize_mse")
+    ws, wsb = _ws(workspace, quantize_workspace(st, n, dt, ld) if workspace is None else 0, st.params.device)
+    _check(_lib.tq_quantize_mse(st.handle, _ptr(x), dt, n, ld, _ptr(codes), _ptr(norms), _ptr(ws), wsb,
+                                _stream(stream)), "tq_quantize_mse")
 
 
-def quantize_prod(st: State, x, codes, qjl, norms, rnorms, stream=None, n=None, ld=None, dtype=None):
+def quantize_prod(st: State, x, codes, qjl, norms, rnorms, stream=None, n=None, ld=None, dtype=None,
+                  workspace=None):
     n = x.shape[0] if n is None else n
     ld = x.stride(0) if ld is None else ld
     dt = _dtype_code(x) if dtype is None else dtype
+    ws, wsb = _ws(workspace, quantize_workspace(st, n, dt, ld) if workspace is None else 0, st.params.device)
     _check(_lib.tq_quantize_prod(st.handle, _ptr(x), dt, n, ld, _ptr(codes), _ptr(qjl), _ptr(norms),
-                                 _ptr(rnorms), _stream(stream)), "tq_quantize_prod")
+                                 _ptr(rnorms), _ptr(ws), wsb, _stream(stream)), "tq_quantize_prod")
 
 
 def dequant(st: State, codes, qjl, norms, rnorms, out, stream=None, n=None):
@@ -319,14 +346,22 @@ def dequant(st: State, codes, qjl, norms, rnorms, out, stream=None, n=None):
                            _stream(stream)), "tq_dequant")
 
 
-def score(st: State, q, codes, qjl, norms, rnorms, scores, groups: int = 1, nq=None, n=None, stream=None):
+def score_workspace(st: State, groups: int, nq: int) -> int:
+    out = _SZ()
+    _check(_lib.tq_score_workspace(st.handle, groups, nq, ctypes.byref(out)), "tq_score_workspace")
+    return out.value
+
+
+def score(st: State, q, codes, qjl, norms, rnorms, scores, groups: int = 1, nq=None, n=None, stream=None,
+          workspace=None):
     """scores[g][i][k] = estimate of <q[g][i], x[g][k]>; q is [groups*nq, d] or [groups, nq, d]."""
     nq = (q.shape[-2] if q.dim() == 3 else q.shape[0] // groups) if nq is None else nq
     n = norms.shape[-1] if n is None else n
     if norms.dim() == 1 and n == norms.shape[0] and groups > 1:
         n = norms.shape[0] // groups
+    ws, wsb = _ws(workspace, score_workspace(st, groups, nq) if workspace is None else 0, st.params.device)
     _check(_lib.tq_score(st.handle, _ptr(q), _dtype_code(q), groups, nq, _ptr(codes), _ptr(qjl), _ptr(norms),
-                         _ptr(rnorms), n, _ptr(scores), _stream(stream)), "tq_score")
+                         _ptr(rnorms), n, _ptr(scores), _ptr(ws), wsb, _stream(stream)), "tq_score")
 
 
 def attend_workspace(ks: State, vs: State, H: int, T: int) -> int:
@@ -461,15 +496,24 @@ def split_dequant(sp: Split, outer_planes, inner_planes, out, stream=None, n=Non
            "tq_split_dequant")
 
 
-def split_score(sp: Split, q, outer_planes, inner_planes, scores, groups: int = 1, nq=None, n=None, stream=None):
+def split_score_workspace(sp: Split, qdtype: int, groups: int, nq: int) -> int:
+    out = _SZ()
+    _check(_lib.tq_split_score_workspace(sp.handle, qdtype, groups, nq, ctypes.byref(out)), "tq_split_score_workspace")
+    return out.value
+
+
+def split_score(sp: Split, q, outer_planes, inner_planes, scores, groups: int = 1, nq=None, n=None, stream=None,
+                workspace=None):
     nq = (q.shape[-2] if q.dim() == 3 else q.shape[0] // groups) if nq is None else nq
     norms = outer_planes[2]
     n = norms.shape[-1] if n is None else n
     if norms.dim() == 1 and n == norms.shape[0] and groups > 1:
         n = norms.shape[0] // groups
     po, pi = _planes(outer_planes), _planes(inner_planes)
+    ws, wsb = _ws(workspace, split_score_workspace(sp, _dtype_code(q), groups, nq) if workspace is None else 0,
+                  sp.outer.params.device)
     _check(_lib.tq_split_score(sp.handle, _ptr(q), _dtype_code(q), groups, nq, ctypes.byref(po), ctypes.byref(pi),
-                               n, _ptr(scores), _stream(stream)), "tq_split_score")
+                               n, _ptr(scores), _ptr(ws), wsb, _stream(stream)), "tq_split_score")
 
 
 def split_attend_workspace(ks: Split, vs: Split, H: int, T: int) -> int:

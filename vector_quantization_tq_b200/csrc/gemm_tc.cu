@@ -73,8 +73,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                         ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBM;
-    const int nt = blockIdx.y;
+    // The N tile varies fastest: the CTAs that share an A tile run together, so A comes from
+    // DRAM once and from L2 for the other N tiles.
+    const int m0 = blockIdx.y * kBM;
+    const int nt = blockIdx.x;
     const int n0 = nt * BN;
     const int ksteps = p.K / kBK;
     constexpr uint32_t kCols = BN;          // power of two >= 32
@@ -286,7 +288,9 @@ int run_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, const GemmP
         if (ce != cudaSuccess) return (int)ce;
         attr_dev = dev;
     }
-    dim3 grid((unsigned)((p.M + kBM - 1) / kBM), (unsigned)(p.N / BN));
+    const int64_t mtiles = (p.M + kBM - 1) / kBM;
+    if (mtiles > 65535) return (int)cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)(p.N / BN), (unsigned)mtiles);
     kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, p);
     return (int)cudaGetLastError();
 }

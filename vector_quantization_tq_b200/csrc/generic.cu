@@ -912,15 +912,22 @@ int launch_gather_rows(const void* q, int dtype, int64_t count, int64_t ldq, con
 }
 
 bool score_lut_supported(const DevState& st);
+size_t score_lut_floats(const DevState& st);
 int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                      const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
-                     float* scores, void* stream);
+                     float* scores, void* ws, void* stream);
+
+size_t score_ws_bytes(const DevState& st, int64_t groups, int64_t nq) {
+    if (!score_lut_supported(st) || groups <= 0 || nq <= 0) return 0;
+    return ((size_t)groups * nq * score_lut_floats(st) * sizeof(float) + 255) & ~(size_t)255;
+}
 
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
-                 float* scores, void* stream) {
+                 float* scores, void* ws, void* stream) {
     if (score_lut_supported(st))
-        return launch_score_lut(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, stream);
+        return launch_score_lut(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, ws,
+                                stream);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t smem = score_smem_bytes(st.d);
     if (smem > 48 * 1024) cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1004,12 +1011,16 @@ namespace {
 size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 }  // namespace
 
-size_t split_attend_ws_bytes(int dk, int dv_outer, int dv, int H, int64_t T) {
+// Layout: scores [H][T] | the queries' channel groups | V partials of each group | the K
+// groups' score tables (one region, used by the two score launches in turn).
+size_t split_attend_ws_bytes(const DevState& ko, const DevState& ki, int dv_outer, int dv, int H, int64_t T) {
     if (H <= 0 || T <= 0) return 0;
     const int sp = attend_splits(H, T);
+    const int dk = ko.d + ki.d;
     return al256((size_t)H * T * sizeof(float)) + al256((size_t)H * dk * sizeof(float)) +
            al256((size_t)H * sp * (dv_outer + 2) * sizeof(float)) +
-           al256((size_t)H * sp * (dv - dv_outer + 2) * sizeof(float));
+           al256((size_t)H * sp * (dv - dv_outer + 2) * sizeof(float)) +
+           std::max(score_ws_bytes(ko, H, 1), score_ws_bytes(ki, H, 1));
 }
 
 int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* kchan, const DevState& vo,
@@ -1030,14 +1041,16 @@ int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* k
     const int nsplit = (int)((T + chunk - 1) / chunk);
     float* part_o = reinterpret_cast<float*>(w);
     float* part_i = reinterpret_cast<float*>(w + al256((size_t)H * sp * (vo.d + 2) * sizeof(float)));
+    void* tables = w + al256((size_t)H * sp * (vo.d + 2) * sizeof(float)) +
+                   al256((size_t)H * sp * (vi.d + 2) * sizeof(float));
     int e = launch_gather_rows(q, qdtype, H, dk, kchan, ko.d, qo, stream);
     if (e == 0) e = launch_gather_rows(q, qdtype, H, dk, kchan + ko.d, ki.d, qi, stream);
     if (e == 0)
         e = launch_score(ko, qo, qdtype, H, 1, kp.codes[0], kp.qjl[0], kp.norms[0], kp.rnorms[0], T, 0, scores,
-                         stream);
+                         tables, stream);
     if (e == 0)
         e = launch_score(ki, qi, qdtype, H, 1, kp.codes[1], kp.qjl[1], kp.norms[1], kp.rnorms[1], T, 1, scores,
-                         stream);
+                         tables, stream);
     if (e != 0) return e;
     for (int g = 0; g < 2; ++g) {
         const DevState& v = g ? vi : vo;

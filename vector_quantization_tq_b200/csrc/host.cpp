@@ -2,6 +2,7 @@
 // The operations are defined in include/tq.h (with the passages they follow).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -460,28 +461,50 @@ int tq_code_layout(const tq_state* st, size_t* code_bytes, size_t* qjl_bytes) {
     return TQ_OK;
 }
 
+int tq_quantize_workspace(const tq_state* st, int dtype, int64_t n, int64_t ld, size_t* bytes) {
+    if (!st || !bytes || n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_EINVAL;
+    *bytes = encode_ws_bytes(st->dev, dtype, n, ld);
+    return TQ_OK;
+}
+
+namespace {
+int check_encode_ws(const tq_state* st, int dtype, int64_t n, int64_t ld, const void* ws, size_t ws_bytes) {
+    const size_t need = encode_ws_min_bytes(st->dev, dtype, n, ld);
+    if (need == 0) return TQ_OK;
+    if (!ws || ((uintptr_t)ws & 255u)) return TQ_EINVAL;
+    return ws_bytes < need ? TQ_ENOMEM : TQ_OK;
+}
+}  // namespace
+
 int tq_quantize_mse(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
-                    uint8_t* codes, float* norms, void* stream) {
+                    uint8_t* codes, float* norms, void* workspace, size_t ws_bytes, void* stream) {
     if (!st || st->p.mode != TQ_MSE) return TQ_EINVAL;
     int rc = check_vectors(st, x, dtype, n, ld);
     if (rc != TQ_OK || n == 0) return rc;
     if (!codes || !norms || !aligned16(codes) || !aligned16(norms)) return TQ_EINVAL;
+    rc = check_encode_ws(st, dtype, n, ld, workspace, ws_bytes);
+    if (rc != TQ_OK) return rc;
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
-    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, nullptr, norms, nullptr, stream));
+    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, nullptr, norms, nullptr,
+                                                  workspace, ws_bytes, stream));
 }
 
 int tq_quantize_prod(const tq_state* st, const void* x, int dtype, int64_t n, int64_t ld,
-                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream) {
+                     uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* workspace, size_t ws_bytes,
+                     void* stream) {
     if (!st || st->p.mode != TQ_PROD) return TQ_EINVAL;
     int rc = check_vectors(st, x, dtype, n, ld);
     if (rc != TQ_OK || n == 0) return rc;
     if ((st->b_mse > 0 && (!codes || !aligned16(codes))) || !qjl || !norms || !rnorms ||
         !aligned16(qjl) || !aligned16(norms) || !aligned16(rnorms))
         return TQ_EINVAL;
+    rc = check_encode_ws(st, dtype, n, ld, workspace, ws_bytes);
+    if (rc != TQ_OK) return rc;
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
-    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, qjl, norms, rnorms, stream));
+    return cuda_status((cudaError_t)launch_encode(st->dev, x, dtype, n, ld, codes, qjl, norms, rnorms, workspace,
+                                                  ws_bytes, stream));
 }
 
 int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
@@ -497,9 +520,15 @@ int tq_dequant(const tq_state* st, const uint8_t* codes, const uint8_t* qjl, con
                                                    prod ? rnorms : nullptr, n, nullptr, st->p.d, out, stream));
 }
 
+int tq_score_workspace(const tq_state* st, int64_t groups, int64_t nq, size_t* bytes) {
+    if (!st || !bytes || groups < 0 || nq < 0) return TQ_EINVAL;
+    *bytes = score_ws_bytes(st->dev, groups, nq);
+    return TQ_OK;
+}
+
 int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int64_t nq,
              const uint8_t* codes, const uint8_t* qjl, const float* norms, const float* rnorms,
-             int64_t n, float* scores, void* stream) {
+             int64_t n, float* scores, void* workspace, size_t ws_bytes, void* stream) {
     if (!st || groups < 0 || nq < 0 || n < 0) return TQ_EINVAL;
     if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
     if (groups == 0 || nq == 0 || n == 0) return TQ_OK;
@@ -508,10 +537,15 @@ int tq_score(const tq_state* st, const void* q, int qdtype, int64_t groups, int6
     if (!q || !scores || !norms || (st->b_mse > 0 && !codes) || (prod && (!qjl || !rnorms)))
         return TQ_EINVAL;
     if (!aligned16(q) || (codes && !aligned16(codes)) || (prod && !aligned16(qjl))) return TQ_EINVAL;
+    const size_t need = score_ws_bytes(st->dev, groups, nq);
+    if (need > 0) {
+        if (!workspace || ((uintptr_t)workspace & 255u)) return TQ_EINVAL;
+        if (ws_bytes < need) return TQ_ENOMEM;
+    }
     DeviceGuard g(st->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
     return cuda_status((cudaError_t)launch_score(st->dev, q, qdtype, groups, nq, codes, prod ? qjl : nullptr,
-                                                 norms, prod ? rnorms : nullptr, n, 0, scores, stream));
+                                                 norms, prod ? rnorms : nullptr, n, 0, scores, workspace, stream));
 }
 
 // ---- prefix coding of the indices -------------------------------------------------------
@@ -729,42 +763,64 @@ int tq_split_dequant(const tq_split* sp, const tq_planes* outer, const tq_planes
     return cuda_status((cudaError_t)e);
 }
 
+namespace {
+// tq_split_score's workspace: the queries' outer channels [rows][m], their inner channels
+// [rows][d - m] (each 256-byte aligned), then one region for the groups' score tables
+// (used by the two score launches in turn).
+size_t split_score_ws(const tq_split* sp, int qdtype, int64_t groups, int64_t nq, size_t* q_inner_off,
+                      size_t* tables_off) {
+    const int m = sp->outer->p.d, r = sp->d - m;
+    const size_t rows = (size_t)groups * nq, es = (qdtype == TQ_F32) ? 4 : 2;
+    const size_t b_out = (rows * m * es + 255) & ~(size_t)255;
+    const size_t b_in = (rows * r * es + 255) & ~(size_t)255;
+    if (q_inner_off) *q_inner_off = b_out;
+    if (tables_off) *tables_off = b_out + b_in;
+    return b_out + b_in + std::max(score_ws_bytes(sp->outer->dev, groups, nq), score_ws_bytes(sp->inner->dev, groups, nq));
+}
+}  // namespace
+
+int tq_split_score_workspace(const tq_split* sp, int qdtype, int64_t groups, int64_t nq, size_t* bytes) {
+    if (!sp || !bytes || groups < 0 || nq < 0 || (qdtype != TQ_F32 && qdtype != TQ_BF16)) return TQ_EINVAL;
+    *bytes = (groups == 0 || nq == 0) ? 0 : split_score_ws(sp, qdtype, groups, nq, nullptr, nullptr);
+    return TQ_OK;
+}
+
 int tq_split_score(const tq_split* sp, const void* q, int qdtype, int64_t groups, int64_t nq,
-                   const tq_planes* outer, const tq_planes* inner, int64_t n, float* scores, void* stream) {
+                   const tq_planes* outer, const tq_planes* inner, int64_t n, float* scores, void* workspace,
+                   size_t ws_bytes, void* stream) {
     if (!sp || groups < 0 || nq < 0 || n < 0) return TQ_EINVAL;
     if (qdtype != TQ_F32 && qdtype != TQ_BF16) return TQ_EINVAL;
     if (groups == 0 || nq == 0 || n == 0) return TQ_OK;
     if (groups > 65535) return TQ_EUNSUPPORTED;
     if (!q || !scores || !aligned16(q) || !planes_ok(sp->outer, outer) || !planes_ok(sp->inner, inner))
         return TQ_EINVAL;
+    size_t q_in_off = 0, tab_off = 0;
+    const size_t need = split_score_ws(sp, qdtype, groups, nq, &q_in_off, &tab_off);
+    if (!workspace || ((uintptr_t)workspace & 255u)) return TQ_EINVAL;
+    if (ws_bytes < need) return TQ_ENOMEM;
     DeviceGuard g(sp->outer->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
-    cudaStream_t s = (cudaStream_t)stream;
     const bool prod = sp->outer->p.mode == TQ_PROD;
     const int m = sp->outer->p.d, r = sp->d - m;
     const int64_t rows = groups * nq;
-    const size_t es = (qdtype == TQ_F32) ? 4 : 2;
-    // [rows][m] then [rows][d - m], each 256-byte aligned
-    const size_t b_out = ((size_t)rows * m * es + 255) & ~(size_t)255;
-    void* qg = nullptr;
-    cudaError_t ce = (cudaError_t)scratch_alloc(&qg, b_out + (size_t)rows * r * es, s);
-    if (ce != cudaSuccess) return cuda_status(ce);
-    void* q_in = reinterpret_cast<unsigned char*>(qg) + b_out;
-    int e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan, m, qg, stream);
+    unsigned char* w = reinterpret_cast<unsigned char*>(workspace);
+    void* q_out = w;
+    void* q_in = w + q_in_off;
+    void* tables = w + tab_off;
+    int e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan, m, q_out, stream);
     if (e == 0) e = launch_gather_rows(q, qdtype, rows, sp->d, sp->d_chan + m, r, q_in, stream);
     if (e == 0)
-        e = launch_score(sp->outer->dev, qg, qdtype, groups, nq, outer->codes, prod ? outer->qjl : nullptr,
-                         outer->norms, prod ? outer->rnorms : nullptr, n, 0, scores, stream);
+        e = launch_score(sp->outer->dev, q_out, qdtype, groups, nq, outer->codes, prod ? outer->qjl : nullptr,
+                         outer->norms, prod ? outer->rnorms : nullptr, n, 0, scores, tables, stream);
     if (e == 0)
         e = launch_score(sp->inner->dev, q_in, qdtype, groups, nq, inner->codes, prod ? inner->qjl : nullptr,
-                         inner->norms, prod ? inner->rnorms : nullptr, n, 1, scores, stream);
-    const cudaError_t fe = (cudaError_t)scratch_free(qg, s);
-    return cuda_status(e ? (cudaError_t)e : fe);
+                         inner->norms, prod ? inner->rnorms : nullptr, n, 1, scores, tables, stream);
+    return cuda_status((cudaError_t)e);
 }
 
 int tq_split_attend_workspace(const tq_split* ks, const tq_split* vs, int H, int64_t T, size_t* bytes) {
     if (!ks || !vs || !bytes || H < 0 || T < 0) return TQ_EINVAL;
-    *bytes = split_attend_ws_bytes(ks->d, vs->outer->p.d, vs->d, H, T);
+    *bytes = split_attend_ws_bytes(ks->outer->dev, ks->inner->dev, vs->outer->p.d, vs->d, H, T);
     return TQ_OK;
 }
 
@@ -783,7 +839,7 @@ int tq_split_attend_decode(const tq_split* ks, const tq_split* vs, const void* q
     if (!planes_ok(ks->outer, k_outer) || !planes_ok(ks->inner, k_inner) || !planes_ok(vs->outer, v_outer) ||
         !planes_ok(vs->inner, v_inner))
         return TQ_EINVAL;
-    const size_t need = split_attend_ws_bytes(ks->d, vs->outer->p.d, vs->d, H, T);
+    const size_t need = split_attend_ws_bytes(ks->outer->dev, ks->inner->dev, vs->outer->p.d, vs->d, H, T);
     if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return TQ_EINVAL;
     DeviceGuard g(ks->outer->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());

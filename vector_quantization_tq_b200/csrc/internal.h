@@ -99,8 +99,13 @@ void paley_hadamard12_rows(uint32_t rows[12]);
 void set_cuda_error(int err);
 
 // ---- kernel launchers (kernels .cu files); all return a cudaError_t value ----
+// Workspace bytes of launch_encode for n vectors (0 when the configuration needs none; with
+// less than this, down to encode_ws_min_bytes, the encoder takes more passes).
+size_t encode_ws_bytes(const DevState& st, int dtype, int64_t n, int64_t ld);
+size_t encode_ws_min_bytes(const DevState& st, int dtype, int64_t n, int64_t ld);
 int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld,
-                  uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
+                  uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* ws, size_t ws_bytes,
+                  void* stream);
 int launch_encode_strided(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, int64_t ostride,
                           uint8_t* codes, uint8_t* qjl, float* norms, float* rnorms, void* stream);
 int launch_encode_channels(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, const int32_t* chan,
@@ -109,10 +114,13 @@ int launch_encode_channels(const DevState& st, const void* x, int dtype, int64_t
 int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl,
                    const float* norms, const float* rnorms, int64_t n, const int32_t* chan, int64_t ldo,
                    float* out, void* stream);
-// accumulate != 0: scores += estimates (else scores = estimates)
+// Workspace bytes of launch_score for groups * nq queries (the per-query lookup tables; 0
+// for the general kernel, which prepares each query in shared memory).
+size_t score_ws_bytes(const DevState& st, int64_t groups, int64_t nq);
+// accumulate != 0: scores += estimates (else scores = estimates); ws: score_ws_bytes, 256-aligned
 int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq,
                  const uint8_t* codes, const uint8_t* qjl, const float* norms,
-                 const float* rnorms, int64_t n, int accumulate, float* scores, void* stream);
+                 const float* rnorms, int64_t n, int accumulate, float* scores, void* ws, void* stream);
 // rows of q [count][ldq] gathered at columns chan[0..m) into out [count][m] (same dtype)
 int launch_gather_rows(const void* q, int dtype, int64_t count, int64_t ldq, const int32_t* chan, int m, void* out,
                        void* stream);
@@ -130,14 +138,11 @@ struct SplitPlanes {
     const float* norms[2];
     const float* rnorms[2];
 };
-size_t split_attend_ws_bytes(int dk, int dv_outer, int dv, int H, int64_t T);
+size_t split_attend_ws_bytes(const DevState& ko, const DevState& ki, int dv_outer, int dv, int H, int64_t T);
 int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* kchan, const DevState& vo,
                         const DevState& vi, const int32_t* vchan, const void* q, int qdtype, int H, int64_t T,
                         const SplitPlanes& kp, const SplitPlanes& vp, float scale, float* out, void* ws,
                         void* stream);
-// Stream-ordered scratch buffers from the library's per-device pool (cudaError_t values).
-int scratch_alloc(void** p, size_t bytes, void* stream);
-int scratch_free(void* p, void* stream);
 int launch_expired_wait(uint64_t limit_ns, void* stream);
 int read_device_error(int* flag);
 int take_device_error_gemm(int* flag);

@@ -375,16 +375,12 @@ int sm_count_lut() {
 template <int D, int B, bool PROD, int QT>
 int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate,
-               float* scores, cudaStream_t s) {
+               float* scores, float* luts, cudaStream_t s) {
     using LS = LutShape<D, B, PROD>;
     const int64_t qtiles = (nq + QT - 1) / QT;
     if (qtiles > 65535 || groups > 65535 || groups * nq > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
-    // Per-query tables in a stream-ordered scratch buffer, built once per query.
-    float* luts = nullptr;
-    cudaError_t ce = (cudaError_t)scratch_alloc(reinterpret_cast<void**>(&luts),
-                                                (size_t)groups * nq * LS::SIZE * sizeof(float), s);
-    if (ce != cudaSuccess) return (int)ce;
-    ce = (cudaError_t)launch_tables<D, B, PROD>(st, q, qdtype, groups * nq, luts, s);
+    // Per-query tables in the caller's workspace, built once per query.
+    cudaError_t ce = (cudaError_t)launch_tables<D, B, PROD>(st, q, qdtype, groups * nq, luts, s);
     if (ce == cudaSuccess) {
         auto kern = score_lut_kernel<D, B, PROD, QT>;
         const size_t smem = (size_t)QT * LS::SIZE * sizeof(float);
@@ -403,35 +399,34 @@ int launch_lut(const DevState& st, const void* q, int qdtype, int64_t groups, in
             ce = cudaGetLastError();
         }
     }
-    cudaError_t fe = (cudaError_t)scratch_free(luts, s);
-    return (int)(ce != cudaSuccess ? ce : fe);
+    return (int)ce;
 }
 
 template <int D, int B, bool PROD>
 int launch_lut_q(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
-                 cudaStream_t s) {
-    if (nq == 1) return launch_lut<D, B, PROD, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-    return launch_lut<D, B, PROD, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+                 float* luts, cudaStream_t s) {
+    if (nq == 1) return launch_lut<D, B, PROD, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+    return launch_lut<D, B, PROD, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
 }
 
 template <int D, int B>
 int launch_lut_m(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
-                 cudaStream_t s) {
-    if (qjl) return launch_lut_q<D, B, true>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-    return launch_lut_q<D, B, false>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+                 float* luts, cudaStream_t s) {
+    if (qjl) return launch_lut_q<D, B, true>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+    return launch_lut_q<D, B, false>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
 }
 
 template <int D>
 int launch_lut_b(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                  const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
-                 cudaStream_t s) {
+                 float* luts, cudaStream_t s) {
     switch (st.b_mse) {
-        case 1: return launch_lut_m<D, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 2: return launch_lut_m<D, 2>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 3: return launch_lut_m<D, 3>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 4: return launch_lut_m<D, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 1: return launch_lut_m<D, 1>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 2: return launch_lut_m<D, 2>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 3: return launch_lut_m<D, 3>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 4: return launch_lut_m<D, 4>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
         default: return (int)cudaErrorInvalidValue;
     }
 }
@@ -467,6 +462,32 @@ int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_
     return launch_tables128_b<false>(st, q, qdtype, count, luts, s);
 }
 
+namespace {
+template <int D>
+size_t lut_floats_d(int b, bool prod) {
+    switch (b) {
+        case 1: return prod ? LutShape<D, 1, true>::SIZE : LutShape<D, 1, false>::SIZE;
+        case 2: return prod ? LutShape<D, 2, true>::SIZE : LutShape<D, 2, false>::SIZE;
+        case 3: return prod ? LutShape<D, 3, true>::SIZE : LutShape<D, 3, false>::SIZE;
+        case 4: return prod ? LutShape<D, 4, true>::SIZE : LutShape<D, 4, false>::SIZE;
+        default: return 0;
+    }
+}
+}  // namespace
+
+// Floats of the lookup tables of one query of the table scorer.
+size_t score_lut_floats(const DevState& st) {
+    const bool prod = st.mode == TQ_PROD;
+    switch (st.d) {
+        case 32: return lut_floats_d<32>(st.b_mse, prod);
+        case 64: return lut_floats_d<64>(st.b_mse, prod);
+        case 96: return lut_floats_d<96>(st.b_mse, prod);
+        case 128: return lut_floats_d<128>(st.b_mse, prod);
+        case 256: return lut_floats_d<256>(st.b_mse, prod);
+        default: return 0;
+    }
+}
+
 bool score_lut_supported(const DevState& st) {
     const bool dim = st.d == 32 || st.d == 64 || st.d == 96 || st.d == 128 || st.d == 256;
     return dim && st.b_mse >= 1 && st.b_mse <= 4;
@@ -474,14 +495,15 @@ bool score_lut_supported(const DevState& st) {
 
 int launch_score_lut(const DevState& st, const void* q, int qdtype, int64_t groups, int64_t nq, const uint8_t* codes,
                      const uint8_t* qjl, const float* norms, const float* rnorms, int64_t n, int accumulate, float* scores,
-                     void* stream) {
+                     void* ws, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
+    float* luts = reinterpret_cast<float*>(ws);
     switch (st.d) {
-        case 32: return launch_lut_b<32>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 64: return launch_lut_b<64>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 96: return launch_lut_b<96>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        case 128: return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
-        default: return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, s);
+        case 32: return launch_lut_b<32>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 64: return launch_lut_b<64>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 96: return launch_lut_b<96>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        case 128: return launch_lut_b<128>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
+        default: return launch_lut_b<256>(st, q, qdtype, groups, nq, codes, qjl, norms, rnorms, n, accumulate, scores, luts, s);
     }
 }
 
