@@ -211,7 +211,71 @@ def measure_decode(tq, torch, dev, stream, steps: int, warmup: int, peak: float)
                         "query per head", "ms": ms, "gkeys_s": n / (ms / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "algorithmic_bytes_per_launch": DEC_BYTES_PER_TOKEN * n},
-            "gpu_launches_per_step": 2}
+            "gpu_launches_per_step": 3}
+
+
+# Streaming decode step: 32 query heads sharing 8 KV heads (G = 4), a cache of 131,072 tokens
+# per KV head (K prod b=4, V mse b=4, dense Pi); each step encodes one new K and V token per
+# KV head into the cache and attends over every token (tq_attend_append_decode).
+STR_H, STR_G, STR_T = 32, 4, 131072
+
+
+def measure_streaming(tq, torch, dev, stream, steps: int, warmup: int, peak: float):
+    """Time tq_attend_append_decode: the per-token append + decode step of a growing cache."""
+    d = D
+    hkv = STR_H // STR_G
+    ks = tq.State(d, 4, tq.PROD, tq.ROT_DENSE, tq.F32, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0),
+                  s=synth.gaussian_matrix(d, synth.SEED_S))
+    vs = tq.State(d, 4, tq.MSE, tq.ROT_DENSE, tq.F32, device=dev.index, gauss_pi=synth.gaussian_matrix(d, 0))
+    nstep = max(3, warmup) + steps
+    t0 = STR_T - nstep   # the cache holds t0 tokens before the first step and STR_T after the last
+    kc, kz, kn, kr = ks.empty_planes(hkv * STR_T, dev)
+    vc, _, vn, _ = vs.empty_planes(hkv * STR_T, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(54321)
+    for h in range(hkv):
+        sl = slice(h * STR_T, h * STR_T + t0)
+        k = torch.randn(t0, d, generator=g, device=dev)
+        v = torch.randn(t0, d, generator=g, device=dev)
+        k /= k.norm(dim=1, keepdim=True)
+        v /= v.norm(dim=1, keepdim=True)
+        tq.quantize_prod(ks, k, kc[sl], kz[sl], kn[sl], kr[sl], stream=stream)
+        tq.quantize_mse(vs, v, vc[sl], vn[sl], stream=stream)
+    qs = torch.randn(nstep, STR_H, d, generator=g, device=dev).to(torch.bfloat16)
+    knew = torch.randn(nstep, hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    vnew = torch.randn(nstep, hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((STR_H, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.attend_workspace(ks, vs, STR_H, STR_T), dtype=torch.uint8, device=dev)
+    scale = 1.0 / d ** 0.5
+
+    def run(i):
+        tq.attend_append_decode(ks, vs, qs[i], STR_G, knew[i], vnew[i], t0 + i, STR_T, kc, kz, kn, kr, vc, vn, scale,
+                                out, ws, stream=stream)
+
+    nw = max(3, warmup)
+    for i in range(nw):
+        run(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(nw, nstep):
+        run(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    tmean = t0 + nw + (steps + 1) / 2.0   # tokens attended per step, on average
+    # the method must read every KV head's compressed cache once per step and write the new rows
+    nbytes = hkv * tmean * DEC_BYTES_PER_TOKEN + hkv * (DEC_BYTES_PER_TOKEN + 2 * 2 * d) + STR_H * (2 + 4) * d
+    gbs = nbytes / (ms / 1e3) / 1e9
+    ks.close()
+    vs.close()
+    return {"workload": "streaming decode step: 32 query heads over 8 KV heads (GQA 4), 131,072-token cache, d=128, "
+                        "K prod b=4, V mse b=4 (dense Pi); one new K/V token per KV head encoded into the cache, "
+                        "then attention over every token", "ms": ms, "steps_per_s": 1e3 / ms,
+            "head_tokens_gkeys_s": STR_H * tmean / (ms / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "algorithmic_bytes_per_launch": nbytes},
+            "gpu_launches_per_step": 3}
 
 
 # Outlier-channel split of the same KV key batch: the 32 channels of largest mean square
@@ -566,6 +630,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=HEADS, help="smaller batch for profiling runs")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
+    ap.add_argument("--no-stream", action="store_true", help="skip the streaming append + decode measurement")
     ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
     ap.add_argument("--no-split", action="store_true", help="skip the outlier-channel split measurement")
     ap.add_argument("--no-entropy", action="store_true", help="skip the prefix-coding measurement")
@@ -704,6 +769,9 @@ def main():
     decode = None
     if not args.no_decode:
         decode = measure_decode(tq, torch, dev, stream, args.steps, args.warmup, peak)
+    streaming = None
+    if not args.no_stream:
+        streaming = measure_streaming(tq, torch, dev, stream, args.steps, args.warmup, peak)
     split = None
     if not args.no_split:
         split = measure_split(tq, torch, x, q, heads, dev, stream, args.steps, args.warmup, peak)
@@ -746,6 +814,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": e2e,
         "decode_attention": decode,
+        "streaming_step": streaming,
         "embedding_search": c5,
         "outlier_split": split,
         "prefix_code": ent,

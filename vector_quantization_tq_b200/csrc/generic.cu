@@ -975,16 +975,28 @@ size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T) {
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H, int64_t T, int G,
                   int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
                   const uint8_t* vcodes, const float* vnorms, float scale, float* out, void* ws, size_t ws_bytes,
-                  void* stream) {
+                  void* stream, const AppendRow* app) {
     cudaStream_t s = (cudaStream_t)stream;
     const int sp = attend_splits(H, T);
     const int64_t chunk = (T + sp - 1) / sp;
     const int nsplit = (int)((T + chunk - 1) / chunk);
     float* part = reinterpret_cast<float*>(ws);
     cudaError_t e;
-    if (attend_lut_supported(ks, vs, kcodes, kqjl, vcodes)) {
+    const bool lut = attend_lut_supported(ks, vs, kcodes, kqjl, vcodes);
+    if (app && !lut) {
+        // the general path appends with the general encoder, one launch per plane set
+        const int Hkv = H / G;
+        e = (cudaError_t)launch_encode_strided(ks, app->k_new, app->dtype, Hkv, ks.d, Tcap, app->kcodes, app->kqjl,
+                                               app->knorms, app->krnorms, stream);
+        if (e == cudaSuccess)
+            e = (cudaError_t)launch_encode_strided(vs, app->v_new, app->dtype, Hkv, vs.d, Tcap, app->vcodes,
+                                                   app->vqjl, app->vnorms, app->vrnorms, stream);
+        if (e != cudaSuccess) return (int)e;
+    }
+    if (lut) {
         float* luts = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ws) + attend_part_bytes(ks, H, T));
-        e = (cudaError_t)launch_query_tables128(ks, q, qdtype, H, luts, stream);
+        e = app ? (cudaError_t)launch_append_tables128(ks, vs, q, qdtype, H, luts, *app, stream)
+                : (cudaError_t)launch_query_tables128(ks, q, qdtype, H, luts, stream);
         if (e == cudaSuccess)
             e = (cudaError_t)launch_attend_lut_split(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms,
                                                      krnorms, vcodes, vnorms, scale, part, stream);

@@ -938,19 +938,22 @@ int tq_attend_append_decode(const tq_state* ks, const tq_state* vs, const void* 
     DeviceGuard g(ks->p.device);
     if (!g.ok) return cuda_status(cudaGetLastError());
     const bool prod = ks->p.mode == TQ_PROD;
-    const int Hkv = H / G, d = ks->p.d;
-    // 1. the new token of every KV head into row T of that head's planes
-    int e = launch_encode_strided(ks->dev, k_new, kvdtype, Hkv, d, Tcap,
-                                  kcodes ? kcodes + T * ks->dev.code_bytes : nullptr,
-                                  prod ? kqjl + T * ks->dev.qjl_bytes : nullptr, knorms + T,
-                                  prod ? krnorms + T : nullptr, stream);
-    if (e == 0)
-        e = launch_encode_strided(vs->dev, v_new, kvdtype, Hkv, d, Tcap, vcodes + T * vs->dev.code_bytes, nullptr,
-                                  vnorms + T, nullptr, stream);
-    // 2. attention over the T + 1 tokens
-    if (e == 0)
-        e = launch_attend(ks->dev, vs->dev, q, qdtype, H, T + 1, G, Tcap, kcodes, prod ? kqjl : nullptr, knorms,
-                          prod ? krnorms : nullptr, vcodes, vnorms, scale, out, workspace, ws_bytes, stream);
+    // the new token of every KV head goes into row T of that head's planes inside the decode
+    // step (d = 128: by the launch that builds the query tables), then attention over T + 1
+    AppendRow app = {};
+    app.k_new = k_new;
+    app.v_new = v_new;
+    app.dtype = kvdtype;
+    app.G = G;
+    app.Tcap = Tcap;
+    app.kcodes = kcodes ? kcodes + T * ks->dev.code_bytes : nullptr;
+    app.kqjl = prod ? kqjl + T * ks->dev.qjl_bytes : nullptr;
+    app.knorms = knorms + T;
+    app.krnorms = prod ? krnorms + T : nullptr;
+    app.vcodes = vcodes + T * vs->dev.code_bytes;
+    app.vnorms = vnorms + T;
+    const int e = launch_attend(ks->dev, vs->dev, q, qdtype, H, T + 1, G, Tcap, kcodes, prod ? kqjl : nullptr, knorms,
+                                prod ? krnorms : nullptr, vcodes, vnorms, scale, out, workspace, ws_bytes, stream, &app);
     return cuda_status((cudaError_t)e);
 }
 

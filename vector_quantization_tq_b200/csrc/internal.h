@@ -150,15 +150,35 @@ int take_device_error_search(int* flag);
 int launch_ip_stats(const float* x, const float* xt, int64_t n, int d, const float* q, int64_t nq, double* out,
                     void* stream);
 size_t attend_workspace_bytes(const DevState& ks, int H, int64_t T);
+// The new token of a streaming decode step: row 0 of KV head g's planes is at g * Tcap rows
+// from the pointers (already offset to the appended row); k_new / v_new are [H / G][d].
+struct AppendRow {
+    const void* k_new;
+    const void* v_new;
+    int dtype;          // of k_new / v_new
+    int G;              // query heads per KV head
+    int64_t Tcap;
+    uint8_t* kcodes;
+    uint8_t* kqjl;
+    float* knorms;
+    float* krnorms;
+    uint8_t* vcodes;
+    uint8_t* vqjl;
+    float* vnorms;
+    float* vrnorms;
+};
+int launch_append_tables128(const DevState& ks, const DevState& vs, const void* q, int qdtype, int64_t count,
+                            float* luts, const AppendRow& app, void* stream);
 // Per-query lookup tables of the d = 128 scorers (rotated query against code groups, and
 // QJL nibbles): floats per query, and a launch building them for `count` query rows.
 size_t query_table_floats(const DevState& st);
 int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, void* stream);
 // H query heads, G of them per KV head; the planes of KV head g start at row g * Tcap
+// app (optional): encode the new token of every KV head into its row before attending
 int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdtype, int H,
                   int64_t T, int G, int64_t Tcap, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
                   const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale,
-                  float* out, void* ws, size_t ws_bytes, void* stream);
+                  float* out, void* ws, size_t ws_bytes, void* stream, const AppendRow* app = nullptr);
 int attend_static_scratch(void** out);
 size_t search_workspace_bytes(const DevState& st, int64_t nq, int64_t n, int k);
 int launch_search(const DevState& st, const void* q, int qdtype, int64_t nq,

@@ -130,9 +130,110 @@ __device__ __forceinline__ void matvec128(const unsigned char* MT, int dtype, co
     __syncthreads();
 }
 
-template <int B, bool PROD>
+// Sylvester Walsh-Hadamard transform of the 128 values in src (signs eps applied first), times
+// 1/sqrt(d), into dst: one warp, lane l holding elements 4l .. 4l+3; stages h = 1, 2 in
+// registers, h >= 4 across lanes.
+__device__ __forceinline__ void warp_rht128(const DevState& st, const float* src, float* dst) {
+    const int l = threadIdx.x & 31;
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = rht_neg(st, 4 * l + i) ? -src[4 * l + i] : src[4 * l + i];
+#pragma unroll
+    for (int h = 1; h < 4; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+        }
+    }
+#pragma unroll
+    for (int hl = 1; hl < 32; hl <<= 1) {
+        const bool upper = (l & hl) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[i], hl);
+            v[i] = upper ? o - v[i] : v[i] + o;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[4 * l + i] = v[i] * st.rsqrt_d;
+}
+
+// One vector x of d = 128 encoded by the whole block (TurboQuant review, Theorem 1 and
+// Definition 1 / Theorem 2): ||x||; y = Pi x / ||x||; code_j = #{k : t_k <= y_j}; prod: the
+// residual r = y - c[code], ||r|| and the signs [(S r)_j >= 0]; codes packed LSB-first.
+// piT / sT are the state's transposed matrices (row-major 128 x 128, in shared or global
+// memory). The state has at most 16 levels. buf: 5 x 128 + 8 floats, cb: 128 bytes, both in
+// shared memory. Every thread of the block calls this.
+__device__ void block_encode128(const DevState& st, const void* x, int dtype, const unsigned char* piT,
+                                const unsigned char* sT, uint8_t* codes, uint8_t* qjl, float* norm, float* rnorm,
+                                float* buf, uint8_t* cb) {
+    float* xs = buf;
+    float* ys = xs + kD128;
+    float* part = ys + kD128;   // 2 x 128
+    float* red = part + 2 * kD128;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float xv = 0.f;
+    if (tid < kD128) {
+        xv = (dtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(x) + tid)
+                               : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(x) + tid));
+        xs[tid] = xv;
+    }
+    const float ss = warp_sum(xv * xv);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    const float nu = sqrtf((red[0] + red[1]) + (red[2] + red[3]));
+    if (st.rot == TQ_ROT_RHT) {
+        if (warp == 0) warp_rht128(st, xs, ys);
+        __syncthreads();
+    } else {
+        matvec128(piT, st.mat_dtype, xs, part, ys);
+    }
+    const float sc = (nu > 0.f) ? 1.f / nu : 0.f;
+    float r = 0.f;
+    if (tid < kD128) {
+        const float y = ys[tid] * sc;
+        const int c = (st.b_mse > 0) ? quantize_coord(st, nullptr, y) : 0;
+        cb[tid] = (uint8_t)c;
+        r = (nu > 0.f) ? (y - (st.b_mse > 0 ? st.c[c] : 0.f)) : 0.f;
+        xs[tid] = r;
+    }
+    const float rr = warp_sum(r * r);
+    if (lane == 0) red[4 + warp] = rr;   // the norm was read before the rotation's barriers
+    __syncthreads();
+    if (tid == 0) {
+        *norm = nu;
+        if (st.mode == TQ_PROD) *rnorm = sqrtf((red[4] + red[5]) + (red[6] + red[7]));
+    }
+    if (st.mode == TQ_PROD) {
+        matvec128(sT, st.mat_dtype, xs, part, ys);   // ys = S r
+        if (tid < kD128) {
+            const uint32_t z = __ballot_sync(0xffffffffu, ys[tid] >= 0.f);
+            if (lane == 0) reinterpret_cast<uint32_t*>(qjl)[warp] = z;
+        }
+    }
+    // stream bit p = 32 w + lane holds bit p % b of code p / b
+    const int b = st.b_mse;
+    for (int w = warp; w < b * kD128 / 32; w += kThreads / 32) {
+        const int p = 32 * w + lane;
+        const int j = p / b;
+        const uint32_t word = __ballot_sync(0xffffffffu, (cb[j] >> (p - j * b)) & 1u);
+        if (lane == 0) reinterpret_cast<uint32_t*>(codes)[w] = word;
+    }
+    __syncthreads();
+}
+
+// Per query (block) the lookup tables of q' = Pi q against the code groups and of u = S q'
+// against the QJL nibbles. APPEND (a decode step that appends one token): the first query
+// head of each group of G also encodes the new K and V vectors of its KV head into row T of
+// that head's planes, before the attention launch that reads them.
+template <int B, bool PROD, bool APPEND>
 __global__ void __launch_bounds__(kThreads)
-tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts) {
+tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts,
+                 const DevState vs, const AppendRow app) {
     using Gr = Groups<B>;
     using LS = LutShape<kD128, B, PROD>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -155,38 +256,27 @@ tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, floa
                                    : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + qi * kD128 + i));
     }
     __syncthreads();
+    if constexpr (APPEND) {
+        if (qi % app.G == 0) {
+            const int64_t g = qi / app.G;   // KV head
+            const size_t es = (app.dtype == TQ_F32) ? 4 : 2;
+            float* buf = part + 2 * kD128;
+            uint8_t* cb = reinterpret_cast<uint8_t*>(buf + 5 * kD128 + 8);
+            const int64_t row = g * app.Tcap;
+            block_encode128(st, reinterpret_cast<const unsigned char*>(app.k_new) + g * kD128 * es, app.dtype, m0, m1,
+                            app.kcodes + row * st.code_bytes, PROD ? app.kqjl + row * st.qjl_bytes : nullptr,
+                            app.knorms + row, PROD ? app.krnorms + row : nullptr, buf, cb);
+            block_encode128(vs, reinterpret_cast<const unsigned char*>(app.v_new) + g * kD128 * es, app.dtype,
+                            reinterpret_cast<const unsigned char*>(vs.piT), reinterpret_cast<const unsigned char*>(vs.sT),
+                            app.vcodes + row * vs.code_bytes,
+                            vs.mode == TQ_PROD ? app.vqjl + row * vs.qjl_bytes : nullptr, app.vnorms + row,
+                            vs.mode == TQ_PROD ? app.vrnorms + row : nullptr, buf, cb);
+        }
+    }
     if (dense) {
         matvec128(m0, st.mat_dtype, qs, part, qp);
     } else {
-        if (threadIdx.x < 32) {
-            // lane l holds elements 4l .. 4l+3; stages h = 1, 2 in registers, h >= 4 across lanes
-            const int l = threadIdx.x;
-            float v[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = rht_neg(st, 4 * l + i) ? -qs[4 * l + i] : qs[4 * l + i];
-#pragma unroll
-            for (int h = 1; h < 4; h <<= 1) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if ((i & h) == 0) {
-                        const float a = v[i], b = v[i + h];
-                        v[i] = a + b;
-                        v[i + h] = a - b;
-                    }
-                }
-            }
-#pragma unroll
-            for (int hl = 1; hl < 32; hl <<= 1) {
-                const bool upper = (l & hl) != 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float o = __shfl_xor_sync(0xffffffffu, v[i], hl);
-                    v[i] = upper ? o - v[i] : v[i] + o;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) qp[4 * l + i] = v[i] * st.rsqrt_d;
-        }
+        if (threadIdx.x < 32) warp_rht128(st, qs, qp);
         __syncthreads();
     }
     if (PROD) matvec128(m1, st.mat_dtype, qp, part, u);
@@ -213,9 +303,12 @@ tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, floa
     }
 }
 
-size_t tables128_smem(const DevState& st) {
+// Shared memory of tables128_kernel: the two staged matrices, the level table, q, q', u and
+// the matrix-vector halves, then (appending) the block encoder's buffers.
+size_t tables128_smem(const DevState& st, bool append) {
     const size_t mbytes = (size_t)kD128 * kD128 * (st.mat_dtype == TQ_F32 ? 4 : 2);
-    return 2 * mbytes + (size_t)(kMaxLevels + 5 * kD128) * sizeof(float);
+    const size_t base = 2 * mbytes + (size_t)(kMaxLevels + 5 * kD128) * sizeof(float);
+    return append ? base + (5 * kD128 + 8) * sizeof(float) + kD128 : base;
 }
 
 // Tables of `count` queries (rows of q) into luts[count][SIZE].
@@ -224,13 +317,13 @@ int launch_tables(const DevState& st, const void* q, int qdtype, int64_t count, 
     if (count <= 0) return 0;
     if (count > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
     if constexpr (D == kD128) {
-        auto k = tables128_kernel<B, PROD>;
-        const size_t smem = tables128_smem(st);
+        auto k = tables128_kernel<B, PROD, false>;
+        const size_t smem = tables128_smem(st, false);
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return (int)e;
         }
-        k<<<(unsigned)count, kThreads, smem, s>>>(st, q, qdtype, luts);
+        k<<<(unsigned)count, kThreads, smem, s>>>(st, q, qdtype, luts, st, AppendRow{});
     } else {
         auto k = score_prep_kernel<D, B, PROD>;
         const size_t smem = (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
@@ -460,6 +553,42 @@ int launch_query_tables128(const DevState& st, const void* q, int qdtype, int64_
     cudaStream_t s = (cudaStream_t)stream;
     if (st.mode == TQ_PROD) return launch_tables128_b<true>(st, q, qdtype, count, luts, s);
     return launch_tables128_b<false>(st, q, qdtype, count, luts, s);
+}
+
+namespace {
+template <int B, bool PROD>
+int launch_append_tables(const DevState& ks, const DevState& vs, const void* q, int qdtype, int64_t count,
+                         float* luts, const AppendRow& app, cudaStream_t s) {
+    auto k = tables128_kernel<B, PROD, true>;
+    const size_t smem = tables128_smem(ks, true);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+    }
+    k<<<(unsigned)count, kThreads, smem, s>>>(ks, q, qdtype, luts, vs, app);
+    return (int)cudaGetLastError();
+}
+
+template <bool PROD>
+int launch_append_tables_b(const DevState& ks, const DevState& vs, const void* q, int qdtype, int64_t count,
+                           float* luts, const AppendRow& app, cudaStream_t s) {
+    switch (ks.b_mse) {
+        case 2: return launch_append_tables<2, PROD>(ks, vs, q, qdtype, count, luts, app, s);
+        case 3: return launch_append_tables<3, PROD>(ks, vs, q, qdtype, count, luts, app, s);
+        case 4: return launch_append_tables<4, PROD>(ks, vs, q, qdtype, count, luts, app, s);
+        default: return (int)cudaErrorInvalidValue;
+    }
+}
+}  // namespace
+
+// The query tables of `count` heads, the first head of each group of app.G also appending the
+// new K and V token of its KV head (d = 128, key and value codes of 2 to 4 bits).
+int launch_append_tables128(const DevState& ks, const DevState& vs, const void* q, int qdtype, int64_t count,
+                            float* luts, const AppendRow& app, void* stream) {
+    if (ks.d != 128 || vs.d != 128 || ks.L > 16 || vs.L > 16 || app.G <= 0) return (int)cudaErrorInvalidValue;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ks.mode == TQ_PROD) return launch_append_tables_b<true>(ks, vs, q, qdtype, count, luts, app, s);
+    return launch_append_tables_b<false>(ks, vs, q, qdtype, count, luts, app, s);
 }
 
 namespace {
