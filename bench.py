@@ -385,10 +385,12 @@ def measure_entropy(tq, torch, dev, stream, steps: int, warmup: int):
 C5_N, C5_D, C5_NQ, C5_K = 1_000_000, 1536, 1000, 10
 
 
-def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: float):
+def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: float, n: int = None):
     """Time the tensor-core encode and the top-10 search on the embedding-search shape, with the
-    dense Haar Pi and with the randomized Hadamard Pi (order 1536 = 12 x 128; S stays Gaussian)."""
+    dense Haar Pi and with the randomized Hadamard Pi (order 1536 = 12 x 128; S stays Gaussian).
+    n: database size (default the full 1,000,000; a smaller n is for profiling captures)."""
     d = C5_D
+    C5_N = globals()["C5_N"] if n is None else n
     g = torch.Generator(device=dev)
     g.manual_seed(4242)
     mu = torch.randn(256, d, generator=g, device=dev)
@@ -441,7 +443,7 @@ def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: flo
         out["encode"]["mvec_s"] = C5_N / (out["encode"]["ms"] / 1e3) / 1e6
         st.close()
         res["dense" if rot == tq.ROT_DENSE else "rht"] = out
-    res["dense"]["workload"] = ("embedding search: 1,000,000 x 1536 bf16 (Gaussian mixture, 256 centres), prod b=2, "
+    res["dense"]["workload"] = (f"embedding search: {C5_N:,} x 1536 bf16 (Gaussian mixture, 256 centres), prod b=2, "
                                 "dense Pi and S bf16 (tensor cores), 1000 queries, top-10")
     res["rht"]["workload"] = ("the same with Pi = H_1536 diag(eps) / sqrt(1536), H_1536 = H_12 (x) H_128 (CUDA cores), "
                               "S Gaussian bf16 (tensor cores)")
@@ -632,6 +634,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
     ap.add_argument("--no-stream", action="store_true", help="skip the streaming append + decode measurement")
     ap.add_argument("--no-c5", action="store_true", help="skip the embedding-search measurement")
+    ap.add_argument("--c5-keys", type=int, default=None, help="embedding database size (profiling runs)")
     ap.add_argument("--no-split", action="store_true", help="skip the outlier-channel split measurement")
     ap.add_argument("--no-entropy", action="store_true", help="skip the prefix-coding measurement")
     ap.add_argument("--no-c1", action="store_true", help="skip the parity-size configuration's rates")
@@ -780,7 +783,7 @@ def main():
         ent = measure_entropy(tq, torch, dev, stream, args.steps, args.warmup)
     c5 = None
     if not args.no_c5:
-        c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak())
+        c5 = measure_c5(tq, torch, dev, stream, args.steps, args.warmup, tensor_peak(), n=args.c5_keys)
     c1 = None if args.no_c1 else measure_c1(tq, torch, dev, stream, args.steps, args.warmup)
     c4 = None if args.no_c4 else measure_c4(tq, torch, dev, stream)
     enc_gbs = ENC_BYTES_PER_VEC * nvec / (enc_ms / 1e3) / 1e9

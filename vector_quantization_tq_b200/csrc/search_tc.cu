@@ -11,7 +11,8 @@
 //               columns [0, 256), the next d accumulate <u, s> in [256, 512);
 //   warps 2-5   epilogue: one query per thread, est for 256 keys, running top-16 in registers;
 //   warps 6-9   expanders: each K-step's 64 bits per key become 64 bf16 +-1 values in shared
-//               memory (a 256-entry byte table gives 8 values per lookup).
+//               memory (arithmetic: one multiply and one logic op per pair of values), with the
+//               key bits fetched a few steps ahead.
 // Each CTA writes its k best (value, index) per query; a merge launch picks the final k.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -55,7 +56,6 @@ struct SearchParams {
 struct __align__(1024) SearchSmem {
     uint8_t a[kStages][kBM * kBK * 2];   // queries, 128B-swizzled (TMA)
     uint8_t b[kStages][kBN * kBK * 2];   // keys as +-1, K-major core matrices
-    uint4 lut[256];                      // byte -> 8 bf16 values (+1 for a set bit)
     float nu[kBN];
     float g2[kBN];
     uint64_t afull[kStages];
@@ -99,23 +99,13 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         ptx::prefetch_tmap(&tma_q);
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&sm.afull[s], 1);
-            ptx::mbar_init(&sm.bfull[s], 1);
+            ptx::mbar_init(&sm.bfull[s], 4);   // one arrival per expander warp
             ptx::mbar_init(&sm.empty[s], 1);
         }
         ptx::mbar_init(&sm.done, 1);
         ptx::mbar_init(&sm.tfree, 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
-    }
-    for (int i = threadIdx.x; i < 256; i += kThreads) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t lo = ((i >> (2 * q)) & 1) ? 0x3F80u : 0xBF80u;
-            const uint32_t hi = ((i >> (2 * q + 1)) & 1) ? 0x3F80u : 0xBF80u;
-            w[q] = lo | (hi << 16);
-        }
-        sm.lut[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&sm.tmem_base, 512);
@@ -180,44 +170,75 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         }
     } else if (warp >= 6) {
         // ---- expanders: key bits -> +-1 bf16 ----
+        // K-step g of the CTA (tile tile_begin + g / ks_per_tile, step g % ks_per_tile) needs 8
+        // bytes of one bit plane for each of the tile's 256 keys; each thread handles two keys.
+        // The global loads run kPrefetch steps ahead of the expansion, so their latency overlaps
+        // the work of the steps in between.
+        constexpr int kPrefetch = 4;
         const int e = threadIdx.x - 6 * 32;   // 0..127
-        int64_t g = 0;
-        bool stop = false;
-        for (int64_t t = tile_begin; t < tile_end; ++t) {
-            for (int ks = 0; ks < ks_per_tile; ++ks, ++g) {
-                const int s = (int)(g % kStages);
-                const int64_t r = g / kStages;
-                bool ok = true;
-                if (e == 0 && r > 0) ok = ptx::mbar_wait(&sm.empty[s], (uint32_t)((r - 1) & 1));
-                if (e == 0 && !ok) atomicExch(&sm.abort, 1);
-                if (named_sync_or(1, 128, e == 0 && (!ok || sm.abort))) {
-                    stop = true;
-                    break;
-                }
-                const uint8_t* plane = (ks < ks_half) ? p.codes : p.qjl;
-                const int byte0 = ((ks < ks_half) ? ks : ks - ks_half) * (kBK / 8);
+        const int64_t nsteps = (tile_end - tile_begin) * ks_per_tile;
+        auto fetch = [&](int64_t g, uint2 (&bits)[2]) {
+            bits[0] = bits[1] = make_uint2(0u, 0u);
+            if (g >= nsteps) return;
+            const int64_t t = tile_begin + g / ks_per_tile;
+            const int ks = (int)(g % ks_per_tile);
+            const uint8_t* plane = (ks < ks_half) ? p.codes : p.qjl;
+            const int byte0 = ((ks < ks_half) ? ks : ks - ks_half) * (kBK / 8);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int nl = e + h * 128;                 // key within the tile
-                    const int64_t key = t * kBN + nl;
-                    uint2 bits = make_uint2(0u, 0u);
-                    if (key < p.n) bits = __ldg(reinterpret_cast<const uint2*>(plane + key * (p.d / 8) + byte0));
-                    uint8_t* dst = sm.b[s] + (nl >> 3) * 128 + (nl & 7) * 16;
+            for (int h = 0; h < 2; ++h) {
+                const int64_t key = t * kBN + e + h * 128;
+                if (key < p.n) bits[h] = __ldg(reinterpret_cast<const uint2*>(plane + key * (p.d / 8) + byte0));
+            }
+        };
+        // expand step g from `bits` into its stage; false when the CTA stops. Each warp waits for
+        // the stage on its own and arrives on bfull once its keys are written (4 arrivals).
+        auto expand = [&](int64_t g, const uint2 (&bits)[2]) -> bool {
+            const int s = (int)(g % kStages);
+            const int64_t r = g / kStages;
+            bool ok = true;
+            if (r > 0) ok = ptx::mbar_wait(&sm.empty[s], (uint32_t)((r - 1) & 1));
+            if (!ok) atomicExch(&sm.abort, 1);
+            if (!__all_sync(0xffffffffu, ok && !sm.abort)) return false;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t byte = ((j < 4 ? bits.x : bits.y) >> (8 * (j & 3))) & 0xffu;
-                        *reinterpret_cast<uint4*>(dst + j * (kBN * 16)) = sm.lut[byte];
-                    }
-                }
-                ptx::fence_proxy_async_smem();
-                named_sync(1, 128);
-                if (e == 0) {
-                    // arrive (no transaction bytes): plain arrive on the barrier
-                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(&sm.bfull[s]))
-                                 : "memory");
+            for (int h = 0; h < 2; ++h) {
+                const int nl = e + h * 128;   // key within the tile
+                uint8_t* dst = sm.b[s] + (nl >> 3) * 128 + (nl & 7) * 16;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    // byte j of the step's 64 bits -> 8 bf16 values, +1 for a set bit: word k holds
+                    // bits 2k (low half) and 2k+1 (high half); one multiply places both sign bits
+                    // (bit 15 and bit 31), one logic op masks them into -1.0 / -1.0
+                    const uint32_t x = __byte_perm(j < 4 ? bits[h].x : bits[h].y, 0u, 0x4440u | (j & 3));
+                    uint4 v;
+                    v.x = (x * 0x40008000u & 0x80008000u) ^ 0xBF80BF80u;
+                    v.y = (x * 0x10002000u & 0x80008000u) ^ 0xBF80BF80u;
+                    v.z = (x * 0x04000800u & 0x80008000u) ^ 0xBF80BF80u;
+                    v.w = (x * 0x01000200u & 0x80008000u) ^ 0xBF80BF80u;
+                    *reinterpret_cast<uint4*>(dst + j * (kBN * 16)) = v;
                 }
             }
-            if (stop) break;
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) {
+                // arrive (no transaction bytes): plain arrive on the barrier
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(&sm.bfull[s])) : "memory");
+            }
+            return true;
+        };
+        uint2 pf[kPrefetch][2];
+#pragma unroll
+        for (int j = 0; j < kPrefetch; ++j) fetch(j, pf[j]);
+        bool run = true;
+        for (int64_t g0 = 0; g0 < nsteps && run; g0 += kPrefetch) {
+#pragma unroll
+            for (int j = 0; j < kPrefetch; ++j) {
+                const int64_t g = g0 + j;
+                if (run && g < nsteps) {
+                    const uint2 cur[2] = {pf[j][0], pf[j][1]};
+                    fetch(g + kPrefetch, pf[j]);
+                    run = expand(g, cur);
+                }
+            }
         }
     } else {
         // ---- epilogue: warps 2..5, one query per thread ----
@@ -251,14 +272,14 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             }
             ptx::tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t a1[32], a2[32];
-                ptx::tmem_ld32(t_lane + c * 32, a1);
-                ptx::tmem_ld32(t_lane + 256 + c * 32, a2);
+            for (int c = 0; c < kBN / 16; ++c) {
+                uint32_t a1[16], a2[16];
+                ptx::tmem_ld16(t_lane + c * 16, a1);
+                ptx::tmem_ld16(t_lane + 256 + c * 16, a2);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int kl = c * 32 + j;
+                for (int j = 0; j < 16; ++j) {
+                    const int kl = c * 16 + j;
                     const int64_t key = t * kBN + kl;
                     const float est = sm.nu[kl] * fmaf(sm.g2[kl], __uint_as_float(a2[j]), p.c1 * __uint_as_float(a1[j]));
                     if (key < p.n && est > best_v[kTopMax - 1]) {
