@@ -181,6 +181,9 @@ CASES = [
     (96, 3, tq.PROD, tq.ROT_RHT, tq.F32), (192, 2, tq.MSE, tq.ROT_RHT, tq.F32),
     (1536, 2, tq.PROD, tq.ROT_RHT, tq.BF16), (160, 2, tq.PROD, tq.ROT_DENSE, tq.F32),
     (224, 3, tq.MSE, tq.ROT_DENSE, tq.F32),
+    # d = 128 with a dense rotation and 1- to 4-bit MSE codes: the tiled CUDA-core encoder
+    (128, 1, tq.MSE, tq.ROT_DENSE, tq.F32), (128, 2, tq.PROD, tq.ROT_DENSE, tq.F32),
+    (128, 3, tq.MSE, tq.ROT_DENSE, tq.BF16), (128, 5, tq.PROD, tq.ROT_DENSE, tq.BF16),
 ]
 
 
@@ -219,6 +222,17 @@ def test_general_paths(d, b, mode, rot, md, bf16_in):
     sg = gpu_score(pair, dev_f32(q), oplanes)[0]
     est = OQ.estimate(q, xt_o)
     assert np.max(np.abs(sg - est)) <= ABS_SCORE
+
+
+@pytest.mark.parametrize("b,mode", [(2, tq.MSE), (4, tq.PROD)])
+def test_dense128_encoder_many_tiles(b, mode):
+    # more 128-vector tiles than SMs, so every persistent block walks several, plus a ragged tail
+    d, n = 128, 148 * 128 * 2 + 77
+    pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.F32)
+    x = synth.unit_vectors(n, d, seed=321).astype(np.float32)
+    enc = pair.encode(x.astype(np.float64))
+    gpu, _ = gpu_encode(pair, dev_f32(x), n)
+    check_codes(pair, gpu, enc)
 
 
 def test_empty_inputs_are_noops():

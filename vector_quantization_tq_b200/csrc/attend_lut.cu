@@ -23,6 +23,8 @@
 
 namespace tq {
 
+int attend_heads_per_block(int G);
+
 namespace {
 
 constexpr int kD = 128;
@@ -62,7 +64,10 @@ struct TileBuf {
     float vn[kThreads];
 };
 
-template <int BK, bool KPROD, int BV>
+// QH query heads of one KV group per block (GQA): the tile of the group's compressed cache is
+// staged once, every token is scored against the QH heads' tables, and the value codes of a
+// token are decoded once for all QH weighted sums.
+template <int BK, bool KPROD, int BV, int QH>
 __global__ void __launch_bounds__(kThreads)
 attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict__ luts, int64_t T, int G, int64_t Tcap,
                   int64_t chunk, const uint8_t* __restrict__ kcodes, const uint8_t* __restrict__ kqjl,
@@ -76,22 +81,21 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     constexpr int LSIZE = KG::NG * KG::E + (KPROD ? NQ * 16 : 0);   // floats of one query's tables
     TB* tb = reinterpret_cast<TB*>(smem_raw);                    // 2 stages
     float* vc = reinterpret_cast<float*>(tb + 2);               // 32 (V centroids)
-    float* tm = vc + 32;                                         // NG * E
-    float* tz = tm + KG::NG * KG::E;                             // NQ * 16
-    float* wt = tm + LSIZE;                                      // kThreads
-    float* red = wt + kThreads;                                  // 32
-    float* accw = red + 32;                                      // kWarps * kD
+    float* tm = vc + 32;                                         // QH x LSIZE: head qh's tables at qh * LSIZE
+    float* wt = tm + QH * LSIZE;                                 // QH x kThreads
+    float* red = wt + QH * kThreads;                             // QH x 32
+    float* accw = red + QH * 32;                                 // kWarps x QH x kD
 
-    const int h = blockIdx.y;
+    const int h0 = blockIdx.y * QH;   // the block's first query head
     const int split = blockIdx.x;
     const int nsplit = gridDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t_begin = (int64_t)split * chunk;
     const int64_t t_end = (T < t_begin + chunk) ? T : t_begin + chunk;
-    const int64_t hT = (int64_t)(h / G) * Tcap;   // planes of this query head's KV head
+    const int64_t hT = (int64_t)(h0 / G) * Tcap;   // planes of the heads' KV head
 
-    // Stage a tile (tokens t0 .. t0+255 of this head) into buffer `sb`; rows past the end of
-    // this split are not copied and not read.
+    // Stage a tile (tokens t0 .. t0+255 of this KV head) into buffer `sb`; rows past the end
+    // of this split are not copied and not read.
     auto stage_tile = [&](int sb, int64_t t0) {
         TB& B = tb[sb];
         const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
@@ -110,15 +114,23 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
         }
     };
 
-    // this head's tables (q' against the K code groups, u against the QJL nibbles), built
-    // once per head by the table launch, arrive with the first tile
-    for (int i = threadIdx.x; i < LSIZE / 4; i += kThreads) cp_async16(tm + 4 * i, luts + (int64_t)h * LSIZE + 4 * i);
+    // the heads' tables (q' against the K code groups, u against the QJL nibbles), built once
+    // per head by the table launch and consecutive in `luts`, arrive with the first tile
+    for (int i = threadIdx.x; i < QH * LSIZE / 4; i += kThreads)
+        cp_async16(tm + 4 * i, luts + (int64_t)h0 * LSIZE + 4 * i);
     if (t_begin < t_end) stage_tile(0, t_begin);
     cp_async_commit();
     if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};       // coordinates 4*lane .. 4*lane+3, this warp's tokens
-    float m_run = -INFINITY, l_run = 0.f;
+    float acc[QH][4];   // per head: coordinates 4*lane .. 4*lane+3, this warp's tokens
+    float m_run[QH], l_run[QH];
+#pragma unroll
+    for (int q = 0; q < QH; ++q) {
+        m_run[q] = -INFINITY;
+        l_run[q] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[q][c] = 0.f;
+    }
     int it = 0;
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads, ++it) {
         const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
@@ -128,8 +140,10 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
         cp_async_wait1();
         __syncthreads();
         const TB& B = tb[sb];
-        // ---- A: score of token t0 + threadIdx.x ----
-        float s = -INFINITY;
+        // ---- A: scores of token t0 + threadIdx.x against the QH heads ----
+        float s[QH];
+#pragma unroll
+        for (int q = 0; q < QH; ++q) s[q] = -INFINITY;
         if ((int)threadIdx.x < cnt) {
             constexpr int CW = kD * BK / 32;
             uint32_t w[CW];
@@ -140,10 +154,12 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                 w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
             }
             // table lookups into paired accumulators (two independent chains, f32x2 adds)
-            float2 p1[1] = {make_float2(0.f, 0.f)};
+            float2 p1[QH];
+#pragma unroll
+            for (int q = 0; q < QH; ++q) p1[q] = make_float2(0.f, 0.f);
             if constexpr (KG::G == 4) {
 #pragma unroll
-                for (int wi = 0; wi < CW; ++wi) add_nibbles<1, 0>(w[wi], tm + 8 * wi * 16, p1);
+                for (int wi = 0; wi < CW; ++wi) add_nibbles<QH, LSIZE>(w[wi], tm + 8 * wi * 16, p1);
             } else {
                 static_assert(KG::NG % 2 == 0, "groups in pairs");
 #pragma unroll
@@ -153,56 +169,75 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                     uint32_t e;
                     if (sh + KG::G <= 32) e = (w[wi] >> sh) & (KG::E - 1);
                     else e = ((w[wi] >> sh) | (w[wi + 1] << (32 - sh))) & (KG::E - 1);
-                    if (k & 1) p1[0].y += tm[k * KG::E + e];
-                    else p1[0].x += tm[k * KG::E + e];
+#pragma unroll
+                    for (int q = 0; q < QH; ++q) {
+                        if (k & 1) p1[q].y += tm[q * LSIZE + k * KG::E + e];
+                        else p1[q].x += tm[q * LSIZE + k * KG::E + e];
+                    }
                 }
             }
-            float2 p2[1] = {make_float2(0.f, 0.f)};
+            float2 p2[QH];
+#pragma unroll
+            for (int q = 0; q < QH; ++q) p2[q] = make_float2(0.f, 0.f);
             float g2 = 0.f;
             if constexpr (KPROD) {
                 const uint4 zv = *reinterpret_cast<const uint4*>(B.kz + threadIdx.x * 16);
                 const uint32_t z[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-                for (int wi = 0; wi < 4; ++wi) add_nibbles<1, 0>(z[wi], tz + 8 * wi * 16, p2);
+                for (int wi = 0; wi < 4; ++wi) add_nibbles<QH, LSIZE>(z[wi], tm + KG::NG * KG::E + 8 * wi * 16, p2);
                 g2 = B.kr[threadIdx.x] * ks.qjl_scale;
             }
-            s = scale * B.kn[threadIdx.x] * fmaf(g2, p2[0].x + p2[0].y, p1[0].x + p1[0].y);
+            const float kn = scale * B.kn[threadIdx.x];
+#pragma unroll
+            for (int q = 0; q < QH; ++q) s[q] = kn * fmaf(g2, p2[q].x + p2[q].y, p1[q].x + p1[q].y);
         }
-        // ---- B: online softmax bookkeeping ----
-        const float wm = warp_max(s);
-        if (lane == 0) red[warp] = wm;
-        __syncthreads();
-        float tmax = red[0];
+        // ---- B: online softmax bookkeeping, per head ----
 #pragma unroll
-        for (int i = 1; i < kWarps; ++i) tmax = fmaxf(tmax, red[i]);
-        const float m_new = fmaxf(m_run, tmax);
-        const float alpha = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
-        const float p = ((int)threadIdx.x < cnt) ? __expf(s - m_new) : 0.f;
-        const float ps = warp_sum(p);
+        for (int q = 0; q < QH; ++q) {
+            const float wm = warp_max(s[q]);
+            if (lane == 0) red[q * 32 + warp] = wm;
+        }
+        __syncthreads();
+        float alpha[QH], p[QH];
+#pragma unroll
+        for (int q = 0; q < QH; ++q) {
+            float tmax = red[q * 32];
+#pragma unroll
+            for (int i = 1; i < kWarps; ++i) tmax = fmaxf(tmax, red[q * 32 + i]);
+            const float m_new = fmaxf(m_run[q], tmax);
+            alpha[q] = (m_run[q] == -INFINITY) ? 0.f : __expf(m_run[q] - m_new);
+            p[q] = ((int)threadIdx.x < cnt) ? __expf(s[q] - m_new) : 0.f;
+            m_run[q] = m_new;
+        }
         __syncthreads();   // everyone has read red[] (max) before it is reused
-        if (lane == 0) red[warp] = ps;
-        if ((int)threadIdx.x < cnt) wt[threadIdx.x] = p * B.vn[threadIdx.x];
+        const float vnt = ((int)threadIdx.x < cnt) ? B.vn[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int q = 0; q < QH; ++q) {
+            const float ps = warp_sum(p[q]);
+            if (lane == 0) red[q * 32 + warp] = ps;
+            wt[q * kThreads + threadIdx.x] = p[q] * vnt;
+        }
         __syncthreads();
-        float tsum = 0.f;
 #pragma unroll
-        for (int i = 0; i < kWarps; ++i) tsum += red[i];
-        l_run = l_run * alpha + tsum;
-        m_run = m_new;
+        for (int q = 0; q < QH; ++q) {
+            float tsum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[c] *= alpha;
-        // ---- C: value sum, one warp per token, 4 coordinates per lane; 32 tokens per warp ----
+            for (int i = 0; i < kWarps; ++i) tsum += red[q * 32 + i];
+            l_run[q] = l_run[q] * alpha[q] + tsum;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[q][c] *= alpha[q];
+        }
+        // ---- C: value sums, one warp per token, 4 coordinates per lane; 32 tokens per warp ----
         const int ntok = (cnt - warp + kWarps - 1) / kWarps;   // tokens t = warp + 8 * i < cnt
         // batches of 8 tokens: the 8 code slices are loaded before their FMAs
 #pragma unroll
         for (int i0 = 0; i0 < kThreads / kWarps; i0 += 8) {
             uint32_t bits[8];
-            float wv[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = i0 + j;
                 const int t = warp + i * kWarps;
                 uint32_t b = 0;
-                float w = 0.f;
                 if (i < ntok) {
                     const uint8_t* row = B.vc + t * TB::VROW;
                     if constexpr (BV == 4) {
@@ -217,75 +252,106 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
                         if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)r32[wi + 1] << 32;
                         b = (uint32_t)(win >> sh);
                     }
-                    w = wt[t];
                 }
                 bits[j] = b;
-                wv[j] = w;
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j;
+                const int t = (i < ntok) ? warp + i * kWarps : 0;   // weights of absent tokens are 0
+                float cv[4];
                 const char* cbase = reinterpret_cast<const char*>(vc);
                 if constexpr (BV == 4) {
                     // byte offsets 4 e of the four nibbles: 0 and 2 from `lo`, 1 and 3 from `hi`
                     const uint32_t lo = (bits[j] << 2) & 0x3C3Cu, hi = (bits[j] >> 2) & 0x3C3Cu;
-                    acc[0] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (lo & 0xFFu)), acc[0]);
-                    acc[1] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (hi & 0xFFu)), acc[1]);
-                    acc[2] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (lo >> 8)), acc[2]);
-                    acc[3] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (hi >> 8)), acc[3]);
+                    cv[0] = *reinterpret_cast<const float*>(cbase + (lo & 0xFFu));
+                    cv[1] = *reinterpret_cast<const float*>(cbase + (hi & 0xFFu));
+                    cv[2] = *reinterpret_cast<const float*>(cbase + (lo >> 8));
+                    cv[3] = *reinterpret_cast<const float*>(cbase + (hi >> 8));
                 } else if constexpr (BV == 2) {
                     const uint32_t b8 = bits[j];
-                    acc[0] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 << 2) & 0xCu)), acc[0]);
-                    acc[1] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + (b8 & 0xCu)), acc[1]);
-                    acc[2] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 >> 2) & 0xCu)), acc[2]);
-                    acc[3] = fmaf(wv[j], *reinterpret_cast<const float*>(cbase + ((b8 >> 4) & 0xCu)), acc[3]);
+                    cv[0] = *reinterpret_cast<const float*>(cbase + ((b8 << 2) & 0xCu));
+                    cv[1] = *reinterpret_cast<const float*>(cbase + (b8 & 0xCu));
+                    cv[2] = *reinterpret_cast<const float*>(cbase + ((b8 >> 2) & 0xCu));
+                    cv[3] = *reinterpret_cast<const float*>(cbase + ((b8 >> 4) & 0xCu));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        acc[c] = fmaf(wv[j], vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)], acc[c]);
+                    for (int c = 0; c < 4; ++c) cv[c] = vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)];
+                }
+#pragma unroll
+                for (int q = 0; q < QH; ++q) {
+                    const float wv = (i < ntok) ? wt[q * kThreads + t] : 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[q][c] = fmaf(wv, cv[c], acc[q][c]);
                 }
             }
         }
         __syncthreads();   // wt / red and the tile buffer are reused
     }
     cp_async_wait0();
-    // ---- reduce the warps' value sums and write the split record ----
+    // ---- reduce the warps' value sums and write the split records ----
 #pragma unroll
-    for (int c = 0; c < 4; ++c) accw[warp * kD + 4 * lane + c] = acc[c];
+    for (int q = 0; q < QH; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) accw[(warp * QH + q) * kD + 4 * lane + c] = acc[q][c];
     __syncthreads();
-    float* rec = part + ((int64_t)h * nsplit + split) * (kD + 2);
-    for (int j = threadIdx.x; j < kD; j += kThreads) {
+    for (int j = threadIdx.x; j < QH * kD; j += kThreads) {
+        const int q = j / kD, jj = j % kD;
         float a = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < kWarps; ++w2) a += accw[w2 * kD + j];
-        rec[2 + j] = a;
+        for (int w2 = 0; w2 < kWarps; ++w2) a += accw[(w2 * QH + q) * kD + jj];
+        part[((int64_t)(h0 + q) * nsplit + split) * (kD + 2) + 2 + jj] = a;
     }
-    if (threadIdx.x == 0) {
-        rec[0] = m_run;
-        rec[1] = l_run;
+#pragma unroll
+    for (int q = 0; q < QH; ++q) {
+        if ((int)threadIdx.x == q) {
+            float* rec = part + ((int64_t)(h0 + q) * nsplit + split) * (kD + 2);
+            rec[0] = m_run[q];
+            rec[1] = l_run[q];
+        }
     }
 }
 
-template <int BK, bool KPROD, int BV>
+template <int BK, bool KPROD, int BV, int QH>
 size_t smem_bytes() {
     using KG = KGroups<BK>;
     return 2 * sizeof(TileBuf<BK, KPROD, BV>) +
-           (size_t)(32 + KG::NG * KG::E + (KPROD ? (kD / 4) * 16 : 0) + kThreads + 32 + kWarps * kD) * sizeof(float);
+           (size_t)(32 + QH * (KG::NG * KG::E + (KPROD ? (kD / 4) * 16 : 0)) + QH * kThreads + QH * 32 +
+                    kWarps * QH * kD) *
+               sizeof(float);
 }
 
-template <int BK, bool KPROD, int BV>
-int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap, int nsplit,
-             int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
-             const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
-    auto kern = attend_lut_kernel<BK, KPROD, BV>;
-    const size_t smem = smem_bytes<BK, KPROD, BV>();
+template <int BK, bool KPROD, int BV, int QH>
+int launch_q(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap,
+             int nsplit, int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms,
+             const float* krnorms, const uint8_t* vcodes, const float* vnorms, float scale, float* part,
+             cudaStream_t s) {
+    auto kern = attend_lut_kernel<BK, KPROD, BV, QH>;
+    const size_t smem = smem_bytes<BK, KPROD, BV, QH>();
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return (int)e;
     }
-    dim3 grid((unsigned)nsplit, (unsigned)H);
+    dim3 grid((unsigned)nsplit, (unsigned)(H / QH));
     kern<<<grid, kThreads, smem, s>>>(ks, vs, luts, T, G, Tcap, chunk, kcodes, kqjl, knorms, krnorms, vcodes, vnorms, scale,
                                       part);
     return (int)cudaGetLastError();
+}
+
+// Query heads per block: 4 (or 2) when every group of G query heads splits evenly.
+template <int BK, bool KPROD, int BV>
+int launch_t(const DevState& ks, const DevState& vs, const float* luts, int H, int64_t T, int G, int64_t Tcap, int nsplit,
+             int64_t chunk, const uint8_t* kcodes, const uint8_t* kqjl, const float* knorms, const float* krnorms,
+             const uint8_t* vcodes, const float* vnorms, float scale, float* part, cudaStream_t s) {
+    const int qh = attend_heads_per_block(G);
+    if (qh == 4)
+        return launch_q<BK, KPROD, BV, 4>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                          vcodes, vnorms, scale, part, s);
+    if (qh == 2)
+        return launch_q<BK, KPROD, BV, 2>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                          vcodes, vnorms, scale, part, s);
+    return launch_q<BK, KPROD, BV, 1>(ks, vs, luts, H, T, G, Tcap, nsplit, chunk, kcodes, kqjl, knorms, krnorms,
+                                      vcodes, vnorms, scale, part, s);
 }
 
 template <int BK, bool KPROD>

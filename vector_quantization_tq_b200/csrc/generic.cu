@@ -944,13 +944,21 @@ int launch_score(const DevState& st, const void* q, int qdtype, int64_t groups, 
 }
 
 namespace {
-int attend_splits(int H, int64_t T) {
+// Token splits of a decode step over `blocks_per_split` blocks (heads, or head groups).
+int attend_splits(int blocks_per_split, int64_t T) {
     int64_t target = (int64_t)num_sms() * 4;
-    int64_t sp = std::max<int64_t>(1, target / std::max(1, H));
+    int64_t sp = std::max<int64_t>(1, target / std::max(1, blocks_per_split));
     sp = std::min<int64_t>(sp, (T + kAttThreads - 1) / kAttThreads);
     return (int)std::max<int64_t>(1, sp);
 }
+
+// Splits the workspace provides for: enough for the largest head group (4 query heads of one
+// KV head per block), so that grouped decode can use as many splits per head group.
+int attend_max_splits(int H, int64_t T) { return attend_splits(std::max(1, H / 4), T); }
 }  // namespace
+
+// Query heads of one KV group that the table-based decode kernel takes per block.
+int attend_heads_per_block(int G) { return (G % 4 == 0) ? 4 : ((G % 2 == 0) ? 2 : 1); }
 
 bool attend_lut_supported(const DevState& ks, const DevState& vs, const void* kcodes, const void* kqjl,
                           const void* vcodes);
@@ -960,7 +968,7 @@ int launch_attend_lut_split(const DevState& ks, const DevState& vs, const float*
                             float scale, float* part, void* stream);
 
 size_t attend_part_bytes(const DevState& ks, int H, int64_t T) {
-    const int sp = attend_splits(H, T);
+    const int sp = attend_max_splits(H, T);
     return ((size_t)H * sp * (ks.d + 2) * sizeof(float) + 255) & ~(size_t)255;
 }
 
@@ -977,12 +985,13 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
                   const uint8_t* vcodes, const float* vnorms, float scale, float* out, void* ws, size_t ws_bytes,
                   void* stream, const AppendRow* app) {
     cudaStream_t s = (cudaStream_t)stream;
-    const int sp = attend_splits(H, T);
+    const bool lut = attend_lut_supported(ks, vs, kcodes, kqjl, vcodes);
+    // the table kernel takes a group's query heads per block: as many splits per head group
+    const int sp = lut ? attend_splits(H / attend_heads_per_block(G), T) : attend_splits(H, T);
     const int64_t chunk = (T + sp - 1) / sp;
     const int nsplit = (int)((T + chunk - 1) / chunk);
     float* part = reinterpret_cast<float*>(ws);
     cudaError_t e;
-    const bool lut = attend_lut_supported(ks, vs, kcodes, kqjl, vcodes);
     if (app && !lut) {
         // the general path appends with the general encoder, one launch per plane set
         const int Hkv = H / G;
