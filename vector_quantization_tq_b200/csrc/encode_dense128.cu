@@ -1,5 +1,6 @@
 // Encoder for d = 128 with a dense rotation (Haar-random Pi stored fp32 or bf16), fp32 or bf16
-// input, TurboQuant_mse or TurboQuant_prod with 1- to 4-bit MSE codes.
+// input, TurboQuant_mse or TurboQuant_prod with 0- to 4-bit MSE codes (0: prod at b = 1, where
+// the residual is the whole rotated vector).
 //
 // TurboQuant review (Jump2Paper): Theorem 1 (store ||x||, rotate by Pi, give every coordinate
 // of the rotated unit vector its Lloyd-Max cell), Definition 1 + Theorem 2 (QJL signs of S r on
@@ -8,7 +9,8 @@
 //   a persistent block of 256 threads stages Pi^T (and S^T) once, as fp32, in shared memory and
 //   then walks tiles of 128 vectors. A tile's input is staged transposed (coordinate-major), so
 //   that for each k the 128 vectors' values are contiguous; thread t owns the 8 x 8 outputs of
-//   vectors 8 (t % 16) .. +7 and coordinates 8 (t / 16) .. +7, reads 8 + 8 operands per k
+//   8 vectors (4 (t % 16) .. +3 and 64 + 4 (t % 16) .. +3) and coordinates 8 (t / 16) .. +7,
+//   reads 8 + 8 operands per k
 //   (four 16-byte shared loads) and does 64 FMAs. Y = X Pi^T in registers is divided by ||x||,
 //   quantized against the boundaries (branch-free binary search), the residual r = y - c[idx]
 //   replaces the input tile, and Z = R S^T gives the signs. Codes and signs are packed per
@@ -45,6 +47,7 @@ struct DenseSmem {
 // boundaries t[0..L-2] (upper cell on a tie).
 template <int B>
 __device__ __forceinline__ int cell(const float* t, float y) {
+    static_assert(B >= 1, "a cell search needs at least two levels");
     int idx = 0;
 #pragma unroll
     for (int step = 1 << (B - 1); step >= 1; step >>= 1) idx += (y >= t[idx + step - 1]) ? step : 0;
@@ -59,8 +62,11 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
     extern __shared__ __align__(16) unsigned char smem_raw[];
     DenseSmem& sm = *reinterpret_cast<DenseSmem*>(smem_raw);
     const int tid = threadIdx.x;
-    const int vg = tid & 15, og = tid >> 4;   // vectors 8 vg .. +7, coordinates 8 og .. +7
-    constexpr int kRow = 16 * B;              // code bytes per vector
+    // vectors 4 vg .. +3 and 64 + 4 vg .. +3 (so that a warp's 16 vector groups read one
+    // contiguous 256-byte run of a row of the tile), coordinates 8 og .. +7
+    const int vg = tid & 15, og = tid >> 4;
+    auto vec_of = [&](int a) { return (a < 4) ? 4 * vg + a : 64 + 4 * vg + (a - 4); };
+    constexpr int kRow = 16 * B;              // code bytes per vector (none for B = 0)
 
     // stage Pi^T (and S^T) as fp32
     for (int i = tid; i < kD * kD; i += kThreads) {
@@ -105,7 +111,7 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
         }
         __syncthreads();
         if (tid < kT) sm.nrm[tid] = sqrtf(sm.rr[0][tid] + sm.rr[1][tid]);
-        // ---- Y = X Pi^T: acc[a][b] = y of vector 8 vg + a, coordinate 8 og + b ----
+        // ---- Y = X Pi^T: acc[a][b] = y of vector vec_of(a), coordinate 8 og + b ----
         float acc[8][8];
 #pragma unroll
         for (int a = 0; a < 8; ++a)
@@ -113,8 +119,8 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
             for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 #pragma unroll 4
         for (int k = 0; k < kD; ++k) {
-            const float4 x0 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 8 * vg]);
-            const float4 x1 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 8 * vg + 4]);
+            const float4 x0 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 4 * vg]);
+            const float4 x1 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 64 + 4 * vg]);
             const float4 p0 = *reinterpret_cast<const float4*>(&sm.piT[k * kD + 8 * og]);
             const float4 p1 = *reinterpret_cast<const float4*>(&sm.piT[k * kD + 8 * og + 4]);
             const float xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -128,7 +134,7 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
         // ---- quantize; residual into the tile buffer; packed codes ----
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
-            const int v = 8 * vg + a;
+            const int v = vec_of(a);
             const float nu = sm.nrm[v];
             const float sc = (nu > 0.f) ? 1.f / nu : 0.f;
             uint32_t word = 0u;   // the 8 codes of coordinates 8 og .. +7: 8 B bits
@@ -136,9 +142,12 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
                 const float y = acc[a][b] * sc;
-                const int c = cell<B>(sm.t, y);
-                word |= (uint32_t)c << (B * b);
-                const float r = (nu > 0.f) ? (y - sm.c[c]) : 0.f;
+                float r = y;   // B = 0: no MSE stage, the residual is y
+                if constexpr (B > 0) {
+                    const int c = cell<B>(sm.t, y);
+                    word |= (uint32_t)c << (B * b);
+                    r = (nu > 0.f) ? (y - sm.c[c]) : 0.f;
+                }
                 r2 = fmaf(r, r, r2);
                 if constexpr (PROD) sm.xt[(8 * og + b) * kLd + v] = r;
             }
@@ -156,8 +165,8 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
                 for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 #pragma unroll 4
             for (int k = 0; k < kD; ++k) {
-                const float4 x0 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 8 * vg]);
-                const float4 x1 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 8 * vg + 4]);
+                const float4 x0 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 4 * vg]);
+                const float4 x1 = *reinterpret_cast<const float4*>(&sm.xt[k * kLd + 64 + 4 * vg]);
                 const float4 p0 = *reinterpret_cast<const float4*>(&sm.sT[k * kD + 8 * og]);
                 const float4 p1 = *reinterpret_cast<const float4*>(&sm.sT[k * kD + 8 * og + 4]);
                 const float xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -172,13 +181,13 @@ encode_dense128_kernel(const DevState st, const void* __restrict__ x, int64_t n,
                 uint32_t z = 0u;
 #pragma unroll
                 for (int b = 0; b < 8; ++b) z |= (acc[a][b] >= 0.f ? 1u : 0u) << b;
-                sm.zrows[(8 * vg + a) * 16 + og] = (uint8_t)z;
+                sm.zrows[vec_of(a) * 16 + og] = (uint8_t)z;
             }
         }
         __syncthreads();
         // ---- write the tile: code rows, sign rows, norms ----
         const int nv = (int)((n - v0) < kT ? (n - v0) : kT);
-        {
+        if constexpr (B > 0) {
             const uint4* src = reinterpret_cast<const uint4*>(sm.rows);
             uint4* dst = reinterpret_cast<uint4*>(codes + v0 * kRow);
             for (int i = tid; i < nv * kRow / 16; i += kThreads) dst[i] = src[i];
@@ -237,6 +246,9 @@ template <bool PROD>
 int launch_dense_b(const DevState& st, int dtype, const void* x, int64_t n, int64_t ld, uint8_t* codes,
                    uint8_t* qjl, float* norms, float* rnorms, cudaStream_t s) {
     switch (st.b_mse) {
+        case 0:
+            if constexpr (PROD) return launch_dense_t<0, true>(st, dtype, x, n, ld, codes, qjl, norms, rnorms, s);
+            return (int)cudaErrorInvalidValue;
         case 1: return launch_dense_t<1, PROD>(st, dtype, x, n, ld, codes, qjl, norms, rnorms, s);
         case 2: return launch_dense_t<2, PROD>(st, dtype, x, n, ld, codes, qjl, norms, rnorms, s);
         case 3: return launch_dense_t<3, PROD>(st, dtype, x, n, ld, codes, qjl, norms, rnorms, s);
@@ -249,8 +261,8 @@ int launch_dense_b(const DevState& st, int dtype, const void* x, int64_t n, int6
 
 // True when the dense d = 128 encoder handles this configuration.
 bool encode_dense128_supported(const DevState& st, int dtype, int64_t n, int64_t ld) {
-    return st.d == kD && st.rot == TQ_ROT_DENSE && st.b_mse >= 1 && st.b_mse <= 4 && n > 0 && ld >= kD &&
-           (dtype == TQ_F32 || dtype == TQ_BF16);
+    const bool bits_ok = (st.b_mse >= 1 && st.b_mse <= 4) || (st.b_mse == 0 && st.mode == TQ_PROD);
+    return st.d == kD && st.rot == TQ_ROT_DENSE && bits_ok && n > 0 && ld >= kD && (dtype == TQ_F32 || dtype == TQ_BF16);
 }
 
 int launch_encode_dense128(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
