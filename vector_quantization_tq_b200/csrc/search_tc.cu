@@ -36,6 +36,7 @@ constexpr int kBK = 64;
 constexpr int kStages = 3;
 constexpr int kThreads = 320;
 constexpr int kTopMax = 16;
+constexpr int kCand = 64;   // candidates a query buffers before merging them into its top list
 
 struct SearchParams {
     int nq;
@@ -58,6 +59,8 @@ struct __align__(1024) SearchSmem {
     uint8_t b[kStages][kBN * kBK * 2];   // keys as +-1, K-major core matrices
     float nu[kBN];
     float g2[kBN];
+    float candv[kCand][kBM];             // per query (column): estimates above its threshold
+    int candi[kCand][kBM];               // and their keys
     uint64_t afull[kStages];
     uint64_t bfull[kStages];
     uint64_t empty[kStages];
@@ -177,17 +180,25 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         constexpr int kPrefetch = 4;
         const int e = threadIdx.x - 6 * 32;   // 0..127
         const int64_t nsteps = (tile_end - tile_begin) * ks_per_tile;
-        auto fetch = [&](int64_t g, uint2 (&bits)[2]) {
+        // The steps are fetched in order, so the fetch position (tile, step) advances by one per
+        // call instead of being divided out of the step index.
+        const int row_bytes = p.d / 8;
+        int64_t f_tile = tile_begin;   // tile and step of the next fetch
+        int f_ks = 0;
+        auto fetch = [&](uint2 (&bits)[2]) {
             bits[0] = bits[1] = make_uint2(0u, 0u);
-            if (g >= nsteps) return;
-            const int64_t t = tile_begin + g / ks_per_tile;
-            const int ks = (int)(g % ks_per_tile);
-            const uint8_t* plane = (ks < ks_half) ? p.codes : p.qjl;
-            const int byte0 = ((ks < ks_half) ? ks : ks - ks_half) * (kBK / 8);
+            if (f_tile >= tile_end) return;
+            const uint8_t* plane = (f_ks < ks_half) ? p.codes : p.qjl;
+            const int byte0 = ((f_ks < ks_half) ? f_ks : f_ks - ks_half) * (kBK / 8);
+            const uint8_t* base = plane + (f_tile * kBN + e) * row_bytes + byte0;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int64_t key = t * kBN + e + h * 128;
-                if (key < p.n) bits[h] = __ldg(reinterpret_cast<const uint2*>(plane + key * (p.d / 8) + byte0));
+                const int64_t key = f_tile * kBN + e + h * 128;
+                if (key < p.n) bits[h] = __ldg(reinterpret_cast<const uint2*>(base + h * 128 * row_bytes));
+            }
+            if (++f_ks == ks_per_tile) {
+                f_ks = 0;
+                ++f_tile;
             }
         };
         // expand step g from `bits` into its stage; false when the CTA stops. Each warp waits for
@@ -227,7 +238,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         };
         uint2 pf[kPrefetch][2];
 #pragma unroll
-        for (int j = 0; j < kPrefetch; ++j) fetch(j, pf[j]);
+        for (int j = 0; j < kPrefetch; ++j) fetch(pf[j]);
         bool run = true;
         for (int64_t g0 = 0; g0 < nsteps && run; g0 += kPrefetch) {
 #pragma unroll
@@ -235,7 +246,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
                 const int64_t g = g0 + j;
                 if (run && g < nsteps) {
                     const uint2 cur[2] = {pf[j][0], pf[j][1]};
-                    fetch(g + kPrefetch, pf[j]);
+                    fetch(pf[j]);   // step g + kPrefetch
                     run = expand(g, cur);
                 }
             }
@@ -253,6 +264,35 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             best_v[i] = -INFINITY;
             best_i[i] = INT_MAX;
         }
+        // Estimates above the current k-th best go to the query's candidate buffer (in key
+        // order); the buffer is merged into the sorted list once per tile, after the tile's
+        // accumulator has been released (so the merge overlaps the next tile's MMAs), or when
+        // it fills up. A sorted insertion per key ran divergently for almost every key while
+        // the threshold was low and held the accumulator for tens of thousands of cycles.
+        float thr = -INFINITY;
+        int cnt = 0;
+        auto merge = [&]() {
+            for (int i = 0; i < cnt; ++i) {
+                const float est = sm.candv[i][row];
+                if (est > best_v[kTopMax - 1]) {
+                    best_v[kTopMax - 1] = est;
+                    best_i[kTopMax - 1] = sm.candi[i][row];
+#pragma unroll
+                    for (int j = kTopMax - 1; j > 0; --j) {
+                        if (best_v[j] > best_v[j - 1]) {
+                            const float tv = best_v[j];
+                            best_v[j] = best_v[j - 1];
+                            best_v[j - 1] = tv;
+                            const int ti = best_i[j];
+                            best_i[j] = best_i[j - 1];
+                            best_i[j - 1] = ti;
+                        }
+                    }
+                }
+            }
+            cnt = 0;
+            thr = best_v[kTopMax - 1];
+        };
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         int64_t it = 0;
         bool failed = false;
@@ -282,20 +322,10 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
                     const int kl = c * 16 + j;
                     const int64_t key = t * kBN + kl;
                     const float est = sm.nu[kl] * fmaf(sm.g2[kl], __uint_as_float(a2[j]), p.c1 * __uint_as_float(a1[j]));
-                    if (key < p.n && est > best_v[kTopMax - 1]) {
-                        best_v[kTopMax - 1] = est;
-                        best_i[kTopMax - 1] = (int)key;
-#pragma unroll
-                        for (int i = kTopMax - 1; i > 0; --i) {
-                            if (best_v[i] > best_v[i - 1]) {
-                                const float tv = best_v[i];
-                                best_v[i] = best_v[i - 1];
-                                best_v[i - 1] = tv;
-                                const int ti = best_i[i];
-                                best_i[i] = best_i[i - 1];
-                                best_i[i - 1] = ti;
-                            }
-                        }
+                    if (key < p.n && est > thr) {
+                        sm.candv[cnt][row] = est;
+                        sm.candi[cnt][row] = (int)key;
+                        if (++cnt == kCand) merge();
                     }
                 }
             }
@@ -303,6 +333,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             named_sync(2, 128);   // every epilogue thread is done with TMEM and sm.nu / sm.g2
             if (et == 0)
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(&sm.tfree)) : "memory");
+            merge();   // while the next tile's MMAs run
         }
         if (failed) {
             if (et == 0) atomicExch(&g_tq_device_error, 1);
