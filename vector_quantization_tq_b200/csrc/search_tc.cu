@@ -9,10 +9,11 @@
 //   warp 0      TMA producer of the query tile (K-steps of 64 through a 3-stage ring);
 //   warp 1      MMA issuer: K-steps of the first d coordinates accumulate <q', sigma> in TMEM
 //               columns [0, 256), the next d accumulate <u, s> in [256, 512);
-//   warps 2-5   epilogue: one query per thread, est for 256 keys, running top-16 in registers;
-//   warps 6-9   expanders: each K-step's 64 bits per key become 64 bf16 +-1 values in shared
-//               memory (arithmetic: one multiply and one logic op per pair of values), with the
-//               key bits fetched a few steps ahead.
+//   warps 2-9   epilogue: two threads per query (keys 0-127 and 128-255 of a tile), est for
+//               their keys, a running top-16 each in registers (both lists go to the merge);
+//   warps 10-17 expanders: each K-step's 64 bits per key become 64 bf16 +-1 values in shared
+//               memory (arithmetic: one multiply and one logic op per pair of values), one key
+//               per thread, with the key bits fetched a few steps ahead.
 // Each CTA writes its k best (value, index) per query; a merge launch picks the final k.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -34,9 +35,10 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;   // 18 warps: TMA, MMA, 8 epilogue, 8 expanders
 constexpr int kTopMax = 16;
-constexpr int kCand = 64;   // candidates a query buffers before merging them into its top list
+constexpr int kCand = 32;   // candidates an epilogue thread buffers before merging them into its top list
+constexpr int kEpiWarp0 = 2, kExpWarp0 = 10;
 
 struct SearchParams {
     int nq;
@@ -59,8 +61,8 @@ struct __align__(1024) SearchSmem {
     uint8_t b[kStages][kBN * kBK * 2];   // keys as +-1, K-major core matrices
     float nu[kBN];
     float g2[kBN];
-    float candv[kCand][kBM];             // per query (column): estimates above its threshold
-    int candi[kCand][kBM];               // and their keys
+    float candv[kCand][2 * kBM];         // per epilogue thread (column): estimates above its threshold
+    int candi[kCand][2 * kBM];           // and their keys
     uint64_t afull[kStages];
     uint64_t bfull[kStages];
     uint64_t empty[kStages];
@@ -102,7 +104,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         ptx::prefetch_tmap(&tma_q);
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&sm.afull[s], 1);
-            ptx::mbar_init(&sm.bfull[s], 4);   // one arrival per expander warp
+            ptx::mbar_init(&sm.bfull[s], 8);   // one arrival per expander warp
             ptx::mbar_init(&sm.empty[s], 1);
         }
         ptx::mbar_init(&sm.done, 1);
@@ -171,55 +173,49 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
                 ptx::mma_commit(&sm.done);
             }
         }
-    } else if (warp >= 6) {
+    } else if (warp >= kExpWarp0) {
         // ---- expanders: key bits -> +-1 bf16 ----
         // K-step g of the CTA (tile tile_begin + g / ks_per_tile, step g % ks_per_tile) needs 8
         // bytes of one bit plane for each of the tile's 256 keys; each thread handles two keys.
         // The global loads run kPrefetch steps ahead of the expansion, so their latency overlaps
         // the work of the steps in between.
         constexpr int kPrefetch = 4;
-        const int e = threadIdx.x - 6 * 32;   // 0..127
+        const int e = threadIdx.x - kExpWarp0 * 32;   // key within the tile, 0..255
         const int64_t nsteps = (tile_end - tile_begin) * ks_per_tile;
         // The steps are fetched in order, so the fetch position (tile, step) advances by one per
         // call instead of being divided out of the step index.
         const int row_bytes = p.d / 8;
         int64_t f_tile = tile_begin;   // tile and step of the next fetch
         int f_ks = 0;
-        auto fetch = [&](uint2 (&bits)[2]) {
-            bits[0] = bits[1] = make_uint2(0u, 0u);
+        auto fetch = [&](uint2& bits) {
+            bits = make_uint2(0u, 0u);
             if (f_tile >= tile_end) return;
             const uint8_t* plane = (f_ks < ks_half) ? p.codes : p.qjl;
             const int byte0 = ((f_ks < ks_half) ? f_ks : f_ks - ks_half) * (kBK / 8);
-            const uint8_t* base = plane + (f_tile * kBN + e) * row_bytes + byte0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t key = f_tile * kBN + e + h * 128;
-                if (key < p.n) bits[h] = __ldg(reinterpret_cast<const uint2*>(base + h * 128 * row_bytes));
-            }
+            const int64_t key = f_tile * kBN + e;
+            if (key < p.n) bits = __ldg(reinterpret_cast<const uint2*>(plane + key * row_bytes + byte0));
             if (++f_ks == ks_per_tile) {
                 f_ks = 0;
                 ++f_tile;
             }
         };
         // expand step g from `bits` into its stage; false when the CTA stops. Each warp waits for
-        // the stage on its own and arrives on bfull once its keys are written (4 arrivals).
-        auto expand = [&](int64_t g, const uint2 (&bits)[2]) -> bool {
+        // the stage on its own and arrives on bfull once its keys are written (8 arrivals).
+        auto expand = [&](int64_t g, const uint2 bits) -> bool {
             const int s = (int)(g % kStages);
             const int64_t r = g / kStages;
             bool ok = true;
             if (r > 0) ok = ptx::mbar_wait(&sm.empty[s], (uint32_t)((r - 1) & 1));
             if (!ok) atomicExch(&sm.abort, 1);
             if (!__all_sync(0xffffffffu, ok && !sm.abort)) return false;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int nl = e + h * 128;   // key within the tile
-                uint8_t* dst = sm.b[s] + (nl >> 3) * 128 + (nl & 7) * 16;
+            {
+                uint8_t* dst = sm.b[s] + (e >> 3) * 128 + (e & 7) * 16;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     // byte j of the step's 64 bits -> 8 bf16 values, +1 for a set bit: word k holds
                     // bits 2k (low half) and 2k+1 (high half); one multiply places both sign bits
                     // (bit 15 and bit 31), one logic op masks them into -1.0 / -1.0
-                    const uint32_t x = __byte_perm(j < 4 ? bits[h].x : bits[h].y, 0u, 0x4440u | (j & 3));
+                    const uint32_t x = __byte_perm(j < 4 ? bits.x : bits.y, 0u, 0x4440u | (j & 3));
                     uint4 v;
                     v.x = (x * 0x40008000u & 0x80008000u) ^ 0xBF80BF80u;
                     v.y = (x * 0x10002000u & 0x80008000u) ^ 0xBF80BF80u;
@@ -236,7 +232,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             }
             return true;
         };
-        uint2 pf[kPrefetch][2];
+        uint2 pf[kPrefetch];
 #pragma unroll
         for (int j = 0; j < kPrefetch; ++j) fetch(pf[j]);
         bool run = true;
@@ -245,18 +241,20 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             for (int j = 0; j < kPrefetch; ++j) {
                 const int64_t g = g0 + j;
                 if (run && g < nsteps) {
-                    const uint2 cur[2] = {pf[j][0], pf[j][1]};
+                    const uint2 cur = pf[j];
                     fetch(pf[j]);   // step g + kPrefetch
                     run = expand(g, cur);
                 }
             }
         }
     } else {
-        // ---- epilogue: warps 2..5, one query per thread ----
+        // ---- epilogue: warps 2..9, two threads per query (one per half of the tile's keys) ----
         const int quad = warp & 3;
+        const int half = (warp - kEpiWarp0) >> 2;
         const int row = quad * 32 + lane;
+        const int col = half * kBM + row;   // this thread's column of the candidate buffer
         const int m = m0 + row;
-        const int et = threadIdx.x - 64;   // 0..127 within the epilogue group
+        const int et = threadIdx.x - kEpiWarp0 * 32;   // 0..255 within the epilogue group
         float best_v[kTopMax];
         int best_i[kTopMax];   // key index (n < 2^31)
 #pragma unroll
@@ -273,10 +271,10 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         int cnt = 0;
         auto merge = [&]() {
             for (int i = 0; i < cnt; ++i) {
-                const float est = sm.candv[i][row];
+                const float est = sm.candv[i][col];
                 if (est > best_v[kTopMax - 1]) {
                     best_v[kTopMax - 1] = est;
-                    best_i[kTopMax - 1] = sm.candi[i][row];
+                    best_i[kTopMax - 1] = sm.candi[i][col];
 #pragma unroll
                     for (int j = kTopMax - 1; j > 0; --j) {
                         if (best_v[j] > best_v[j - 1]) {
@@ -298,7 +296,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         bool failed = false;
         for (int64_t t = tile_begin; t < tile_end; ++t, ++it) {
             // per-key scales of this tile
-            for (int i = et; i < kBN; i += 128) {
+            for (int i = et; i < kBN; i += 256) {
                 const int64_t key = t * kBN + i;
                 sm.nu[i] = (key < p.n) ? __ldg(p.norms + key) : 0.f;
                 sm.g2[i] = (key < p.n) ? __ldg(p.rnorms + key) * p.qjl_scale : 0.f;
@@ -306,31 +304,31 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             bool ok = true;
             if (et == 0) ok = ptx::mbar_wait(&sm.done, (uint32_t)(it & 1));
             if (et == 0 && !ok) atomicExch(&sm.abort, 1);
-            if (named_sync_or(2, 128, et == 0 && (!ok || sm.abort))) {
+            if (named_sync_or(2, 256, et == 0 && (!ok || sm.abort))) {
                 failed = true;
                 break;
             }
             ptx::tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kBN / 16; ++c) {
-                uint32_t a1[16], a2[16];
-                ptx::tmem_ld16(t_lane + c * 16, a1);
-                ptx::tmem_ld16(t_lane + 256 + c * 16, a2);
+            for (int c = half * (kBN / 16); c < (half + 1) * (kBN / 16); ++c) {
+                uint32_t a1[8], a2[8];
+                ptx::tmem_ld8(t_lane + c * 8, a1);
+                ptx::tmem_ld8(t_lane + 256 + c * 8, a2);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int kl = c * 16 + j;
+                for (int j = 0; j < 8; ++j) {
+                    const int kl = c * 8 + j;
                     const int64_t key = t * kBN + kl;
                     const float est = sm.nu[kl] * fmaf(sm.g2[kl], __uint_as_float(a2[j]), p.c1 * __uint_as_float(a1[j]));
                     if (key < p.n && est > thr) {
-                        sm.candv[cnt][row] = est;
-                        sm.candi[cnt][row] = (int)key;
+                        sm.candv[cnt][col] = est;
+                        sm.candi[cnt][col] = (int)key;
                         if (++cnt == kCand) merge();
                     }
                 }
             }
             ptx::tc_fence_before();
-            named_sync(2, 128);   // every epilogue thread is done with TMEM and sm.nu / sm.g2
+            named_sync(2, 256);   // every epilogue thread is done with TMEM and sm.nu / sm.g2
             if (et == 0)
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(&sm.tfree)) : "memory");
             merge();   // while the next tile's MMAs run
@@ -338,7 +336,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         if (failed) {
             if (et == 0) atomicExch(&g_tq_device_error, 1);
         } else if (m < p.nq) {
-            const int64_t o = ((int64_t)m * gridDim.y + blockIdx.y) * p.k;
+            const int64_t o = (((int64_t)m * gridDim.y + blockIdx.y) * 2 + half) * p.k;
 #pragma unroll
             for (int i = 0; i < kTopMax; ++i)
                 if (i < p.k) {
@@ -462,7 +460,7 @@ size_t search_tc_ws_bytes(const DevState& st, int64_t nq, int64_t n, int k) {
     add(nq * d * 4);          // u
     add(nq * 2 * d * 2);      // split / packed bf16 operand
     add(nq * 2 * d * 2);      // packed queries
-    const size_t nc = (size_t)nq * search_ctas_y(n) * k;
+    const size_t nc = (size_t)nq * search_ctas_y(n) * 2 * k;   // two lists per (query, CTA)
     add(nc * 4);
     add(nc * 8);
     return b;
@@ -485,7 +483,7 @@ int launch_search_tc(const DevState& st, const void* q, int qdtype, int64_t nq, 
     uint16_t* split = reinterpret_cast<uint16_t*>(take(nq * 2 * d * 2));
     uint16_t* qpack = reinterpret_cast<uint16_t*>(take(nq * 2 * d * 2));
     const int cy = search_ctas_y(n);
-    const size_t nc = (size_t)nq * cy * k;
+    const size_t nc = (size_t)nq * cy * 2 * k;
     float* cand_v = reinterpret_cast<float*>(take(nc * 4));
     int64_t* cand_i = reinterpret_cast<int64_t*>(take(nc * 8));
     const int threads = 256;
@@ -546,7 +544,7 @@ int launch_search_tc(const DevState& st, const void* q, int qdtype, int64_t nq, 
     dim3 grid((unsigned)((nq + kBM - 1) / kBM), (unsigned)cy);
     search_tc_kernel<<<grid, kThreads, smem, s>>>(tm, p);
     if ((e = (int)cudaGetLastError())) return e;
-    return launch_search_merge(nq, (int64_t)cy * k, k, cand_v, cand_i, idx, vals, stream);
+    return launch_search_merge(nq, (int64_t)cy * 2 * k, k, cand_v, cand_i, idx, vals, stream);
 }
 
 int take_device_error_search(int* flag) {
