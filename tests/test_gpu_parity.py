@@ -184,6 +184,10 @@ CASES = [
     # d = 128 with a dense rotation and 1- to 4-bit MSE codes: the tiled CUDA-core encoder
     (128, 1, tq.MSE, tq.ROT_DENSE, tq.F32), (128, 2, tq.PROD, tq.ROT_DENSE, tq.F32),
     (128, 3, tq.MSE, tq.ROT_DENSE, tq.BF16), (128, 5, tq.PROD, tq.ROT_DENSE, tq.BF16),
+    # d = 256 with a dense fp32 rotation: the streamed-matrix CUDA-core encoder
+    (256, 2, tq.MSE, tq.ROT_DENSE, tq.F32), (256, 4, tq.MSE, tq.ROT_DENSE, tq.F32),
+    (256, 1, tq.PROD, tq.ROT_DENSE, tq.F32), (256, 3, tq.PROD, tq.ROT_DENSE, tq.F32),
+    (256, 5, tq.PROD, tq.ROT_DENSE, tq.F32),
 ]
 
 
@@ -224,10 +228,11 @@ def test_general_paths(d, b, mode, rot, md, bf16_in):
     assert np.max(np.abs(sg - est)) <= ABS_SCORE
 
 
-@pytest.mark.parametrize("b,mode", [(2, tq.MSE), (4, tq.PROD)])
-def test_dense128_encoder_many_tiles(b, mode):
-    # more 128-vector tiles than SMs, so every persistent block walks several, plus a ragged tail
-    d, n = 128, 148 * 128 * 2 + 77
+@pytest.mark.parametrize("d,b,mode", [(128, 2, tq.MSE), (128, 4, tq.PROD), (256, 3, tq.MSE), (256, 2, tq.PROD)])
+def test_dense_tiled_encoder_many_tiles(d, b, mode):
+    # more tiles (128 vectors at d = 128, 64 at d = 256) than SMs, so every persistent block
+    # walks several, plus a ragged tail
+    n = 148 * 128 * 2 + 77
     pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.F32)
     x = synth.unit_vectors(n, d, seed=321).astype(np.float32)
     enc = pair.encode(x.astype(np.float64))

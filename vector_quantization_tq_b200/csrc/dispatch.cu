@@ -1,6 +1,6 @@
 // Chooses the encoder for a state: the tensor-core encoders where one exists for the
-// configuration, the tiled CUDA-core encoder for d = 128 with a dense rotation, else the
-// general kernel.
+// configuration, the tiled CUDA-core encoders for d = 128 and d = 256 with a dense rotation,
+// else the general kernel.
 #include "common.cuh"
 
 namespace tq {
@@ -14,6 +14,10 @@ int launch_encode_tc(const DevState& st, const void* x, int64_t n, int64_t ld, u
 
 bool encode_dense128_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
 int launch_encode_dense128(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
+                           uint8_t* qjl, float* norms, float* rnorms, void* stream);
+
+bool encode_dense256_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
+int launch_encode_dense256(const DevState& st, const void* x, int dtype, int64_t n, int64_t ld, uint8_t* codes,
                            uint8_t* qjl, float* norms, float* rnorms, void* stream);
 
 bool encode_gemm_supported(const DevState& st, int dtype, int64_t n, int64_t ld);
@@ -81,6 +85,8 @@ int launch_encode(const DevState& st, const void* x, int dtype, int64_t n, int64
         return launch_encode_tc(st, x, n, ld, codes, qjl, norms, rnorms, stream);
     if (encode_dense128_supported(st, dtype, n, ld))
         return launch_encode_dense128(st, x, dtype, n, ld, codes, qjl, norms, rnorms, stream);
+    if (encode_dense256_supported(st, dtype, n, ld))
+        return launch_encode_dense256(st, x, dtype, n, ld, codes, qjl, norms, rnorms, stream);
     return launch_encode_generic(st, x, dtype, n, ld, nullptr, 1, codes, qjl, norms, rnorms, stream);
 }
 
