@@ -122,14 +122,17 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     cp_async_commit();
     if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
 
-    float acc[QH][4];   // per head: coordinates 4*lane .. 4*lane+3, this warp's tokens
+    // per head: this warp's value sums, coordinates 4 lane .. +3 (8 (lane % 16) .. +7 for 4-bit
+    // values, the two half-warps taking different tokens)
+    constexpr int VC = (BV == 4) ? 8 : 4;
+    float acc[QH][VC];
     float m_run[QH], l_run[QH];
 #pragma unroll
     for (int q = 0; q < QH; ++q) {
         m_run[q] = -INFINITY;
         l_run[q] = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[q][c] = 0.f;
+        for (int c = 0; c < VC; ++c) acc[q][c] = 0.f;
     }
     int it = 0;
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads, ++it) {
@@ -225,64 +228,97 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
             for (int i = 0; i < kWarps; ++i) tsum += red[q * 32 + i];
             l_run[q] = l_run[q] * alpha[q] + tsum;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[q][c] *= alpha[q];
+            for (int c = 0; c < VC; ++c) acc[q][c] *= alpha[q];
         }
-        // ---- C: value sums, one warp per token, 4 coordinates per lane; 32 tokens per warp ----
-        const int ntok = (cnt - warp + kWarps - 1) / kWarps;   // tokens t = warp + 8 * i < cnt
-        // batches of 8 tokens: the 8 code slices are loaded before their FMAs
+        if constexpr (BV == 4) {
+            // ---- C: value sums, two tokens per warp step (at step i half-warp h takes token
+            // 16 i + 2 warp + h, so the two rows lie in different banks), 8 coordinates per lane: a 4-byte slice of the token's code row,
+            // one lookup per coordinate in the 16-entry table (one entry per bank: no conflicts)
+            // and paired FMAs ----
+            const int hsel = lane >> 4, hl = lane & 15;
+            const char* cbase = reinterpret_cast<const char*>(vc);
 #pragma unroll
-        for (int i0 = 0; i0 < kThreads / kWarps; i0 += 8) {
-            uint32_t bits[8];
+            for (int i0 = 0; i0 < kThreads / kWarps / 2; i0 += 8) {
+                uint32_t bits[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = i0 + j;
-                const int t = warp + i * kWarps;
-                uint32_t b = 0;
-                if (i < ntok) {
-                    const uint8_t* row = B.vc + t * TB::VROW;
-                    if constexpr (BV == 4) {
-                        b = reinterpret_cast<const uint16_t*>(row)[lane];
-                    } else if constexpr (BV == 2) {
-                        b = row[lane];
-                    } else {
-                        const int b0 = lane * 4 * BV;
-                        const int wi = b0 >> 5, sh = b0 & 31;
-                        const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row);
-                        uint64_t win = r32[wi];
-                        if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)r32[wi + 1] << 32;
-                        b = (uint32_t)(win >> sh);
+                for (int j = 0; j < 8; ++j) {
+                    const int t = 16 * (i0 + j) + 2 * warp + hsel;
+                    bits[j] = (t < cnt) ? reinterpret_cast<const uint32_t*>(B.vc + t * TB::VROW)[hl] : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int tt = 16 * (i0 + j) + 2 * warp + hsel;
+                    const bool live = tt < cnt;
+                    const int t = live ? tt : 0;   // weights of absent tokens are 0
+                    // byte offsets 4 e of the eight nibbles: even coordinates in `lo`, odd in `hi`
+                    const uint32_t lo = (bits[j] << 2) & 0x3C3C3C3Cu, hi = (bits[j] >> 2) & 0x3C3C3C3Cu;
+                    float2 cv[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        cv[c] = make_float2(*reinterpret_cast<const float*>(cbase + __byte_perm(lo, 0u, 0x4440u | c)),
+                                            *reinterpret_cast<const float*>(cbase + __byte_perm(hi, 0u, 0x4440u | c)));
+#pragma unroll
+                    for (int q = 0; q < QH; ++q) {
+                        const float wv = live ? wt[q * kThreads + t] : 0.f;
+                        const float2 w2 = make_float2(wv, wv);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const float2 a = __ffma2_rn(w2, cv[c], make_float2(acc[q][2 * c], acc[q][2 * c + 1]));
+                            acc[q][2 * c] = a.x;
+                            acc[q][2 * c + 1] = a.y;
+                        }
                     }
                 }
-                bits[j] = b;
             }
+        } else {
+            // ---- C: value sums, one warp per token, 4 coordinates per lane; 32 tokens per warp ----
+            const int ntok = (cnt - warp + kWarps - 1) / kWarps;   // tokens t = warp + 8 * i < cnt
+            // batches of 8 tokens: the 8 code slices are loaded before their FMAs
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = i0 + j;
-                const int t = (i < ntok) ? warp + i * kWarps : 0;   // weights of absent tokens are 0
-                float cv[4];
-                const char* cbase = reinterpret_cast<const char*>(vc);
-                if constexpr (BV == 4) {
-                    // byte offsets 4 e of the four nibbles: 0 and 2 from `lo`, 1 and 3 from `hi`
-                    const uint32_t lo = (bits[j] << 2) & 0x3C3Cu, hi = (bits[j] >> 2) & 0x3C3Cu;
-                    cv[0] = *reinterpret_cast<const float*>(cbase + (lo & 0xFFu));
-                    cv[1] = *reinterpret_cast<const float*>(cbase + (hi & 0xFFu));
-                    cv[2] = *reinterpret_cast<const float*>(cbase + (lo >> 8));
-                    cv[3] = *reinterpret_cast<const float*>(cbase + (hi >> 8));
-                } else if constexpr (BV == 2) {
-                    const uint32_t b8 = bits[j];
-                    cv[0] = *reinterpret_cast<const float*>(cbase + ((b8 << 2) & 0xCu));
-                    cv[1] = *reinterpret_cast<const float*>(cbase + (b8 & 0xCu));
-                    cv[2] = *reinterpret_cast<const float*>(cbase + ((b8 >> 2) & 0xCu));
-                    cv[3] = *reinterpret_cast<const float*>(cbase + ((b8 >> 4) & 0xCu));
-                } else {
+            for (int i0 = 0; i0 < kThreads / kWarps; i0 += 8) {
+                uint32_t bits[8];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) cv[c] = vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)];
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j;
+                    const int t = warp + i * kWarps;
+                    uint32_t b = 0;
+                    if (i < ntok) {
+                        const uint8_t* row = B.vc + t * TB::VROW;
+                        if constexpr (BV == 2) {
+                            b = row[lane];
+                        } else {
+                            const int b0 = lane * 4 * BV;
+                            const int wi = b0 >> 5, sh = b0 & 31;
+                            const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row);
+                            uint64_t win = r32[wi];
+                            if ((sh + 4 * BV > 32) && (wi + 1) * 32 < kD * BV) win |= (uint64_t)r32[wi + 1] << 32;
+                            b = (uint32_t)(win >> sh);
+                        }
+                    }
+                    bits[j] = b;
                 }
 #pragma unroll
-                for (int q = 0; q < QH; ++q) {
-                    const float wv = (i < ntok) ? wt[q * kThreads + t] : 0.f;
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j;
+                    const int t = (i < ntok) ? warp + i * kWarps : 0;   // weights of absent tokens are 0
+                    float cv[4];
+                    if constexpr (BV == 2) {
+                        const char* cbase = reinterpret_cast<const char*>(vc);
+                        const uint32_t b8 = bits[j];
+                        cv[0] = *reinterpret_cast<const float*>(cbase + ((b8 << 2) & 0xCu));
+                        cv[1] = *reinterpret_cast<const float*>(cbase + (b8 & 0xCu));
+                        cv[2] = *reinterpret_cast<const float*>(cbase + ((b8 >> 2) & 0xCu));
+                        cv[3] = *reinterpret_cast<const float*>(cbase + ((b8 >> 4) & 0xCu));
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[q][c] = fmaf(wv, cv[c], acc[q][c]);
+                        for (int c = 0; c < 4; ++c) cv[c] = vc[(bits[j] >> (BV * c)) & ((1u << BV) - 1u)];
+                    }
+#pragma unroll
+                    for (int q = 0; q < QH; ++q) {
+                        const float wv = (i < ntok) ? wt[q * kThreads + t] : 0.f;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) acc[q][c] = fmaf(wv, cv[c], acc[q][c]);
+                    }
                 }
             }
         }
@@ -290,10 +326,26 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     }
     cp_async_wait0();
     // ---- reduce the warps' value sums and write the split records ----
+    if constexpr (BV == 4) {
+        // the two half-warps hold the same coordinates for different tokens
 #pragma unroll
-    for (int q = 0; q < QH; ++q)
+        for (int q = 0; q < QH; ++q)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) accw[(warp * QH + q) * kD + 4 * lane + c] = acc[q][c];
+            for (int c = 0; c < 8; ++c) acc[q][c] += __shfl_xor_sync(0xffffffffu, acc[q][c], 16);
+        if (lane < 16) {
+#pragma unroll
+            for (int q = 0; q < QH; ++q)
+#pragma unroll
+                for (int c = 0; c < 8; c += 4)
+                    *reinterpret_cast<float4*>(&accw[(warp * QH + q) * kD + 8 * lane + c]) =
+                        make_float4(acc[q][c], acc[q][c + 1], acc[q][c + 2], acc[q][c + 3]);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < QH; ++q)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) accw[(warp * QH + q) * kD + 4 * lane + c] = acc[q][c];
+    }
     __syncthreads();
     for (int j = threadIdx.x; j < QH * kD; j += kThreads) {
         const int q = j / kD, jj = j % kD;

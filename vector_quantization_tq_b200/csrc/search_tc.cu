@@ -176,25 +176,31 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
     } else if (warp >= kExpWarp0) {
         // ---- expanders: key bits -> +-1 bf16 ----
         // K-step g of the CTA (tile tile_begin + g / ks_per_tile, step g % ks_per_tile) needs 8
-        // bytes of one bit plane for each of the tile's 256 keys; each thread handles two keys.
-        // The global loads run kPrefetch steps ahead of the expansion, so their latency overlaps
-        // the work of the steps in between.
-        constexpr int kPrefetch = 4;
+        // bytes of one bit plane for each of the tile's 256 keys; each thread handles one key.
+        // The bytes of four consecutive steps are contiguous in the key's row (d is a multiple of
+        // 256, so a group of four never crosses the plane or the tile), so a thread fetches them
+        // with two 16-byte loads one group ahead of the expansion.
         const int e = threadIdx.x - kExpWarp0 * 32;   // key within the tile, 0..255
         const int64_t nsteps = (tile_end - tile_begin) * ks_per_tile;
-        // The steps are fetched in order, so the fetch position (tile, step) advances by one per
-        // call instead of being divided out of the step index.
+        // The groups are fetched in order, so the fetch position (tile, step) advances by four
+        // per call instead of being divided out of the step index.
         const int row_bytes = p.d / 8;
         int64_t f_tile = tile_begin;   // tile and step of the next fetch
         int f_ks = 0;
-        auto fetch = [&](uint2& bits) {
-            bits = make_uint2(0u, 0u);
+        auto fetch = [&](uint4& lo, uint4& hi) {
+            lo = make_uint4(0u, 0u, 0u, 0u);
+            hi = lo;
             if (f_tile >= tile_end) return;
             const uint8_t* plane = (f_ks < ks_half) ? p.codes : p.qjl;
             const int byte0 = ((f_ks < ks_half) ? f_ks : f_ks - ks_half) * (kBK / 8);
             const int64_t key = f_tile * kBN + e;
-            if (key < p.n) bits = __ldg(reinterpret_cast<const uint2*>(plane + key * row_bytes + byte0));
-            if (++f_ks == ks_per_tile) {
+            if (key < p.n) {
+                const uint4* src = reinterpret_cast<const uint4*>(plane + key * row_bytes + byte0);
+                lo = __ldg(src);
+                hi = __ldg(src + 1);
+            }
+            f_ks += 4;
+            if (f_ks == ks_per_tile) {
                 f_ks = 0;
                 ++f_tile;
             }
@@ -232,20 +238,14 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             }
             return true;
         };
-        uint2 pf[kPrefetch];
-#pragma unroll
-        for (int j = 0; j < kPrefetch; ++j) fetch(pf[j]);
+        uint4 nlo, nhi;
+        fetch(nlo, nhi);
         bool run = true;
-        for (int64_t g0 = 0; g0 < nsteps && run; g0 += kPrefetch) {
-#pragma unroll
-            for (int j = 0; j < kPrefetch; ++j) {
-                const int64_t g = g0 + j;
-                if (run && g < nsteps) {
-                    const uint2 cur = pf[j];
-                    fetch(pf[j]);   // step g + kPrefetch
-                    run = expand(g, cur);
-                }
-            }
+        for (int64_t g0 = 0; g0 < nsteps && run; g0 += 4) {
+            const uint4 clo = nlo, chi = nhi;
+            fetch(nlo, nhi);   // steps g0 + 4 .. g0 + 7
+            run = expand(g0, make_uint2(clo.x, clo.y)) && expand(g0 + 1, make_uint2(clo.z, clo.w)) &&
+                  expand(g0 + 2, make_uint2(chi.x, chi.y)) && expand(g0 + 3, make_uint2(chi.z, chi.w));
         }
     } else {
         // ---- epilogue: warps 2..9, two threads per query (one per half of the tile's keys) ----
