@@ -264,9 +264,10 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
         }
         // Estimates above the current k-th best go to the query's candidate buffer (in key
         // order); the buffer is merged into the sorted list once per tile, after the tile's
-        // accumulator has been released (so the merge overlaps the next tile's MMAs), or when
-        // it fills up. A sorted insertion per key ran divergently for almost every key while
-        // the threshold was low and held the accumulator for tens of thousands of cycles.
+        // accumulator has been released (so the merge overlaps the next tile's MMAs), or by the
+        // whole warp when some lane's buffer could overflow. The result does not depend on when
+        // the merges happen: the threshold is never above the list's k-th best, and the list
+        // takes keys in key order with strict comparisons (ties stay with the lower key).
         float thr = -INFINITY;
         int cnt = 0;
         auto merge = [&]() {
@@ -311,6 +312,10 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
             ptx::tc_fence_after();
 #pragma unroll 1
             for (int c = half * (kBN / 16); c < (half + 1) * (kBN / 16); ++c) {
+                // room for this group's 8 keys: the whole warp merges together (a merge taken by
+                // one lane at a time ran once per lane, serialised, while the first tile filled
+                // the buffers)
+                if (__any_sync(0xffffffffu, cnt > kCand - 8)) merge();
                 uint32_t a1[8], a2[8];
                 ptx::tmem_ld8(t_lane + c * 8, a1);
                 ptx::tmem_ld8(t_lane + 256 + c * 8, a2);
@@ -323,7 +328,7 @@ search_tc_kernel(const __grid_constant__ CUtensorMap tma_q, const SearchParams p
                     if (key < p.n && est > thr) {
                         sm.candv[cnt][col] = est;
                         sm.candi[cnt][col] = (int)key;
-                        if (++cnt == kCand) merge();
+                        ++cnt;
                     }
                 }
             }
