@@ -3,10 +3,11 @@
 // plain matrix product). Used for d >= 512 with bf16-stored Pi and S and bf16 input.
 //
 // C[M x N] = A[M x K] * B[N x K]^T, A and B bf16 K-major in global memory, fp32 accumulate.
-// Warp-specialised CTA of 6 warps per 128 x BN output tile:
+// Warp-specialised CTA of 10 warps per 128 x BN output tile:
 //   warp 0  TMA producer: K-steps of 64 through a 2-stage shared-memory ring (two CTAs per SM);
 //   warp 1  MMA issuer: 4 x tcgen05.mma (M128 N=BN K16) per stage, commit frees the stage;
-//   warps 2-5 epilogue: one TMEM lane (= output row) per thread, 32 columns at a time.
+//   warps 2-9 epilogue: two warps per TMEM lane quadrant, each thread one output row and half
+//           of the tile's columns, 32 at a time.
 // Epilogues:
 //   kStoreF32  C in fp32 (query preparation).
 //   kRotate    y = acc / ||x||, b-bit Lloyd-Max cell, residual r = y - c[idx] written as a
@@ -29,7 +30,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 2;   // 2 x 48 KB: two CTAs per SM, so one's epilogue overlaps the other's MMAs
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 
 enum EpiKind { kStoreF32 = 0, kRotate = 1, kSigns = 2 };
 
@@ -60,6 +61,7 @@ struct __align__(1024) GemmSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t done;
+    float rr_half[kBM];        // the second column half's partial ||r||^2 per row
     uint32_t tmem_base;
     int abort;
 };
@@ -79,6 +81,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     const int nt = blockIdx.x;
     const int n0 = nt * BN;
     const int ksteps = p.K / kBK;
+    static_assert(BN % 64 == 0, "each epilogue column half is a whole number of 32-column chunks");
     constexpr uint32_t kCols = BN;          // power of two >= 32
 
     if (threadIdx.x == 0) {
@@ -137,13 +140,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             ptx::mma_commit(&sm.done);   // arrives once every MMA above has completed
         }
     } else {
-        // ---- epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1 ----
+        // ---- epilogue: warps 2..9; lane quadrant warp % 4, column half (warp - 2) / 4 ----
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const int m = m0 + row;
         bool ok = true;
         if (lane == 0) ok = ptx::mbar_wait(&sm.done, 0);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        float rr = 0.f;
         if (!ok || sm.abort) {
             if (lane == 0) atomicExch(&g_tq_device_error, 1);
         } else {
@@ -154,9 +159,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                 const float nu = (m < p.M) ? __ldg(p.norms + m) : 0.f;
                 inv_nu = (nu > 0.f) ? 1.f / nu : 0.f;
             }
-            float rr = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
                 uint32_t acc[32];
                 ptx::tmem_ld32(t_lane + c * 32, acc);
                 ptx::tmem_wait_ld();
@@ -220,16 +224,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                     reinterpret_cast<uint32_t*>(p.qjl + (size_t)m * (p.N / 8))[ncol / 32] = z;
                 }
             }
-            if constexpr (EPI == kRotate) {
-                if (m < p.M) p.rho_part[(size_t)m * p.n_tiles + nt] = rr;
-            }
             if constexpr (EPI == kSigns) {
-                if (nt == 0 && m < p.M) {
+                if (half == 0 && nt == 0 && m < p.M) {
                     float s = 0.f;
                     for (int t = 0; t < p.n_tiles; ++t) s += p.rho_part[(size_t)m * p.n_tiles + t];
                     p.rnorms[m] = sqrtf(s);
                 }
             }
+        }
+        if constexpr (EPI == kRotate) {
+            // the row's partial ||r||^2 over this N tile: both column halves
+            if (half == 1) sm.rr_half[row] = rr;
+            asm volatile("bar.sync 1, 256;" ::: "memory");   // the eight epilogue warps
+            if (half == 0 && m < p.M) p.rho_part[(size_t)m * p.n_tiles + nt] = rr + sm.rr_half[row];
         }
     }
     ptx::tc_fence_before();
