@@ -722,18 +722,38 @@ def main():
         hs = torch.empty(scores.shape, dtype=scores.dtype).pin_memory()
         dx = torch.empty_like(x)
         dq = torch.empty_like(q)
+        # The batch goes through in groups of heads so that the copies overlap the kernels:
+        # group g's inputs come in on `cin` while group g-1 is encoded and scored on `stream`
+        # and group g-2's planes and scores go out on `cout` (the two copy directions run on
+        # separate copy engines).
+        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        hg = 4 if heads % 4 == 0 else 1
+        groups_e2e = [(h0, h0 + hg) for h0 in range(0, heads, hg)]
+        ev_in = [torch.cuda.Event() for _ in groups_e2e]
+        ev_k = [torch.cuda.Event() for _ in groups_e2e]
 
         def e2e_step():
-            dx.copy_(hx, non_blocking=True)
-            dq.copy_(hq, non_blocking=True)
-            tq.quantize_prod(st, dx, codes, qjl, norms, rnorms, stream=stream)
-            tq.score(st, dq, codes, qjl, norms, rnorms, scores, groups=heads, nq=1, n=TOKENS, stream=stream,
-                     workspace=sws)
-            hc.copy_(codes, non_blocking=True)
-            hz.copy_(qjl, non_blocking=True)
-            hn.copy_(norms, non_blocking=True)
-            hr.copy_(rnorms, non_blocking=True)
-            hs.copy_(scores, non_blocking=True)
+            cin.wait_stream(stream)    # the previous step's kernels are done with dx / dq
+            for g, (h0, h1) in enumerate(groups_e2e):
+                r0, r1 = h0 * TOKENS, h1 * TOKENS
+                with torch.cuda.stream(cin):
+                    dx[r0:r1].copy_(hx[r0:r1], non_blocking=True)
+                    dq[h0:h1].copy_(hq[h0:h1], non_blocking=True)
+                    ev_in[g].record(cin)
+                stream.wait_event(ev_in[g])
+                tq.quantize_prod(st, dx[r0:r1], codes[r0:r1], qjl[r0:r1], norms[r0:r1], rnorms[r0:r1],
+                                 stream=stream)
+                tq.score(st, dq[h0:h1], codes[r0:r1], qjl[r0:r1], norms[r0:r1], rnorms[r0:r1], scores[h0:h1],
+                         groups=h1 - h0, nq=1, n=TOKENS, stream=stream, workspace=sws)
+                ev_k[g].record(stream)
+                cout.wait_event(ev_k[g])
+                with torch.cuda.stream(cout):
+                    hc[r0:r1].copy_(codes[r0:r1], non_blocking=True)
+                    hz[r0:r1].copy_(qjl[r0:r1], non_blocking=True)
+                    hn[r0:r1].copy_(norms[r0:r1], non_blocking=True)
+                    hr[r0:r1].copy_(rnorms[r0:r1], non_blocking=True)
+                    hs[h0:h1].copy_(scores[h0:h1], non_blocking=True)
+            stream.wait_stream(cout)   # the step ends when its results are on the host
 
         for _ in range(3):
             e2e_step()

@@ -81,7 +81,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     const int nt = blockIdx.x;
     const int n0 = nt * BN;
     const int ksteps = p.K / kBK;
-    static_assert(BN % 64 == 0, "each epilogue column half is a whole number of 32-column chunks");
+    static_assert(BN % 128 == 0, "each epilogue column half is a whole number of 32-column chunk pairs");
+    static_assert(sizeof(GemmSmem<BN>::a) + sizeof(GemmSmem<BN>::b) >= 8 * 8192, "epilogue staging fits in the ring");
     constexpr uint32_t kCols = BN;          // power of two >= 32
 
     if (threadIdx.x == 0) {
@@ -164,7 +165,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                 uint32_t acc[32];
                 ptx::tmem_ld32(t_lane + c * 32, acc);
                 ptx::tmem_wait_ld();
-                if (m >= p.M) continue;
+                if (EPI != kRotate && m >= p.M) continue;   // the quantize pass stages every row
                 const int ncol = n0 + c * 32;
                 if constexpr (EPI == kStoreF32) {
                     float4* dst = reinterpret_cast<float4*>(p.c + (size_t)m * p.ldc + ncol);
@@ -203,15 +204,42 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         hi[j >> 1] = hb;
                         lo[j >> 1] = *reinterpret_cast<const uint32_t*>(&l);
                     }
-                    uint4* dh = reinterpret_cast<uint4*>(p.r2 + (size_t)m * 2 * p.N + ncol);
-                    uint4* dl = reinterpret_cast<uint4*>(p.r2 + (size_t)m * 2 * p.N + p.N + ncol);
+                    // The residual of two chunks (64 columns: 128 bytes of hi and of lo per row)
+                    // is staged in this warp's 8 KB of the operand ring, idle once every MMA is
+                    // done, with the row's 16-byte slots rotated by (row % 8) so that the lanes'
+                    // writes fall into different banks; the warp then stores whole 128-byte
+                    // lines, four rows per instruction, instead of 16 bytes per row.
+                    uint8_t* stg = reinterpret_cast<uint8_t*>(sm.a) + (warp - 2) * 8192;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        dh[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-                        dl[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+                        const int slot = (((c & 1) * 4 + j) ^ (lane & 7)) * 16;
+                        *reinterpret_cast<uint4*>(stg + lane * 128 + slot) =
+                            make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+                        *reinterpret_cast<uint4*>(stg + 4096 + lane * 128 + slot) =
+                            make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
                     }
-                    uint32_t* cdst = reinterpret_cast<uint32_t*>(p.codes + (size_t)m * p.code_bytes) + (ncol / 32) * b;
-                    for (int w = 0; w < b; ++w) cdst[w] = cw[w];
+                    if (c & 1) {
+                        __syncwarp();
+                        const int c0 = n0 + (c - 1) * 32;   // first column of the pair
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr8 = 4 * i + (lane >> 3), sl = lane & 7;   // row of the warp, 16-byte slot
+                            const int64_t mr = m0 + quad * 32 + rr8;
+                            const int off = rr8 * 128 + ((sl ^ (rr8 & 7)) * 16);
+                            const uint4 vh = *reinterpret_cast<const uint4*>(stg + off);
+                            const uint4 vl = *reinterpret_cast<const uint4*>(stg + 4096 + off);
+                            if (mr < p.M) {
+                                uint16_t* row = p.r2 + (size_t)mr * 2 * p.N;
+                                *reinterpret_cast<uint4*>(row + c0 + sl * 8) = vh;
+                                *reinterpret_cast<uint4*>(row + p.N + c0 + sl * 8) = vl;
+                            }
+                        }
+                        __syncwarp();   // the staging area is rewritten by the next pair
+                    }
+                    if (m < p.M) {
+                        uint32_t* cdst = reinterpret_cast<uint32_t*>(p.codes + (size_t)m * p.code_bytes) + (ncol / 32) * b;
+                        for (int w = 0; w < b; ++w) cdst[w] = cw[w];
+                    }
                 } else {   // kSigns
                     uint32_t neg = 0u;
 #pragma unroll
