@@ -3,11 +3,15 @@
 // plain matrix product). Used for d >= 512 with bf16-stored Pi and S and bf16 input.
 //
 // C[M x N] = A[M x K] * B[N x K]^T, A and B bf16 K-major in global memory, fp32 accumulate.
-// Warp-specialised CTA of 10 warps per 128 x BN output tile:
-//   warp 0  TMA producer: K-steps of 64 through a 2-stage shared-memory ring (two CTAs per SM);
-//   warp 1  MMA issuer: 4 x tcgen05.mma (M128 N=BN K16) per stage, commit frees the stage;
+// Persistent CTA (one per SM) of 10 warps walking 128 x BN output tiles (N tile fastest, so
+// the CTAs that share an A tile run together and A comes from DRAM once):
+//   warp 0  TMA producer: K-steps of 64 through a shared-memory ring, continuing into the next
+//           tile without draining;
+//   warp 1  MMA issuer: 4 x tcgen05.mma (M128 N=BN K16) per stage into one of two TMEM
+//           accumulators (tiles alternate), commit frees the stage;
 //   warps 2-9 epilogue: two warps per TMEM lane quadrant, each thread one output row and half
-//           of the tile's columns, 32 at a time.
+//           of the tile's columns, 32 at a time, while the MMAs of the next tile run into the
+//           other accumulator.
 // Epilogues:
 //   kStoreF32  C in fp32 (query preparation).
 //   kRotate    y = acc / ||x||, b-bit Lloyd-Max cell, residual r = y - c[idx] written as a
@@ -29,10 +33,16 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 2;   // 2 x 48 KB: two CTAs per SM, so one's epilogue overlaps the other's MMAs
 constexpr int kGemmThreads = 320;
 
 enum EpiKind { kStoreF32 = 0, kRotate = 1, kSigns = 2 };
+
+// Ring depth: the quantize epilogue keeps 64 KB of staging for its residual stores.
+template <int EPI>
+struct GemmCfg {
+    static constexpr int kStages = (EPI == kRotate) ? 3 : 4;
+    static constexpr int kStageBytes = (EPI == kRotate) ? 8 * 8192 : 16;
+};
 
 struct GemmParams {
     int M, N, K;
@@ -54,36 +64,50 @@ struct GemmParams {
     float c_cent[16];
 };
 
-template <int BN>
+template <int BN, int EPI>
 struct __align__(1024) GemmSmem {
-    uint8_t a[kStages][kBM * kBK * 2];
-    uint8_t b[kStages][BN * kBK * 2];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t done;
-    float rr_half[kBM];        // the second column half's partial ||r||^2 per row
+    uint8_t a[GemmCfg<EPI>::kStages][kBM * kBK * 2];
+    uint8_t b[GemmCfg<EPI>::kStages][BN * kBK * 2];
+    uint8_t stage[GemmCfg<EPI>::kStageBytes];   // kRotate: 8 KB of residual staging per epilogue warp
+    uint64_t full[GemmCfg<EPI>::kStages];
+    uint64_t empty[GemmCfg<EPI>::kStages];
+    uint64_t acc_full[2];      // the tile's MMAs are done (commit)
+    uint64_t acc_empty[2];     // the epilogue has read the accumulator (one arrival per warp)
+    float rr_half[2][kBM];     // the second column half's partial ||r||^2 per row, by tile parity
     uint32_t tmem_base;
     int abort;
 };
 
+// Barrier over the eight epilogue warps (named barrier 2) that returns the OR of `pred`.
+__device__ __forceinline__ bool epi_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "barrier.cta.red.or.pred po, 2, 256, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
 // BQ: code width of the kRotate epilogue (compile-time, so the code words stay in registers).
 template <int BN, int EPI, int BQ>
-__global__ void __launch_bounds__(kGemmThreads, 2)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                const GemmParams p) {
+    using Cfg = GemmCfg<EPI>;
+    constexpr int kStages = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
-    GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                        ~uintptr_t(1023));
+    GemmSmem<BN, EPI>& sm = *reinterpret_cast<GemmSmem<BN, EPI>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                                ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // The N tile varies fastest: the CTAs that share an A tile run together, so A comes from
-    // DRAM once and from L2 for the other N tiles.
-    const int m0 = blockIdx.y * kBM;
-    const int nt = blockIdx.x;
-    const int n0 = nt * BN;
+    const int ntn = p.N / BN;
+    const int64_t ntiles = (int64_t)((p.M + kBM - 1) / kBM) * ntn;
     const int ksteps = p.K / kBK;
-    static_assert(BN % 128 == 0, "each epilogue column half is a whole number of 32-column chunk pairs");
-    static_assert(sizeof(GemmSmem<BN>::a) + sizeof(GemmSmem<BN>::b) >= 8 * 8192, "epilogue staging fits in the ring");
-    constexpr uint32_t kCols = BN;          // power of two >= 32
+    constexpr uint32_t kCols = 2 * BN;      // two accumulators
+    static_assert(BN % 128 == 0 && 2 * BN <= 512, "two accumulators of BN columns; chunk pairs per column half");
 
     if (threadIdx.x == 0) {
         ptx::prefetch_tmap(&tma_a);
@@ -92,7 +116,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             ptx::mbar_init(&sm.full[s], 1);
             ptx::mbar_init(&sm.empty[s], 1);
         }
-        ptx::mbar_init(&sm.done, 1);
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&sm.acc_full[a], 1);
+            ptx::mbar_init(&sm.acc_empty[a], 8);   // one arrival per epilogue warp
+        }
         sm.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -106,60 +133,81 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0) {
+        // ---- TMA producer: the K steps of every tile of this CTA, one ring position each ----
         if (lane == 0) {
-            for (int ks = 0; ks < ksteps; ++ks) {
-                const int s = ks % kStages;
-                if (ks >= kStages && !ptx::mbar_wait(&sm.empty[s], ((ks / kStages) - 1) & 1)) {
-                    atomicExch(&sm.abort, 1);
-                    break;
+            int64_t g = 0;
+            for (int64_t t = blockIdx.x; t < ntiles && !sm.abort; t += gridDim.x) {
+                const int m0 = (int)(t / ntn) * kBM, n0 = (int)(t % ntn) * BN;
+                for (int ks = 0; ks < ksteps; ++ks, ++g) {
+                    const int s = (int)(g % kStages);
+                    if (g >= kStages && !ptx::mbar_wait(&sm.empty[s], (uint32_t)(((g / kStages) - 1) & 1))) {
+                        atomicExch(&sm.abort, 1);
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&sm.full[s], (kBM + BN) * kBK * 2);
+                    ptx::tma_load_2d(sm.a[s], &tma_a, ks * kBK, m0, &sm.full[s]);
+                    ptx::tma_load_2d(sm.b[s], &tma_b, (ks * kBK) % p.b_kwrap, n0, &sm.full[s]);
                 }
-                if (sm.abort) break;
-                ptx::mbar_arrive_expect_tx(&sm.full[s], (kBM + BN) * kBK * 2);
-                ptx::tma_load_2d(sm.a[s], &tma_a, ks * kBK, m0, &sm.full[s]);
-                ptx::tma_load_2d(sm.b[s], &tma_b, (ks * kBK) % p.b_kwrap, n0, &sm.full[s]);
             }
         }
     } else if (warp == 1) {
+        // ---- MMA issue: tile i accumulates into columns [BN (i % 2), BN (i % 2) + BN) ----
         if (lane == 0) {
             const uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN);
-            int ks = 0;
-            for (; ks < ksteps; ++ks) {
-                const int s = ks % kStages;
-                if (!ptx::mbar_wait(&sm.full[s], (ks / kStages) & 1)) {
+            int64_t g = 0, i = 0;
+            for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+                const int acc = (int)(i & 1);
+                if (i >= 2 && !ptx::mbar_wait(&sm.acc_empty[acc], (uint32_t)(((i >> 1) - 1) & 1)))
                     atomicExch(&sm.abort, 1);
-                    break;
-                }
+                if (sm.abort) break;
                 ptx::tc_fence_after();
-                const uint32_t a_addr = ptx::smem_addr(sm.a[s]);
-                const uint32_t b_addr = ptx::smem_addr(sm.b[s]);
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                for (int ks = 0; ks < ksteps; ++ks, ++g) {
+                    const int s = (int)(g % kStages);
+                    if (!ptx::mbar_wait(&sm.full[s], (uint32_t)((g / kStages) & 1))) {
+                        atomicExch(&sm.abort, 1);
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_addr(sm.a[s]);
+                    const uint32_t b_addr = ptx::smem_addr(sm.b[s]);
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    ptx::mma_ss(tmem, ptx::smem_desc_kmajor_sw128(a_addr + kk * 32),
-                                ptx::smem_desc_kmajor_sw128(b_addr + kk * 32), idesc, (ks | kk) ? 1u : 0u);
-                ptx::mma_commit(&sm.empty[s]);
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        ptx::mma_ss(d_tmem, ptx::smem_desc_kmajor_sw128(a_addr + kk * 32),
+                                    ptx::smem_desc_kmajor_sw128(b_addr + kk * 32), idesc, (ks | kk) ? 1u : 0u);
+                    ptx::mma_commit(&sm.empty[s]);
+                }
+                if (sm.abort) break;
+                ptx::mma_commit(&sm.acc_full[acc]);   // arrives once every MMA above has completed
             }
-            ptx::mma_commit(&sm.done);   // arrives once every MMA above has completed
         }
     } else {
         // ---- epilogue: warps 2..9; lane quadrant warp % 4, column half (warp - 2) / 4 ----
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
-        const int m = m0 + row;
-        bool ok = true;
-        if (lane == 0) ok = ptx::mbar_wait(&sm.done, 0);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        float rr = 0.f;
-        if (!ok || sm.abort) {
-            if (lane == 0) atomicExch(&g_tq_device_error, 1);
-        } else {
+        const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+        int64_t i = 0;
+        bool failed = false;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+            const int acc_i = (int)(i & 1);
+            const int m0 = (int)(t / ntn) * kBM, nt = (int)(t % ntn), n0 = nt * BN;
+            const int m = m0 + row;
+            bool ok = true;
+            if (lane == 0) ok = ptx::mbar_wait(&sm.acc_full[acc_i], (uint32_t)((i >> 1) & 1));
+            // the eight epilogue warps stop together (they meet at a named barrier per tile)
+            if (epi_sync_or(!ok || sm.abort)) {
+                failed = true;
+                break;
+            }
             ptx::tc_fence_after();
-            const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+            const uint32_t t_lane = t_quad + (uint32_t)(acc_i * BN);
             float inv_nu = 0.f;
             if constexpr (EPI == kRotate) {
                 const float nu = (m < p.M) ? __ldg(p.norms + m) : 0.f;
                 inv_nu = (nu > 0.f) ? 1.f / nu : 0.f;
             }
+            float rr = 0.f;
 #pragma unroll 1
             for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
                 uint32_t acc[32];
@@ -205,11 +253,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         lo[j >> 1] = *reinterpret_cast<const uint32_t*>(&l);
                     }
                     // The residual of two chunks (64 columns: 128 bytes of hi and of lo per row)
-                    // is staged in this warp's 8 KB of the operand ring, idle once every MMA is
-                    // done, with the row's 16-byte slots rotated by (row % 8) so that the lanes'
-                    // writes fall into different banks; the warp then stores whole 128-byte
-                    // lines, four rows per instruction, instead of 16 bytes per row.
-                    uint8_t* stg = reinterpret_cast<uint8_t*>(sm.a) + (warp - 2) * 8192;
+                    // is staged in this warp's 8 KB, with the row's 16-byte slots rotated by
+                    // (row % 8) so that the lanes' writes fall into different banks; the warp then
+                    // stores whole 128-byte lines, four rows per instruction, instead of 16 bytes
+                    // per row.
+                    uint8_t* stg = sm.stage + (warp - 2) * 8192;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int slot = (((c & 1) * 4 + j) ^ (lane & 7)) * 16;
@@ -222,16 +270,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         __syncwarp();
                         const int c0 = n0 + (c - 1) * 32;   // first column of the pair
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int rr8 = 4 * i + (lane >> 3), sl = lane & 7;   // row of the warp, 16-byte slot
+                        for (int k = 0; k < 8; ++k) {
+                            const int rr8 = 4 * k + (lane >> 3), sl = lane & 7;   // row of the warp, 16-byte slot
                             const int64_t mr = m0 + quad * 32 + rr8;
                             const int off = rr8 * 128 + ((sl ^ (rr8 & 7)) * 16);
                             const uint4 vh = *reinterpret_cast<const uint4*>(stg + off);
                             const uint4 vl = *reinterpret_cast<const uint4*>(stg + 4096 + off);
                             if (mr < p.M) {
-                                uint16_t* row = p.r2 + (size_t)mr * 2 * p.N;
-                                *reinterpret_cast<uint4*>(row + c0 + sl * 8) = vh;
-                                *reinterpret_cast<uint4*>(row + p.N + c0 + sl * 8) = vl;
+                                uint16_t* rowp = p.r2 + (size_t)mr * 2 * p.N;
+                                *reinterpret_cast<uint4*>(rowp + c0 + sl * 8) = vh;
+                                *reinterpret_cast<uint4*>(rowp + p.N + c0 + sl * 8) = vl;
                             }
                         }
                         __syncwarp();   // the staging area is rewritten by the next pair
@@ -252,20 +300,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                     reinterpret_cast<uint32_t*>(p.qjl + (size_t)m * (p.N / 8))[ncol / 32] = z;
                 }
             }
+            // the accumulator is free for tile i + 2 once every epilogue warp has read it
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_addr(&sm.acc_empty[acc_i]))
+                             : "memory");
             if constexpr (EPI == kSigns) {
                 if (half == 0 && nt == 0 && m < p.M) {
-                    float s = 0.f;
-                    for (int t = 0; t < p.n_tiles; ++t) s += p.rho_part[(size_t)m * p.n_tiles + t];
-                    p.rnorms[m] = sqrtf(s);
+                    float sq = 0.f;
+                    for (int k = 0; k < p.n_tiles; ++k) sq += p.rho_part[(size_t)m * p.n_tiles + k];
+                    p.rnorms[m] = sqrtf(sq);
                 }
             }
+            if constexpr (EPI == kRotate) {
+                // the row's partial ||r||^2 over this N tile: both column halves (the buffer
+                // alternates with the tile, so one barrier per tile orders its writes and reads)
+                if (half == 1) sm.rr_half[acc_i][row] = rr;
+                asm volatile("bar.sync 1, 256;" ::: "memory");   // the eight epilogue warps
+                if (half == 0 && m < p.M) p.rho_part[(size_t)m * p.n_tiles + nt] = rr + sm.rr_half[acc_i][row];
+            }
         }
-        if constexpr (EPI == kRotate) {
-            // the row's partial ||r||^2 over this N tile: both column halves
-            if (half == 1) sm.rr_half[row] = rr;
-            asm volatile("bar.sync 1, 256;" ::: "memory");   // the eight epilogue warps
-            if (half == 0 && m < p.M) p.rho_part[(size_t)m * p.n_tiles + nt] = rr + sm.rr_half[row];
-        }
+        if (failed && lane == 0) atomicExch(&g_tq_device_error, 1);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -314,7 +370,7 @@ int run_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, const GemmP
     e = make_map(&tb, B, p.N, p.K, ldb, BN);
     if (e) return e;
     auto kern = gemm_tc_kernel<BN, EPI, BQ>;
-    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+    const size_t smem = sizeof(GemmSmem<BN, EPI>) + 1024;
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -323,9 +379,10 @@ int run_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, const GemmP
         if (ce != cudaSuccess) return (int)ce;
         attr_dev = dev;
     }
-    const int64_t mtiles = (p.M + kBM - 1) / kBM;
-    if (mtiles > 65535) return (int)cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)(p.N / BN), (unsigned)mtiles);
+    const int64_t ntiles = (int64_t)((p.M + kBM - 1) / kBM) * (p.N / BN);
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = (int)std::min<int64_t>(ntiles, (int64_t)(sms > 0 ? sms : 148));
     kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, p);
     return (int)cudaGetLastError();
 }
