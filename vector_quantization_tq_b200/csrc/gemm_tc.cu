@@ -37,11 +37,12 @@ constexpr int kGemmThreads = 320;
 
 enum EpiKind { kStoreF32 = 0, kRotate = 1, kSigns = 2 };
 
-// Ring depth: the quantize epilogue keeps 64 KB of staging for its residual stores.
+// Ring depth 4 (the TMA latency from L2 is about three steps' MMAs); the quantize epilogue
+// keeps 4 KB per warp of staging for its residual stores.
 template <int EPI>
 struct GemmCfg {
-    static constexpr int kStages = (EPI == kRotate) ? 3 : 4;
-    static constexpr int kStageBytes = (EPI == kRotate) ? 8 * 8192 : 16;
+    static constexpr int kStages = 4;
+    static constexpr int kStageBytes = (EPI == kRotate) ? 8 * 4096 : 16;
 };
 
 struct GemmParams {
@@ -68,7 +69,7 @@ template <int BN, int EPI>
 struct __align__(1024) GemmSmem {
     uint8_t a[GemmCfg<EPI>::kStages][kBM * kBK * 2];
     uint8_t b[GemmCfg<EPI>::kStages][BN * kBK * 2];
-    uint8_t stage[GemmCfg<EPI>::kStageBytes];   // kRotate: 8 KB of residual staging per epilogue warp
+    uint8_t stage[GemmCfg<EPI>::kStageBytes];   // kRotate: 4 KB of residual staging per epilogue warp
     uint64_t full[GemmCfg<EPI>::kStages];
     uint64_t empty[GemmCfg<EPI>::kStages];
     uint64_t acc_full[2];      // the tile's MMAs are done (commit)
@@ -107,7 +108,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     const int64_t ntiles = (int64_t)((p.M + kBM - 1) / kBM) * ntn;
     const int ksteps = p.K / kBK;
     constexpr uint32_t kCols = 2 * BN;      // two accumulators
-    static_assert(BN % 128 == 0 && 2 * BN <= 512, "two accumulators of BN columns; chunk pairs per column half");
+    static_assert(BN % 64 == 0 && 2 * BN <= 512, "two accumulators of BN columns; whole chunks per column half");
 
     if (threadIdx.x == 0) {
         ptx::prefetch_tmap(&tma_a);
@@ -252,38 +253,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         hi[j >> 1] = hb;
                         lo[j >> 1] = *reinterpret_cast<const uint32_t*>(&l);
                     }
-                    // The residual of two chunks (64 columns: 128 bytes of hi and of lo per row)
-                    // is staged in this warp's 8 KB, with the row's 16-byte slots rotated by
-                    // (row % 8) so that the lanes' writes fall into different banks; the warp then
-                    // stores whole 128-byte lines, four rows per instruction, instead of 16 bytes
-                    // per row.
-                    uint8_t* stg = sm.stage + (warp - 2) * 8192;
+                    // The chunk's residual (64 bytes of hi and of lo per row) is staged in this
+                    // warp's 4 KB, each row's 16-byte slots rotated by (row / 2) % 4 so that a
+                    // quarter-warp's writes fall into different banks; the warp then stores
+                    // 64-byte row pieces (two whole sectors), eight rows per instruction, instead
+                    // of 16 bytes per row.
+                    uint8_t* stg = sm.stage + (warp - 2) * 4096;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const int slot = (((c & 1) * 4 + j) ^ (lane & 7)) * 16;
-                        *reinterpret_cast<uint4*>(stg + lane * 128 + slot) =
+                        const int slot = (j ^ ((lane >> 1) & 3)) * 16;
+                        *reinterpret_cast<uint4*>(stg + lane * 64 + slot) =
                             make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-                        *reinterpret_cast<uint4*>(stg + 4096 + lane * 128 + slot) =
+                        *reinterpret_cast<uint4*>(stg + 2048 + lane * 64 + slot) =
                             make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
                     }
-                    if (c & 1) {
-                        __syncwarp();
-                        const int c0 = n0 + (c - 1) * 32;   // first column of the pair
+                    __syncwarp();
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int rr8 = 4 * k + (lane >> 3), sl = lane & 7;   // row of the warp, 16-byte slot
-                            const int64_t mr = m0 + quad * 32 + rr8;
-                            const int off = rr8 * 128 + ((sl ^ (rr8 & 7)) * 16);
-                            const uint4 vh = *reinterpret_cast<const uint4*>(stg + off);
-                            const uint4 vl = *reinterpret_cast<const uint4*>(stg + 4096 + off);
-                            if (mr < p.M) {
-                                uint16_t* rowp = p.r2 + (size_t)mr * 2 * p.N;
-                                *reinterpret_cast<uint4*>(rowp + c0 + sl * 8) = vh;
-                                *reinterpret_cast<uint4*>(rowp + p.N + c0 + sl * 8) = vl;
-                            }
+                    for (int k = 0; k < 4; ++k) {
+                        const int r8 = 8 * k + (lane >> 2), sl = lane & 3;   // row of the warp, 16-byte slot
+                        const int64_t mr = m0 + quad * 32 + r8;
+                        const int off = r8 * 64 + ((sl ^ ((r8 >> 1) & 3)) * 16);
+                        const uint4 vh = *reinterpret_cast<const uint4*>(stg + off);
+                        const uint4 vl = *reinterpret_cast<const uint4*>(stg + 2048 + off);
+                        if (mr < p.M) {
+                            uint16_t* rowp = p.r2 + (size_t)mr * 2 * p.N;
+                            *reinterpret_cast<uint4*>(rowp + ncol + sl * 8) = vh;
+                            *reinterpret_cast<uint4*>(rowp + p.N + ncol + sl * 8) = vl;
                         }
-                        __syncwarp();   // the staging area is rewritten by the next pair
                     }
+                    __syncwarp();   // the staging area is rewritten by the next chunk
                     if (m < p.M) {
                         uint32_t* cdst = reinterpret_cast<uint32_t*>(p.codes + (size_t)m * p.code_bytes) + (ncol / 32) * b;
                         for (int w = 0; w < b; ++w) cdst[w] = cw[w];
