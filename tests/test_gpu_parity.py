@@ -240,6 +240,19 @@ def test_dense_tiled_encoder_many_tiles(d, b, mode):
     check_codes(pair, gpu, enc)
 
 
+@pytest.mark.parametrize("b,mode", [(2, tq.PROD), (3, tq.PROD), (4, tq.MSE)])
+def test_dense_gemm_encoder_many_tiles(b, mode):
+    # d = 512 on the tensor-core encoder: 297 row tiles of 128 (the last one ragged) x 2 column
+    # tiles over at most one persistent block per SM, so every block takes several tiles and
+    # reuses both accumulators and every ring stage more than once
+    d, n = 512, 148 * 128 * 2 + 77
+    pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.BF16)
+    bits = synth.bf16_bits(synth.unit_vectors(n, d, seed=322).astype(np.float32))
+    enc = pair.encode(synth.bf16_from_bits(bits))
+    gpu, _ = gpu_encode(pair, dev_bf16(bits), n)
+    check_codes(pair, gpu, enc)
+
+
 def test_empty_inputs_are_noops():
     pair = Pair(tq, 128, 3, tq.MSE, tq.ROT_DENSE, tq.F32)
     x = torch.empty((0, 128), dtype=torch.float32, device="cuda")
