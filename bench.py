@@ -577,7 +577,8 @@ def measure_c4(tq, torch, dev, stream):
                 else:
                     enc = lambda: tq.quantize_prod(st, x, codes, qjl, norms, rnorms, stream=stream)  # noqa: E731
                 enc_ms = time_on_stream(torch, enc, stream, dev, 3, 1)
-                tq.dequant(st, codes, qjl, norms, rnorms, xt, stream=stream)
+                dec = lambda: tq.dequant(st, codes, qjl, norms, rnorms, xt, stream=stream)  # noqa: E731
+                dec_ms = time_on_stream(torch, dec, stream, dev, 3, 1)
                 tq.ip_stats(x, xt, q, sums, device=dev.index, stream=stream)
                 torch.cuda.synchronize(dev)
                 s = sums.cpu().numpy()
@@ -590,7 +591,8 @@ def measure_c4(tq, torch, dev, stream):
                              "D_prod": s[3] / n_pairs if mode == tq.PROD else None,
                              "slope": s[4] / s[5], "mean_ip_err": mean_e,
                              "sd_ip_err": math.sqrt(max(0.0, s[3] / n_pairs - mean_e ** 2)),
-                             "encode_ms": enc_ms, "encode_mvec_s": C4_N / (enc_ms / 1e3) / 1e6})
+                             "encode_ms": enc_ms, "encode_mvec_s": C4_N / (enc_ms / 1e3) / 1e6,
+                             "decode_ms": dec_ms, "decode_mvec_s": C4_N / (dec_ms / 1e3) / 1e6})
                 st.close()
     return {"workload": "distortion / bias sweep: 2^20 uniform unit vectors, d=128 and 256, b=1..4, mse and prod, "
                         "dense Haar Pi, 1024 unit queries (statistics on the device)", "rows": rows}

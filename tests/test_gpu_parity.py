@@ -230,14 +230,17 @@ def test_general_paths(d, b, mode, rot, md, bf16_in):
 
 @pytest.mark.parametrize("d,b,mode", [(128, 2, tq.MSE), (128, 4, tq.PROD), (256, 3, tq.MSE), (256, 2, tq.PROD)])
 def test_dense_tiled_encoder_many_tiles(d, b, mode):
-    # more tiles (128 vectors at d = 128, 64 at d = 256) than SMs, so every persistent block
-    # walks several, plus a ragged tail
+    # more tiles (128 vectors at d = 128, 64 at d = 256) than SMs, so every persistent block of
+    # the tiled encoder and dequantizer walks several, plus a ragged tail
     n = 148 * 128 * 2 + 77
     pair = Pair(tq, d, b, mode, tq.ROT_DENSE, tq.F32)
     x = synth.unit_vectors(n, d, seed=321).astype(np.float32)
     enc = pair.encode(x.astype(np.float64))
     gpu, _ = gpu_encode(pair, dev_f32(x), n)
     check_codes(pair, gpu, enc)
+    # the tiled dequantizer over the same tiles: the oracle's planes back to vectors
+    xt_g = gpu_dequant(pair, planes_to_dev(pair.packed(enc)), n)
+    assert np.max(rel_l2(xt_g, pair.decode(enc))) <= REL_L2
 
 
 @pytest.mark.parametrize("b,mode", [(2, tq.PROD), (3, tq.PROD), (4, tq.MSE)])

@@ -874,9 +874,17 @@ int launch_encode_residual(const DevState& st, const void* x, int dtype, int64_t
     });
 }
 
+bool dequant_dense_supported(const DevState& st, int64_t n, const int32_t* chan, int64_t ldo);
+int launch_dequant_dense(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
+                         const float* rnorms, int64_t n, int64_t ldo, float* out, void* stream);
+
 int launch_dequant(const DevState& st, const uint8_t* codes, const uint8_t* qjl, const float* norms,
                    const float* rnorms, int64_t n, const int32_t* chan, int64_t ldo, float* out, void* stream) {
     cudaStream_t s = (cudaStream_t)stream;
+    // d = 128 / 256 with dense fp32 matrices: the tiled dequantizer (both products as
+    // register-tiled GEMMs over a tile of vectors)
+    if (dequant_dense_supported(st, n, chan, ldo))
+        return launch_dequant_dense(st, codes, qjl, norms, rnorms, n, ldo, out, stream);
     return with_layout(st.d, [&](auto e, auto nt) {
         return launch_dequant_t<decltype(e)::value, decltype(nt)::value>(st, codes, qjl, norms, rnorms, n, chan,
                                                                           ldo, out, s);
