@@ -303,6 +303,87 @@ tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, floa
     }
 }
 
+// The same tables without an append, split over kParts blocks per query (grid count x kParts):
+// block p writes the quarter p of the code-group tables and the QJL tables of nibbles
+// 8p .. 8p + 7, so it needs all of q' but only u_j for j in [32p, 32p + 32). The matrices are
+// read from L2 (no staging): q' = Pi q by the whole block (or the Hadamard transform by one
+// warp), u_j = sum_k S^T[k][j] q'_k by 8 threads per output.
+constexpr int kParts = 4;
+
+template <int B, bool PROD>
+__global__ void __launch_bounds__(kThreads)
+tables128_part_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts) {
+    using Gr = Groups<B>;
+    using LS = LutShape<kD128, B, PROD>;
+    static_assert(LS::NG % kParts == 0 && LS::NQ % kParts == 0, "whole tables per part");
+    __shared__ float ctab[16];
+    __shared__ float qs[kD128], qp[kD128], part[2 * kD128], uq[kD128 / kParts];
+    __shared__ float upart[8][kD128 / kParts];
+    const int64_t qi = blockIdx.x;
+    const int pt = blockIdx.y;
+    if (threadIdx.x < 16) ctab[threadIdx.x] = (threadIdx.x < st.L) ? st.c[threadIdx.x] : 0.f;
+    if (threadIdx.x < kD128) {
+        const int i = threadIdx.x;
+        qs[i] = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + qi * kD128 + i)
+                                   : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + qi * kD128 + i));
+    }
+    __syncthreads();
+    if (st.rot != TQ_ROT_RHT) {
+        matvec128(reinterpret_cast<const unsigned char*>(st.piT), st.mat_dtype, qs, part, qp);
+    } else {
+        if (threadIdx.x < 32) warp_rht128(st, qs, qp);
+        __syncthreads();
+    }
+    if constexpr (PROD) {
+        // u_j, j = 32 pt + jl: thread (jl, h) sums k in [16 h, 16 h + 16)
+        constexpr int kJ = kD128 / kParts;
+        const int jl = threadIdx.x % kJ, h = threadIdx.x / kJ;
+        const int j = pt * kJ + jl;
+        float a = 0.f;
+        if (st.mat_dtype == TQ_F32) {
+            const float* m = reinterpret_cast<const float*>(st.sT) + (size_t)(16 * h) * kD128 + j;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) a = fmaf(__ldg(m + k * kD128), qp[16 * h + k], a);
+        } else {
+            const uint16_t* m = reinterpret_cast<const uint16_t*>(st.sT) + (size_t)(16 * h) * kD128 + j;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) a = fmaf(bf16_bits_to_float(__ldg(m + k * kD128)), qp[16 * h + k], a);
+        }
+        upart[h][jl] = a;
+        __syncthreads();
+        if (threadIdx.x < kJ) {
+            float sum = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 8; ++hh) sum += upart[hh][threadIdx.x];
+            uq[threadIdx.x] = sum;
+        }
+        __syncthreads();
+    }
+    float* out = luts + qi * LS::SIZE;
+    constexpr int kMsePart = LS::MSE / kParts;
+    for (int i = pt * kMsePart + threadIdx.x; i < (pt + 1) * kMsePart; i += kThreads) {
+        const int k = i / Gr::E, e = i % Gr::E;
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < Gr::CPG; ++c)
+            a = fmaf(qp[k * Gr::CPG + c], ctab[(e >> (B * c)) & ((1 << B) - 1)], a);
+        out[i] = a;
+    }
+    if constexpr (PROD) {
+        constexpr int kQjlPart = LS::QJL / kParts;   // 8 nibble tables of 16
+        for (int i = threadIdx.x; i < kQjlPart; i += kThreads) {
+            const int kl = i / 16, e = i % 16;   // nibble 8 pt + kl: u_j for j = 4 (8 pt + kl) + c
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = uq[4 * kl + c];
+                a += ((e >> c) & 1) ? v : -v;
+            }
+            out[LS::MSE + pt * kQjlPart + i] = a;
+        }
+    }
+}
+
 // Shared memory of tables128_kernel: the two staged matrices, the level table, q, q', u and
 // the matrix-vector halves, then (appending) the block encoder's buffers.
 size_t tables128_smem(const DevState& st, bool append) {
@@ -317,13 +398,7 @@ int launch_tables(const DevState& st, const void* q, int qdtype, int64_t count, 
     if (count <= 0) return 0;
     if (count > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
     if constexpr (D == kD128) {
-        auto k = tables128_kernel<B, PROD, false>;
-        const size_t smem = tables128_smem(st, false);
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return (int)e;
-        }
-        k<<<(unsigned)count, kThreads, smem, s>>>(st, q, qdtype, luts, st, AppendRow{});
+        tables128_part_kernel<B, PROD><<<dim3((unsigned)count, kParts), kThreads, 0, s>>>(st, q, qdtype, luts);
     } else {
         auto k = score_prep_kernel<D, B, PROD>;
         const size_t smem = (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
