@@ -585,27 +585,63 @@ attend_values_kernel(const DevState vs, const float* __restrict__ scores, float 
     }
 }
 
+// Shared memory of attend_combine_kernel: o[d], partial sums [max(256, d)], the splits'
+// weights [nsplit], a reduction scratch [32].
+size_t combine_smem_bytes(int d, int nsplit) { return (size_t)(d + std::max(256, d) + nsplit + 32) * sizeof(float); }
+
+// Merge of the splits' (m, l, acc[d]) records per head, then out = Pi_V^T o. The splits are
+// reduced in parallel: their maxima and weights exp(m_s - M) by a block reduction, the value
+// sums by P = 256 / d groups of threads over interleaved splits (independent loads in flight).
 __global__ void __launch_bounds__(256)
 attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ part, const int32_t* __restrict__ chan,
                       int64_t ldo, float* __restrict__ out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int d = vs.d;
     const int h = blockIdx.x;
+    const int tid = threadIdx.x, nt = blockDim.x;
     float* o = reinterpret_cast<float*>(smem_raw);   // d
-    const float* base = part + (int64_t)h * nsplit * (d + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (d + 2)]);
-    float Lsum = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float m = base[s * (d + 2)];
-        if (m != -INFINITY) Lsum += base[s * (d + 2) + 1] * __expf(m - M);
+    float* acc = o + d;                               // max(nt, d)
+    float* w = acc + (nt > d ? nt : d);               // nsplit
+    float* red = w + nsplit;                          // 32
+    const int64_t rs = d + 2;
+    const float* base = part + (int64_t)h * nsplit * rs;
+    float mloc = -INFINITY;
+    for (int s = tid; s < nsplit; s += nt) mloc = fmaxf(mloc, base[s * rs]);
+    mloc = warp_max(mloc);
+    if ((tid & 31) == 0) red[tid >> 5] = mloc;
+    __syncthreads();
+    float M = red[0];
+    for (int i = 1; i < nt / 32; ++i) M = fmaxf(M, red[i]);
+    __syncthreads();   // red is reused for the sum
+    float lloc = 0.f;
+    for (int s = tid; s < nsplit; s += nt) {
+        const float m = base[s * rs];
+        const float wt = (m == -INFINITY) ? 0.f : __expf(m - M);
+        w[s] = wt;
+        lloc = fmaf(base[s * rs + 1], wt, lloc);
     }
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        float a = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float m = base[s * (d + 2)];
-            if (m != -INFINITY) a = fmaf(base[s * (d + 2) + 2 + j], __expf(m - M), a);
+    lloc = warp_sum(lloc);
+    if ((tid & 31) == 0) red[tid >> 5] = lloc;
+    __syncthreads();   // also publishes w
+    float Lsum = 0.f;
+    for (int i = 0; i < nt / 32; ++i) Lsum += red[i];
+    const int P = (d < nt) ? nt / d : 1;
+    for (int idx = tid; idx < P * d; idx += nt) {
+        const int j = idx % d, p = idx / d;
+        float a0 = 0.f, a1 = 0.f;
+        int s = p;
+#pragma unroll 4
+        for (; s + P < nsplit; s += 2 * P) {
+            a0 = fmaf(w[s], base[s * rs + 2 + j], a0);
+            a1 = fmaf(w[s + P], base[(s + P) * rs + 2 + j], a1);
         }
+        if (s < nsplit) a0 = fmaf(w[s], base[s * rs + 2 + j], a0);
+        acc[idx] = a0 + a1;
+    }
+    __syncthreads();
+    for (int j = tid; j < d; j += nt) {
+        float a = 0.f;
+        for (int p = 0; p < P; ++p) a += acc[p * d + j];
         o[j] = a / Lsum;
     }
     __syncthreads();
@@ -628,9 +664,13 @@ attend_combine_kernel(const DevState vs, int nsplit, const float* __restrict__ p
             out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = (rht_neg(vs, k) ? -o[k] : o[k]) * vs.rsqrt_d;
     } else {
         for (int k = threadIdx.x; k < d; k += blockDim.x) {
-            float a = 0.f;
-            for (int j = 0; j < d; ++j) a = fmaf(mat_elem(vs.pi, vs.mat_dtype, (int64_t)j * d + k), o[j], a);
-            out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = a;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+            for (int j = 0; j < d; j += 2) {   // d is even
+                a0 = fmaf(mat_elem(vs.pi, vs.mat_dtype, (int64_t)j * d + k), o[j], a0);
+                a1 = fmaf(mat_elem(vs.pi, vs.mat_dtype, (int64_t)(j + 1) * d + k), o[j + 1], a1);
+            }
+            out[(int64_t)h * ldo + (chan ? __ldg(chan + k) : k)] = a0 + a1;
         }
     }
 }
@@ -1027,7 +1067,7 @@ int launch_attend(const DevState& ks, const DevState& vs, const void* q, int qdt
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return (int)e;
-    attend_combine_kernel<<<H, 256, vs.d * sizeof(float), s>>>(vs, nsplit, part, nullptr, vs.d, out);
+    attend_combine_kernel<<<H, 256, combine_smem_bytes(vs.d, nsplit), s>>>(vs, nsplit, part, nullptr, vs.d, out);
     return (int)cudaGetLastError();
 }
 
@@ -1089,8 +1129,8 @@ int launch_split_attend(const DevState& ko, const DevState& ki, const int32_t* k
         dim3 grid((unsigned)nsplit, (unsigned)H);
         attend_values_kernel<<<grid, kAttThreads, smem, s>>>(v, scores, scale, T, chunk, vp.codes[g], vp.norms[g],
                                                              part);
-        attend_combine_kernel<<<H, 256, v.d * sizeof(float), s>>>(v, nsplit, part, g ? vchan + vo.d : vchan, dv,
-                                                                  out);
+        attend_combine_kernel<<<H, 256, combine_smem_bytes(v.d, nsplit), s>>>(v, nsplit, part,
+                                                                             g ? vchan + vo.d : vchan, dv, out);
     }
     return (int)cudaGetLastError();
 }
