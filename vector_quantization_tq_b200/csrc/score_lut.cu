@@ -80,30 +80,11 @@ score_prep_kernel(const DevState st, const void* __restrict__ q, int qdtype, flo
     }
 }
 
-// d = 128: the same preparation with the d x d matrices staged whole in shared memory,
-// every load of a thread in flight at once, the RHT butterfly done by one warp with
-// shuffles, and the matrix-vector products split over all 256 threads.
+// d = 128: the same preparation split over several blocks per query, the RHT butterfly done
+// by one warp with shuffles and the matrix-vector products split over all 256 threads.
 constexpr int kD128 = 128;
 
-__device__ __forceinline__ void stage_matrix128(const void* M, int dtype, unsigned char* dst) {
-    const uint4* src = reinterpret_cast<const uint4*>(M);
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-    if (dtype == TQ_F32) {
-        uint4 v[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) v[r] = __ldg(src + threadIdx.x + r * kThreads);
-#pragma unroll
-        for (int r = 0; r < 16; ++r) d4[threadIdx.x + r * kThreads] = v[r];
-    } else {
-        uint4 v[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) v[r] = __ldg(src + threadIdx.x + r * kThreads);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) d4[threadIdx.x + r * kThreads] = v[r];
-    }
-}
-
-// out[j] = sum_k MT[k][j] in[k] (MT staged row-major 128 x 128); threads (j, half) each sum
+// out[j] = sum_k MT[k][j] in[k] (MT row-major 128 x 128, shared or global); threads (j, half) each sum
 // 64 rows, `part` holds the halves.
 __device__ __forceinline__ void matvec128(const unsigned char* MT, int dtype, const float* in, float* part,
                                           float* out) {
@@ -226,93 +207,21 @@ __device__ void block_encode128(const DevState& st, const void* x, int dtype, co
     __syncthreads();
 }
 
-// Per query (block) the lookup tables of q' = Pi q against the code groups and of u = S q'
-// against the QJL nibbles. APPEND (a decode step that appends one token): the first query
-// head of each group of G also encodes the new K and V vectors of its KV head into row T of
-// that head's planes, before the attention launch that reads them.
-template <int B, bool PROD, bool APPEND>
-__global__ void __launch_bounds__(kThreads)
-tables128_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts,
-                 const DevState vs, const AppendRow app) {
-    using Gr = Groups<B>;
-    using LS = LutShape<kD128, B, PROD>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const size_t mbytes = (size_t)kD128 * kD128 * (st.mat_dtype == TQ_F32 ? 4 : 2);
-    unsigned char* m0 = smem_raw;              // Pi^T (dense rotation)
-    unsigned char* m1 = smem_raw + mbytes;     // S^T
-    float* ctab = reinterpret_cast<float*>(smem_raw + 2 * mbytes);
-    float* qs = ctab + kMaxLevels;
-    float* qp = qs + kD128;
-    float* u = qp + kD128;
-    float* part = u + kD128;                   // 2 x 128
-    const int64_t qi = blockIdx.x;
-    const bool dense = st.rot != TQ_ROT_RHT;
-    if (dense) stage_matrix128(st.piT, st.mat_dtype, m0);
-    if (PROD) stage_matrix128(st.sT, st.mat_dtype, m1);
-    for (int i = threadIdx.x; i < st.L; i += kThreads) ctab[i] = st.c[i];
-    if (threadIdx.x < kD128) {
-        const int i = threadIdx.x;
-        qs[i] = (qdtype == TQ_F32) ? __ldg(reinterpret_cast<const float*>(q) + qi * kD128 + i)
-                                   : bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(q) + qi * kD128 + i));
-    }
-    __syncthreads();
-    if constexpr (APPEND) {
-        if (qi % app.G == 0) {
-            const int64_t g = qi / app.G;   // KV head
-            const size_t es = (app.dtype == TQ_F32) ? 4 : 2;
-            float* buf = part + 2 * kD128;
-            uint8_t* cb = reinterpret_cast<uint8_t*>(buf + 5 * kD128 + 8);
-            const int64_t row = g * app.Tcap;
-            block_encode128(st, reinterpret_cast<const unsigned char*>(app.k_new) + g * kD128 * es, app.dtype, m0, m1,
-                            app.kcodes + row * st.code_bytes, PROD ? app.kqjl + row * st.qjl_bytes : nullptr,
-                            app.knorms + row, PROD ? app.krnorms + row : nullptr, buf, cb);
-            block_encode128(vs, reinterpret_cast<const unsigned char*>(app.v_new) + g * kD128 * es, app.dtype,
-                            reinterpret_cast<const unsigned char*>(vs.piT), reinterpret_cast<const unsigned char*>(vs.sT),
-                            app.vcodes + row * vs.code_bytes,
-                            vs.mode == TQ_PROD ? app.vqjl + row * vs.qjl_bytes : nullptr, app.vnorms + row,
-                            vs.mode == TQ_PROD ? app.vrnorms + row : nullptr, buf, cb);
-        }
-    }
-    if (dense) {
-        matvec128(m0, st.mat_dtype, qs, part, qp);
-    } else {
-        if (threadIdx.x < 32) warp_rht128(st, qs, qp);
-        __syncthreads();
-    }
-    if (PROD) matvec128(m1, st.mat_dtype, qp, part, u);
-    float* out = luts + qi * LS::SIZE;
-    for (int i = threadIdx.x; i < LS::MSE; i += kThreads) {
-        const int k = i / Gr::E, e = i % Gr::E;
-        float a = 0.f;
-#pragma unroll
-        for (int c = 0; c < Gr::CPG; ++c)
-            a = fmaf(qp[k * Gr::CPG + c], ctab[(e >> (B * c)) & ((1 << B) - 1)], a);
-        out[i] = a;
-    }
-    if constexpr (PROD) {
-        for (int i = threadIdx.x; i < LS::QJL; i += kThreads) {
-            const int k = i / 16, e = i % 16;
-            float a = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float v = u[4 * k + c];
-                a += ((e >> c) & 1) ? v : -v;
-            }
-            out[LS::MSE + i] = a;
-        }
-    }
-}
-
-// The same tables without an append, split over kParts blocks per query (grid count x kParts):
-// block p writes the quarter p of the code-group tables and the QJL tables of nibbles
-// 8p .. 8p + 7, so it needs all of q' but only u_j for j in [32p, 32p + 32). The matrices are
-// read from L2 (no staging): q' = Pi q by the whole block (or the Hadamard transform by one
-// warp), u_j = sum_k S^T[k][j] q'_k by 8 threads per output.
+// Per query the lookup tables of q' = Pi q against the code groups and of u = S q' against the
+// QJL nibbles, split over kParts blocks (grid count x kParts): block p writes the quarter p of
+// the code-group tables and the QJL tables of nibbles 8p .. 8p + 7, so it needs all of q' but
+// only u_j for j in [32p, 32p + 32). The matrices are read from L2 (no staging): q' = Pi q by
+// the whole block (or the Hadamard transform by one warp), u_j = sum_k S^T[k][j] q'_k by 8
+// threads per output. APPEND (a decode step that appends one token): one more block per query
+// (blockIdx.y == kParts) in which the first query head of each group of G encodes the new K and
+// V vectors of its KV head into row T of that head's planes, before the attention launch that
+// reads them.
 constexpr int kParts = 4;
 
-template <int B, bool PROD>
+template <int B, bool PROD, bool APPEND>
 __global__ void __launch_bounds__(kThreads)
-tables128_part_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts) {
+tables128_part_kernel(const DevState st, const void* __restrict__ q, int qdtype, float* __restrict__ luts,
+                      const DevState vs, const AppendRow app) {
     using Gr = Groups<B>;
     using LS = LutShape<kD128, B, PROD>;
     static_assert(LS::NG % kParts == 0 && LS::NQ % kParts == 0, "whole tables per part");
@@ -321,6 +230,28 @@ tables128_part_kernel(const DevState st, const void* __restrict__ q, int qdtype,
     __shared__ float upart[8][kD128 / kParts];
     const int64_t qi = blockIdx.x;
     const int pt = blockIdx.y;
+    if constexpr (APPEND) {
+        if (pt == kParts) {
+            if (qi % app.G == 0) {
+                __shared__ __align__(16) float ebuf[5 * kD128 + 8];
+                __shared__ uint8_t ecb[kD128];
+                const int64_t g = qi / app.G;   // KV head
+                const size_t es = (app.dtype == TQ_F32) ? 4 : 2;
+                const int64_t row = g * app.Tcap;
+                block_encode128(st, reinterpret_cast<const unsigned char*>(app.k_new) + g * kD128 * es, app.dtype,
+                                reinterpret_cast<const unsigned char*>(st.piT),
+                                reinterpret_cast<const unsigned char*>(st.sT), app.kcodes + row * st.code_bytes,
+                                PROD ? app.kqjl + row * st.qjl_bytes : nullptr, app.knorms + row,
+                                PROD ? app.krnorms + row : nullptr, ebuf, ecb);
+                block_encode128(vs, reinterpret_cast<const unsigned char*>(app.v_new) + g * kD128 * es, app.dtype,
+                                reinterpret_cast<const unsigned char*>(vs.piT),
+                                reinterpret_cast<const unsigned char*>(vs.sT), app.vcodes + row * vs.code_bytes,
+                                vs.mode == TQ_PROD ? app.vqjl + row * vs.qjl_bytes : nullptr, app.vnorms + row,
+                                vs.mode == TQ_PROD ? app.vrnorms + row : nullptr, ebuf, ecb);
+            }
+            return;
+        }
+    }
     if (threadIdx.x < 16) ctab[threadIdx.x] = (threadIdx.x < st.L) ? st.c[threadIdx.x] : 0.f;
     if (threadIdx.x < kD128) {
         const int i = threadIdx.x;
@@ -384,21 +315,14 @@ tables128_part_kernel(const DevState st, const void* __restrict__ q, int qdtype,
     }
 }
 
-// Shared memory of tables128_kernel: the two staged matrices, the level table, q, q', u and
-// the matrix-vector halves, then (appending) the block encoder's buffers.
-size_t tables128_smem(const DevState& st, bool append) {
-    const size_t mbytes = (size_t)kD128 * kD128 * (st.mat_dtype == TQ_F32 ? 4 : 2);
-    const size_t base = 2 * mbytes + (size_t)(kMaxLevels + 5 * kD128) * sizeof(float);
-    return append ? base + (5 * kD128 + 8) * sizeof(float) + kD128 : base;
-}
-
 // Tables of `count` queries (rows of q) into luts[count][SIZE].
 template <int D, int B, bool PROD>
 int launch_tables(const DevState& st, const void* q, int qdtype, int64_t count, float* luts, cudaStream_t s) {
     if (count <= 0) return 0;
     if (count > (1ll << 31) - 1) return (int)cudaErrorInvalidConfiguration;
     if constexpr (D == kD128) {
-        tables128_part_kernel<B, PROD><<<dim3((unsigned)count, kParts), kThreads, 0, s>>>(st, q, qdtype, luts);
+        tables128_part_kernel<B, PROD, false><<<dim3((unsigned)count, kParts), kThreads, 0, s>>>(st, q, qdtype, luts,
+                                                                                               st, AppendRow{});
     } else {
         auto k = score_prep_kernel<D, B, PROD>;
         const size_t smem = (size_t)(kMaxLevels + 3 * D) * sizeof(float) + kPrepStageBytes;
@@ -634,13 +558,8 @@ namespace {
 template <int B, bool PROD>
 int launch_append_tables(const DevState& ks, const DevState& vs, const void* q, int qdtype, int64_t count,
                          float* luts, const AppendRow& app, cudaStream_t s) {
-    auto k = tables128_kernel<B, PROD, true>;
-    const size_t smem = tables128_smem(ks, true);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return (int)e;
-    }
-    k<<<(unsigned)count, kThreads, smem, s>>>(ks, q, qdtype, luts, vs, app);
+    tables128_part_kernel<B, PROD, true><<<dim3((unsigned)count, kParts + 1), kThreads, 0, s>>>(ks, q, qdtype, luts,
+                                                                                              vs, app);
     return (int)cudaGetLastError();
 }
 
