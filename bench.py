@@ -429,17 +429,18 @@ def measure_c5(tq, torch, dev, stream, steps: int, warmup: int, tflops_peak: flo
                 fn()
             torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = max(2, min(steps, 5))
-            e0.record(stream)
-            for _ in range(reps):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
+            reps = max(2, min(steps, 20))   # a few hundred ms, so the clock record has samples
+            with ClockSampler(dev.index) as clk:
+                e0.record(stream)
+                for _ in range(reps):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
             ms = e0.elapsed_time(e1) / reps
             tf = flops / (ms / 1e3) / 1e12
-            out[name] = {"ms": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": tflops_peak,
-                                                "unit": "TFLOP/s", "frac": tf / tflops_peak,
-                                                "algorithmic_flops_per_launch": flops}}
+            out[name] = {"ms": ms, "reps": reps, "clocks": clk.summary(),
+                         "roofline": {"bound": "tensor", "achieved": tf, "peak": tflops_peak, "unit": "TFLOP/s",
+                                      "frac": tf / tflops_peak, "algorithmic_flops_per_launch": flops}}
         out["encode"]["mvec_s"] = C5_N / (out["encode"]["ms"] / 1e3) / 1e6
         st.close()
         res["dense" if rot == tq.ROT_DENSE else "rht"] = out
