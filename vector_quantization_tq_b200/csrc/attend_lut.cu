@@ -79,12 +79,16 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     constexpr int NQ = kD / 4;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     constexpr int LSIZE = KG::NG * KG::E + (KPROD ? NQ * 16 : 0);   // floats of one query's tables
-    TB* tb = reinterpret_cast<TB*>(smem_raw);                    // 2 stages
-    float* vc = reinterpret_cast<float*>(tb + 2);               // 32 (V centroids)
+    // Four query heads per block: one tile buffer, and the warps' value sums laid over it at
+    // the end, so that two blocks fit on an SM (16 warps to hide the table lookups' latency);
+    // otherwise two tile buffers, the next tile staged while this one is processed.
+    constexpr int kBufs = (QH == 4) ? 1 : 2;
+    TB* tb = reinterpret_cast<TB*>(smem_raw);
+    float* vc = reinterpret_cast<float*>(tb + kBufs);           // 32 (V centroids)
     float* tm = vc + 32;                                         // QH x LSIZE: head qh's tables at qh * LSIZE
     float* wt = tm + QH * LSIZE;                                 // QH x kThreads
     float* red = wt + QH * kThreads;                             // QH x 32
-    float* accw = red + QH * 32;                                 // kWarps x QH x kD
+    float* accw = (kBufs == 1) ? reinterpret_cast<float*>(tb) : red + QH * 32;   // kWarps x QH x kD
 
     const int h0 = blockIdx.y * QH;   // the block's first query head
     const int split = blockIdx.x;
@@ -118,7 +122,7 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     // per head by the table launch and consecutive in `luts`, arrive with the first tile
     for (int i = threadIdx.x; i < QH * LSIZE / 4; i += kThreads)
         cp_async16(tm + 4 * i, luts + (int64_t)h0 * LSIZE + 4 * i);
-    if (t_begin < t_end) stage_tile(0, t_begin);
+    if (kBufs == 2 && t_begin < t_end) stage_tile(0, t_begin);
     cp_async_commit();
     if (threadIdx.x < 32) vc[threadIdx.x] = (threadIdx.x < vs.L) ? vs.c[threadIdx.x] : 0.f;
 
@@ -137,10 +141,16 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
     int it = 0;
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kThreads, ++it) {
         const int cnt = (int)((t_end - t0) < kThreads ? (t_end - t0) : kThreads);
-        const int sb = it & 1;
-        if (t0 + kThreads < t_end) stage_tile(sb ^ 1, t0 + kThreads);   // prefetch the next tile
-        cp_async_commit();
-        cp_async_wait1();
+        const int sb = (kBufs == 2) ? (it & 1) : 0;
+        if constexpr (kBufs == 2) {
+            if (t0 + kThreads < t_end) stage_tile(sb ^ 1, t0 + kThreads);   // prefetch the next tile
+            cp_async_commit();
+            cp_async_wait1();
+        } else {
+            stage_tile(0, t0);
+            cp_async_commit();
+            cp_async_wait0();
+        }
         __syncthreads();
         const TB& B = tb[sb];
         // ---- A: scores of token t0 + threadIdx.x against the QH heads ----
@@ -367,9 +377,12 @@ attend_lut_kernel(const DevState ks, const DevState vs, const float* __restrict_
 template <int BK, bool KPROD, int BV, int QH>
 size_t smem_bytes() {
     using KG = KGroups<BK>;
-    return 2 * sizeof(TileBuf<BK, KPROD, BV>) +
+    constexpr int kBufs = (QH == 4) ? 1 : 2;   // as in the kernel
+    static_assert(kBufs == 2 || sizeof(TileBuf<BK, KPROD, BV>) >= sizeof(float) * kWarps * QH * kD,
+                  "the value sums fit over the tile buffer");
+    return kBufs * sizeof(TileBuf<BK, KPROD, BV>) +
            (size_t)(32 + QH * (KG::NG * KG::E + (KPROD ? (kD / 4) * 16 : 0)) + QH * kThreads + QH * 32 +
-                    kWarps * QH * kD) *
+                    (kBufs == 2 ? kWarps * QH * kD : 0)) *
                sizeof(float);
 }
 
