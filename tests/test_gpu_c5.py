@@ -6,7 +6,7 @@ call. The oracle then re-encodes the whole database block by block: every block'
 checked under the band rule, and the estimates of all 1000 queries against all 10^6 keys give
 the oracle's own top-10 of every query, which the library's top-10 must match (a swap at the
 cut counts as a match when the two estimates are within the score tolerance; a key whose
-planes differ from the oracle's in-band is judged by the oracle's estimate from the library's
+planes differ from the oracle's in-band is checked against the oracle's estimate from the library's
 planes).
 """
 import numpy as np
